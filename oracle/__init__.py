@@ -1,0 +1,186 @@
+"""fp64 CPU oracle for the spatial-temporal block-sparse attention path.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product package never imports
+this module, and this module never imports the product package.
+
+The arithmetic lives in ``vsa_oracle.c`` (plain C, fp64, OpenMP over rows); this file
+only marshals numpy arrays in and out and converts the oracle's boolean block masks into
+the list and bitset formats the GPU library emits, so that the two can be compared.
+Each function names the passage of the pages it follows in the C source.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+SPATIAL, TEMPORAL, CUBE = 0, 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC", "-ffp-contract=off",
+               _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        i64, dbl, vp = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+        lib.or_num_cubes.restype = i64
+        lib.or_num_cubes.argtypes = [i64] * 6
+        lib.or_layout_rows.restype = i64
+        lib.or_layout_rows.argtypes = [ctypes.c_int] + [i64] * 6
+        lib.or_layout_slots.restype = None
+        lib.or_layout_slots.argtypes = [ctypes.c_int] + [i64] * 6 + [vp]
+        lib.or_pattern_keep.restype = None
+        lib.or_pattern_keep.argtypes = [ctypes.c_int] + [i64] * 5 + [vp]
+        lib.or_kept_fraction.restype = dbl
+        lib.or_kept_fraction.argtypes = [ctypes.c_int] + [i64] * 5
+        lib.or_window_for_target.restype = i64
+        lib.or_window_for_target.argtypes = [ctypes.c_int] + [i64] * 4 + [dbl]
+        lib.or_cube_topk_keep.restype = ctypes.c_int
+        lib.or_cube_topk_keep.argtypes = [vp, vp] + [i64] * 8 + [vp, vp]
+        lib.or_attention_rows.restype = None
+        lib.or_attention_rows.argtypes = [vp, vp, vp, i64, i64, dbl, vp, i64, vp, i64, vp, i64, vp, vp]
+        lib.or_profile_rows.restype = i64
+        lib.or_profile_rows.argtypes = [i64, dbl]
+        lib.or_profile_head.restype = ctypes.c_int
+        lib.or_profile_head.argtypes = [vp, vp, vp] + [i64] * 4 + [dbl] + [i64] * 3 + [dbl, vp, vp]
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(x) -> np.ndarray:
+    """Widen a torch tensor or array to a C-contiguous fp64 numpy array."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def num_cubes(F, Hl, Wl, cube=(4, 4, 8)) -> int:
+    return int(_load().or_num_cubes(F, Hl, Wl, *cube))
+
+
+def layout_rows(kind, F, Hl, Wl, cube=(4, 4, 8)) -> int:
+    return int(_load().or_layout_rows(kind, F, Hl, Wl, *cube))
+
+
+def layout_slots(kind, F, Hl, Wl, cube=(4, 4, 8)) -> np.ndarray:
+    """Slot of every natural token under a head's layout (int64 [N])."""
+    out = np.empty(F * Hl * Wl, dtype=np.int64)
+    _load().or_layout_slots(kind, F, Hl, Wl, *cube, _p(out))
+    return out
+
+
+def pattern_keep(kind, F, Hl, Wl, block, w) -> np.ndarray:
+    """Boolean block mask [nblk, nblk] of a spatial or temporal head with window w."""
+    nb = -(-(F * Hl * Wl) // block)
+    out = np.empty((nb, nb), dtype=np.uint8)
+    _load().or_pattern_keep(kind, F, Hl, Wl, block, w, _p(out))
+    return out.astype(bool)
+
+
+def kept_fraction(kind, F, Hl, Wl, block, w) -> float:
+    return float(_load().or_kept_fraction(kind, F, Hl, Wl, block, w))
+
+
+def window_for_target(kind, F, Hl, Wl, block, target) -> int:
+    return int(_load().or_window_for_target(kind, F, Hl, Wl, block, float(target)))
+
+
+def cube_topk_keep(q, k, F, Hl, Wl, topk, cube=(4, 4, 8), return_scores=False):
+    """Cube mask [C, C] from pooled-QK^T top-k (one head, natural-order q, k [N, d])."""
+    q, k = _f64(q), _f64(k)
+    d = q.shape[-1]
+    C = num_cubes(F, Hl, Wl, cube)
+    keep = np.empty((C, C), dtype=np.uint8)
+    score = np.empty((C, C), dtype=np.float64)
+    rc = _load().or_cube_topk_keep(_p(q), _p(k), F, Hl, Wl, d, *cube, topk, _p(keep), _p(score))
+    if rc != 0:
+        raise MemoryError("oracle cube top-k allocation failed")
+    return (keep.astype(bool), score) if return_scores else keep.astype(bool)
+
+
+def attention_rows(q, k, v, slots, block, keep, rows=None, scale=None):
+    """Masked softmax attention on natural-order rows of one head.
+
+    Returns (out [len(rows), d] fp64, lse [len(rows)] fp64, natural log).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    slots = np.ascontiguousarray(slots, dtype=np.int64)
+    keep8 = np.ascontiguousarray(keep, dtype=np.uint8)
+    nb = keep8.shape[0]
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((len(rows), d), dtype=np.float64)
+    lse = np.empty(len(rows), dtype=np.float64)
+    _load().or_attention_rows(_p(q), _p(k), _p(v), N, d, scale, _p(slots), block, _p(keep8), nb,
+                              _p(rows), len(rows), _p(out), _p(lse))
+    return out, lse
+
+
+def profile_rows(N, frac) -> int:
+    return int(_load().or_profile_rows(N, float(frac)))
+
+
+def profile_head(q, k, v, F, Hl, Wl, block, w_s, w_t, frac=0.01, scale=None):
+    """Profile one head: returns (kind, mse[2] = (spatial, temporal), sampled rows)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    r = profile_rows(N, frac)
+    mse = np.empty(2, dtype=np.float64)
+    rows = np.empty(r, dtype=np.int64)
+    kind = _load().or_profile_head(_p(q), _p(k), _p(v), F, Hl, Wl, d, scale, block, w_s, w_t, float(frac),
+                                   _p(mse), _p(rows))
+    if kind < 0:
+        raise MemoryError("oracle profiling allocation failed")
+    return int(kind), mse, rows
+
+
+# ---------------------------------------------------------------------------------------
+# Format conversion of an oracle mask into the GPU library's output formats.
+# ---------------------------------------------------------------------------------------
+
+def keep_to_lists(keep: np.ndarray, max_kv: int):
+    """Ascending kept-column list per row, padded with -1, and the per-row count."""
+    nq = keep.shape[0]
+    idx = np.full((nq, max_kv), -1, dtype=np.int32)
+    cnt = np.zeros(nq, dtype=np.int32)
+    for i in range(nq):
+        cols = np.nonzero(keep[i])[0]
+        cnt[i] = len(cols)
+        idx[i, :min(len(cols), max_kv)] = cols[:max_kv]
+    return idx, cnt
+
+
+def keep_to_bits(keep: np.ndarray) -> np.ndarray:
+    """Bitset [nq, ceil(nk/32)] uint32, bit (j % 32) of word j // 32 set when kept."""
+    nq, nk = keep.shape
+    nw = -(-nk // 32)
+    padded = np.zeros((nq, nw * 32), dtype=np.uint64)
+    padded[:, :nk] = keep
+    weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
+    words = (padded.reshape(nq, nw, 32) * weights).sum(axis=2)
+    return words.astype(np.uint32)
