@@ -1,0 +1,112 @@
+"""Spatial-temporal block-sparse self-attention for video diffusion transformers on B200.
+
+The compute lives in ``libvsa.so`` (hand-written CUDA for sm_100a behind the C ABI in
+``include/vsa.h``).  This package is its thin Python binding: ``_lib`` mirrors each C entry
+point under the same name, and :class:`SparseAttention` owns the device buffers (from
+PyTorch) of one configured call and invokes ``vsa_attention``.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (VSA_BF16, VSA_CUBE, VSA_F32, VSA_SELECT_CUBE, VSA_SELECT_GIVEN, VSA_SELECT_PROFILE, VSA_SPATIAL,
+                   VSA_TEMPORAL, Params, QKVO, Shape, VsaError, make_params, make_shape, qkvo, vsa_attention,
+                   vsa_attention_workspace_layout, vsa_attention_workspace_size, vsa_build_mask,
+                   vsa_get_device_error, vsa_layout_rows, vsa_mask_workspace_size, vsa_max_kv, vsa_num_blocks,
+                   vsa_pattern_window, vsa_permute, vsa_profile_heads, vsa_profile_rows, vsa_profile_workspace_size,
+                   vsa_sparse_attn_fwd, vsa_unpermute)
+
+_SELECT = {"profile": VSA_SELECT_PROFILE, "given": VSA_SELECT_GIVEN, "cube": VSA_SELECT_CUBE}
+_DTYPE = {torch.float32: VSA_F32, torch.bfloat16: VSA_BF16}
+
+
+class SparseAttention:
+    """One configured attention call over a B x H x (F x Hl x Wl) x d problem.
+
+    select:  "profile" (heads pick spatial/temporal by online profiling), "given" (kinds
+             passed per call) or "cube" (own cube + top-k pooled cubes for every head).
+    Windows: pass ``w_s``/``w_t`` directly, or ``target`` (a kept-block fraction) to use the
+             smallest windows reaching it.
+    """
+
+    def __init__(self, B: int, H: int, F: int, Hl: int, Wl: int, d: int, block: int = 128, *,
+                 dtype: torch.dtype = torch.bfloat16, select: str = "profile", w_s: Optional[int] = None,
+                 w_t: Optional[int] = None, target: Optional[float] = None, topk: int = 0,
+                 cube: Optional[Sequence[int]] = None, profile_frac: float = 0.01, scale: float = 0.0,
+                 with_lse: bool = False, device="cuda"):
+        if dtype not in _DTYPE:
+            raise ValueError(f"unsupported dtype {dtype}")
+        self.B, self.H, self.F, self.Hl, self.Wl, self.d, self.block = B, H, F, Hl, Wl, d, block
+        self.N = F * Hl * Wl
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.dtype, self.select, self.device = dtype, _SELECT[select], dev
+        self.shape = make_shape(B, H, F, Hl, Wl, d, block, tuple(cube) if cube else None)
+        if target is not None:
+            w_s_t, self.kept_s = vsa_pattern_window(self.shape, VSA_SPATIAL, target)
+            w_t_t, self.kept_t = vsa_pattern_window(self.shape, VSA_TEMPORAL, target)
+            w_s = w_s_t if w_s is None else w_s
+            w_t = w_t_t if w_t is None else w_t
+        self.w_s, self.w_t = int(w_s or 0), int(w_t or 0)
+        self.params = make_params(self.w_s, self.w_t, profile_frac, topk, scale)
+        self.ws_bytes = vsa_attention_workspace_size(self.shape, self.params, _DTYPE[dtype], self.select)
+        if self.ws_bytes == 0:
+            raise VsaError(_lib.VSA_ERR_INVALID_ARG, "vsa_attention_workspace_size")
+        off_bits, off_idx, off_cnt, self.max_kv = vsa_attention_workspace_layout(self.shape, self.params,
+                                                                                 _DTYPE[dtype], self.select)
+        self.nblk = vsa_num_blocks(self.shape)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        nwords = (self.nblk + 31) // 32
+        rows = B * H * self.nblk
+        self.bits = self.ws[off_bits:off_bits + rows * nwords * 4].view(torch.int32).view(B, H, self.nblk, nwords)
+        self.kv_idx = self.ws[off_idx:off_idx + rows * self.max_kv * 4].view(torch.int32).view(B, H, self.nblk,
+                                                                                               self.max_kv)
+        self.kv_cnt = self.ws[off_cnt:off_cnt + rows * 4].view(torch.int32).view(B, H, self.nblk)
+        self.kinds = torch.zeros(B * H, dtype=torch.uint8, device=self.device)
+        self.mse = torch.zeros(B * H * 2, dtype=torch.float32, device=self.device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.with_lse = with_lse
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, kinds: Optional[torch.Tensor] = None, stream=None):
+        for t in (q, k, v):
+            if t.dtype != self.dtype or t.device != self.device or not t.is_contiguous():
+                raise ValueError("q, k, v must be contiguous tensors of the configured dtype and device")
+            if tuple(t.shape) != (self.B, self.H, self.N, self.d):
+                raise ValueError(f"expected shape {(self.B, self.H, self.N, self.d)}, got {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty_like(q)
+        if self.with_lse and lse is None:
+            lse = torch.empty(self.B, self.H, self.N, dtype=torch.float32, device=self.device)
+        if self.select == VSA_SELECT_GIVEN:
+            if kinds is None:
+                raise ValueError("select='given' needs kinds")
+            self.kinds.copy_(kinds.reshape(-1).to(torch.uint8))
+        vsa_attention(qkvo(q, k, v, out, lse), _DTYPE[self.dtype], self.shape, self.params, self.select, self.kinds,
+                      self.mse, self.ws, self.ws_bytes, self.err, stream)
+        return (out, lse) if self.with_lse else out
+
+    def device_error(self) -> int:
+        return vsa_get_device_error(self.err)
+
+    def clear_error(self):
+        self.err.zero_()
+
+
+def attention(q, k, v, F: int, Hl: int, Wl: int, **kw):
+    """Convenience wrapper: build a :class:`SparseAttention` for q's shape and run it once."""
+    B, H, N, d = q.shape
+    plan = SparseAttention(B, H, F, Hl, Wl, d, dtype=q.dtype, device=q.device, **kw)
+    return plan(q, k, v)
+
+
+__all__ = ["SparseAttention", "attention", "VsaError", "Shape", "Params", "QKVO", "make_shape", "make_params", "qkvo",
+           "vsa_attention", "vsa_attention_workspace_layout", "vsa_attention_workspace_size", "vsa_build_mask",
+           "vsa_get_device_error", "vsa_layout_rows", "vsa_mask_workspace_size", "vsa_max_kv", "vsa_num_blocks",
+           "vsa_pattern_window", "vsa_permute", "vsa_profile_heads", "vsa_profile_rows",
+           "vsa_profile_workspace_size", "vsa_sparse_attn_fwd", "vsa_unpermute", "VSA_SPATIAL", "VSA_TEMPORAL",
+           "VSA_CUBE", "VSA_F32", "VSA_BF16", "VSA_SELECT_PROFILE", "VSA_SELECT_GIVEN", "VSA_SELECT_CUBE"]

@@ -1,0 +1,64 @@
+// kernels.h -- host-side launchers of the libvsa kernels (internal to the library).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace vsa {
+
+cudaError_t launch_permute(const void* src, bool src_f32, void* dst, const uint8_t* kinds, const Geom& g, int BH,
+                           int d, int* err, cudaStream_t stream);
+cudaError_t launch_unpermute(const void* src, const float* src_lse, void* dst, bool dst_f32, float* dst_lse,
+                             const uint8_t* kinds, const Geom& g, int BH, int d, int* err, cudaStream_t stream);
+
+cudaError_t launch_pattern_mask(const uint8_t* kinds, const Geom& g, int BH, int w_s, int w_t, uint32_t* bits,
+                                int32_t* kv_idx, int32_t* kv_cnt, int max_kv, int* err, cudaStream_t stream);
+// Workspace: 2 * BH * ncubes * d doubles.
+size_t cube_mask_workspace_bytes(const Geom& g, int BH, int d);
+cudaError_t launch_cube_mask(const uint8_t* kinds, const void* q_cube, const void* k_cube, const Geom& g, int BH, int d,
+                             int topk, uint32_t* bits, int32_t* kv_idx, int32_t* kv_cnt, int max_kv, void* ws,
+                             int* err, cudaStream_t stream);
+
+// Tensor maps of one attention problem (3D: d, rows, B*H).
+struct AttnMaps {
+  CUtensorMap q, k, v, o;
+};
+
+struct AttnArgs {
+  const uint8_t* kinds;
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  float* lse_nat;
+  float* lse_perm;
+  int* err;
+  int BH;
+  int max_kv;
+  int has_perm;
+  int nat_rows;  // rows per head of the natural buffers (N, or R when they hold every layout)
+  float scale_log2;
+  Geom g;
+};
+
+cudaError_t launch_sparse_attn(const AttnMaps& nat, const AttnMaps& perm, const AttnArgs& a, int d,
+                               cudaStream_t stream);
+
+// Profiling (see profile.cu).
+struct ProfilePlan {
+  int r;        // sampled rows
+  int r_pad;    // rounded up to the 128-row tile
+  int tiles;    // r_pad / 128
+  int splits;   // key-range splits per tile
+  size_t off_qs, off_ranges, off_opart, off_ml, bytes;
+};
+ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac);
+cudaError_t launch_profile(const void* q, const void* k, const void* v, const Geom& g, int BH, int d, int w_s,
+                           int w_t, float scale_log2, const ProfilePlan& plan, void* ws, uint8_t* kinds_out,
+                           float* mse_out, int* err, cudaStream_t stream);
+
+// Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
+cudaError_t encode_rows_map(CUtensorMap* map, const void* base, int d, int rows, int BH, int box_rows);
+
+}  // namespace vsa

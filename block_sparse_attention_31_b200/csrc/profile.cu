@@ -1,0 +1,503 @@
+// profile.cu -- online head profiling (vsa_profile_heads).
+//
+// "Sparse Video-Gen" summary page, "Approach": a profiling step on about 1% of the query
+// rows picks, per head, the pattern (spatial or temporal) with the lower error; its
+// "Measured effects" table reports 1% as the profiled share.  Reading used here: the
+// sampled rows are rho_i = floor((2i+1)N/(2r)), r = ceil(frac*N); the error of a pattern
+// is the mean squared difference between its output and dense attention over those rows
+// and all d outputs, under the block masks that the attention kernel would execute;
+// ties pick the spatial pattern.
+//
+// Three kernels:
+//   prep     gathers the sampled Q rows of every head into a 128-row-padded tile buffer
+//            and, per sampled row, the contiguous key range each pattern allows (spatial:
+//            a natural-order token range; temporal: a frame-major slot range);
+//   attn3    one CTA per (head, 128-row tile, key split): S = Q K^T on tcgen05 into TMEM,
+//            then three online softmaxes (dense, spatial-masked, temporal-masked) sharing
+//            that S, and three P V products into three TMEM accumulators; writes the
+//            partial (max, sum, unnormalised O) of each variant;
+//   reduce   one CTA per head: merges the splits, forms the three outputs, accumulates the
+//            two squared errors in fp64 in a fixed order and picks the kind.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace vsa {
+
+constexpr int kProfThreads = 192;
+constexpr int kPM = 128;  // rows per tile
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
+  ProfilePlan p{};
+  long long r = static_cast<long long>(ceil(frac * static_cast<double>(g.N)));
+  if (r < 1) r = 1;
+  if (r > g.N) r = g.N;
+  p.r = static_cast<int>(r);
+  p.r_pad = (p.r + kPM - 1) / kPM * kPM;
+  p.tiles = p.r_pad / kPM;
+  const int nb = (g.N + g.block - 1) / g.block;
+  const long long ctas = static_cast<long long>(BH) * p.tiles;
+  int splits = static_cast<int>((2 * 148 + ctas - 1) / ctas);
+  if (splits < 1) splits = 1;
+  if (splits > nb) splits = nb;
+  p.splits = splits;
+  size_t off = 0;
+  p.off_qs = off;
+  off = align256(off + static_cast<size_t>(BH) * p.r_pad * d * 2);
+  p.off_ranges = off;
+  off = align256(off + static_cast<size_t>(p.r_pad) * 4 * sizeof(int));
+  p.off_opart = off;
+  off = align256(off + static_cast<size_t>(BH) * splits * 3 * p.r_pad * d * sizeof(float));
+  p.off_ml = off;
+  off = align256(off + static_cast<size_t>(BH) * splits * 3 * p.r_pad * 2 * sizeof(float));
+  p.bytes = off;
+  return p;
+}
+
+// Contiguous range [lo, hi] of key blocks kept for query block i, groups of G slots.
+__device__ __forceinline__ void kept_block_range(int i, int N, int B, int G, int w, int& lo, int& hi) {
+  const int nb = (N + B - 1) / B;
+  const int ai = (i * B) / G, bi = (min(N, (i + 1) * B) - 1) / G;
+  lo = nb;
+  hi = -1;
+  for (int j = 0; j < nb; ++j) {
+    const int aj = (j * B) / G, bj = (min(N, (j + 1) * B) - 1) / G;
+    if (max(0, max(aj - bi, ai - bj)) <= w) {
+      lo = min(lo, j);
+      hi = j;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) profile_prep_kernel(const __nv_bfloat16* __restrict__ q, Geom g, int d, int r,
+                                                           int r_pad, int w_s, int w_t,
+                                                           __nv_bfloat16* __restrict__ qs, int4* __restrict__ ranges) {
+  const int bh = blockIdx.y;
+  const int vpr = d / 8;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = idx / vpr, v = idx - (idx / vpr) * vpr;
+  if (i >= r_pad) return;
+  const long long t = i < r ? (static_cast<long long>(2 * i + 1) * g.N) / (2LL * r) : -1;
+  uint4 val = make_uint4(0, 0, 0, 0);
+  if (t >= 0) val = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<size_t>(bh) * g.N + t) * d + v * 8));
+  *reinterpret_cast<uint4*>(qs + (static_cast<size_t>(bh) * r_pad + i) * d + v * 8) = val;
+  if (bh == 0 && v == 0) {
+    int4 rg = make_int4(0, 0, 0, 0);
+    if (t >= 0) {
+      int lo, hi;
+      kept_block_range(static_cast<int>(t) / g.block, g.N, g.block, g.S, w_s, lo, hi);
+      rg.x = lo * g.block;
+      rg.y = min(g.N, (hi + 1) * g.block);
+      const int p = slot_of_token(g, kTemporal, static_cast<int>(t));
+      kept_block_range(p / g.block, g.N, g.block, g.F, w_t, lo, hi);
+      rg.z = lo * g.block;
+      rg.w = min(g.N, (hi + 1) * g.block);
+    }
+    ranges[i] = rg;
+  }
+}
+
+template <int D, int BN>
+struct ProfCfg {
+  static constexpr int Q_BYTES = kPM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int P_BYTES = kPM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_P = OFF_V + KV_BYTES;  // three P tiles
+  static constexpr int OFF_BAR = OFF_P + 3 * P_BYTES;
+  static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+  static constexpr int BYTES = OFF_MISC + 64;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr int TMEM_S = 0, TMEM_O = BN;
+  static constexpr int TMEM_COLS = (BN + 3 * D) <= 256 ? 256 : 512;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kPM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kPM, D, false, true);
+};
+
+enum { PB_Q = 0, PB_FULL_K, PB_FULL_V, PB_EMPTY_K, PB_EMPTY_V, PB_S_FULL, PB_S_FREE, PB_P_FULL, PB_O_DONE, PB_DRAIN };
+
+struct ProfArgs {
+  const int4* ranges;
+  float* opart;
+  float* ml;
+  int* err;
+  int r_pad, tiles, splits, per_split;
+  float scale_log2;
+  Geom g;
+};
+
+template <int D, int BN>
+__global__ void __launch_bounds__(kProfThreads, 1)
+    profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
+                         const __grid_constant__ CUtensorMap tv, const ProfArgs a) {
+  using C = ProfCfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_u32);
+  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sP = sbase + C::OFF_P;
+  uint8_t* pP = smem + C::OFF_P;
+  auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = misc + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Geom& g = a.g;
+  const int split = blockIdx.x % a.splits;
+  const int tile = (blockIdx.x / a.splits) % a.tiles;
+  const int bh = blockIdx.x / (a.splits * a.tiles);
+  const int nb = (g.N + BN - 1) / BN;
+  const int kb0 = split * a.per_split;
+  const int cnt = max(0, min(nb, kb0 + a.per_split) - kb0);
+  bool stop = false;
+  if (tid == 0) stop = (*reinterpret_cast<volatile int*>(a.err) & kDevErrTimeout) != 0;
+  if (__syncthreads_or(stop)) return;
+
+  if (tid == 0) {
+    mbar_init(bar(PB_Q), 1);
+    mbar_init(bar(PB_FULL_K), 1);
+    mbar_init(bar(PB_FULL_V), 1);
+    mbar_init(bar(PB_EMPTY_K), 1);
+    mbar_init(bar(PB_EMPTY_V), 1);
+    mbar_init(bar(PB_S_FULL), 1);
+    mbar_init(bar(PB_S_FREE), 128);
+    mbar_init(bar(PB_P_FULL), 128);
+    mbar_init(bar(PB_O_DONE), 1);
+    mbar_init(bar(PB_DRAIN), 1);
+    misc[1] = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  if (warp == 0) {
+    if (lane == 0 && cnt > 0) {
+      int nk = 0, nv = 0;
+      mbar_arrive_expect_tx(bar(PB_Q), C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * kPM * 128, &tqs, bar(PB_Q), c * 64, tile * kPM, bh);
+      for (int j = 0; j < cnt; ++j) {
+        const int kb = kb0 + j;
+        if (j >= 1 && !mbar_wait(bar(PB_EMPTY_K), (j - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(PB_FULL_K), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BN * 128, &tk, bar(PB_FULL_K), c * 64, kb * BN, bh);
+        nk = j + 1;
+        if (j >= 1 && !mbar_wait(bar(PB_EMPTY_V), (j - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(PB_FULL_V), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_3d(sV + c * BN * 128, &tv, bar(PB_FULL_V), c * 64, kb * BN, bh);
+        nv = j + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(bar(PB_Q), 0, a.err);
+        if (nk > 0) mbar_wait_drain(bar(PB_FULL_K), (nk - 1) & 1, a.err);
+        if (nv > 0) mbar_wait_drain(bar(PB_FULL_V), (nv - 1) & 1, a.err);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && cnt > 0) {
+      auto issue_pv = [&](int jp) -> bool {
+        if (!mbar_wait(bar(PB_P_FULL), jp & 1, abort_flag, a.err)) return false;
+        if (!mbar_wait(bar(PB_FULL_V), jp & 1, abort_flag, a.err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int vv = 0; vv < 3; ++vv)
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t ad =
+                sdesc_sw128(sP + vv * C::P_BYTES + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sV + kk * 16 * 128, BN * 128, 1024);
+            tc_mma_ss(tmem + C::TMEM_O + vv * D, ad, bd, C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+          }
+        tc_commit(bar(PB_EMPTY_V));
+        tc_commit(bar(PB_O_DONE));
+        return true;
+      };
+      bool ok = mbar_wait(bar(PB_Q), 0, abort_flag, a.err);
+      for (int j = 0; ok && j < cnt; ++j) {
+        if (!mbar_wait(bar(PB_FULL_K), j & 1, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        if (j >= 1 && !mbar_wait(bar(PB_S_FREE), (j - 1) & 1, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+          tc_mma_ss(tmem + C::TMEM_S, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(PB_EMPTY_K));
+        tc_commit(bar(PB_S_FULL));
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) issue_pv(cnt - 1);
+      tc_commit(bar(PB_DRAIN));
+      mbar_wait_drain(bar(PB_DRAIN), 0, a.err);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
+    const int4 rg = a.ranges[tile * kPM + row];
+    float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f};
+    bool ok = true;
+    for (int j = 0; j < cnt; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_S_FULL), j & 1, abort_flag, a.err));
+      if (!ok) break;
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + C::TMEM_S + c * 32, s + c * 32);
+      tc_fence_before();
+      mbar_arrive(bar(PB_S_FREE));
+      // masks of the three variants for this block's key tokens t = kb*BN + c
+      const int t0 = (kb0 + j) * BN;
+      uint32_t mk[3][BN / 32];
+      {
+        int f = t0 / g.S, sp = t0 - (t0 / g.S) * g.S;
+#pragma unroll
+        for (int w = 0; w < BN / 32; ++w) {
+          uint32_t md = 0, ms = 0, mt = 0;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int t = t0 + w * 32 + c;
+            const int p = sp * g.F + f;
+            const bool valid = t < g.N;
+            md |= (valid ? 1u : 0u) << c;
+            ms |= ((valid && t >= rg.x && t < rg.y) ? 1u : 0u) << c;
+            mt |= ((valid && p >= rg.z && p < rg.w) ? 1u : 0u) << c;
+            if (++sp == g.S) {
+              sp = 0;
+              ++f;
+            }
+          }
+          mk[0][w] = md;
+          mk[1][w] = ms;
+          mk[2][w] = mt;
+        }
+      }
+      float mnew[3], muse[3];
+#pragma unroll
+      for (int vv = 0; vv < 3; ++vv) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if ((mk[vv][c >> 5] >> (c & 31)) & 1u) mx = fmaxf(mx, s[c]);
+        mnew[vv] = fmaxf(m[vv], mx * sl2);
+        muse[vv] = mnew[vv] == -INFINITY ? 0.f : mnew[vv];
+      }
+      if (j >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (j - 1) & 1, abort_flag, a.err));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int vv = 0; vv < 3; ++vv) {
+          const float alpha = fast_exp2(m[vv] - muse[vv]);
+          if (__any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              float o[32];
+              tmem_ld32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+#pragma unroll
+              for (int x = 0; x < 32; ++x) o[x] *= alpha;
+              tmem_st32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+            }
+          }
+          l[vv] *= alpha;
+        }
+      }
+#pragma unroll
+      for (int vv = 0; vv < 3; ++vv) {
+        float rs = 0.f;
+        uint8_t* pv = pP + vv * C::P_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < BN / 8; ++ch) {
+          float p[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const int c = ch * 8 + x;
+            p[x] = ((mk[vv][c >> 5] >> (c & 31)) & 1u) ? fast_exp2(fmaf(s[c], sl2, -muse[vv])) : 0.f;
+            rs += p[x];
+          }
+          uint4 pk;
+          pk.x = pack_bf16x2(p[0], p[1]);
+          pk.y = pack_bf16x2(p[2], p[3]);
+          pk.z = pack_bf16x2(p[4], p[5]);
+          pk.w = pack_bf16x2(p[6], p[7]);
+          const int kc = ch >> 3, cc = ch & 7;
+          *reinterpret_cast<uint4*>(pv + kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = pk;
+        }
+        l[vv] += rs;
+        m[vv] = mnew[vv];
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(PB_P_FULL));
+    }
+    if (ok && cnt > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
+      tc_fence_after();
+    }
+    // partials: (m, l) and unnormalised O of each variant
+    const size_t base = ((static_cast<size_t>(bh) * a.splits + split) * 3) * a.r_pad + tile * kPM + row;
+#pragma unroll
+    for (int vv = 0; vv < 3; ++vv) {
+      const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
+      const bool have = ok && cnt > 0;
+      a.ml[prow * 2 + 0] = have ? m[vv] : -INFINITY;
+      a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
+      float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (have) {
+          tmem_ld32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = 0.f;
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) dst[c * 8 + x] = make_float4(o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+constexpr int kRedThreads = 256;
+
+__global__ void __launch_bounds__(kRedThreads) profile_reduce_kernel(const float* __restrict__ opart,
+                                                                     const float* __restrict__ ml, int r, int r_pad,
+                                                                     int splits, int d, uint8_t* __restrict__ kinds,
+                                                                     float* __restrict__ mse) {
+  __shared__ double red[2][kRedThreads];
+  const int bh = blockIdx.x;
+  double es = 0.0, et = 0.0;
+  for (int idx = threadIdx.x; idx < r * d; idx += kRedThreads) {
+    const int i = idx / d, x = idx - (idx / d) * d;
+    float o[3];
+#pragma unroll
+    for (int vv = 0; vv < 3; ++vv) {
+      float M = -INFINITY;
+      for (int sp = 0; sp < splits; ++sp) {
+        const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
+        M = fmaxf(M, ml[prow * 2]);
+      }
+      float L = 0.f, acc = 0.f;
+      for (int sp = 0; sp < splits; ++sp) {
+        const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
+        const float ms = ml[prow * 2];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        L += ml[prow * 2 + 1] * w;
+        acc += opart[prow * d + x] * w;
+      }
+      o[vv] = L > 0.f ? acc / L : 0.f;
+    }
+    const double ds = static_cast<double>(o[1]) - o[0], dt = static_cast<double>(o[2]) - o[0];
+    es += ds * ds;
+    et += dt * dt;
+  }
+  red[0][threadIdx.x] = es;
+  red[1][threadIdx.x] = et;
+  __syncthreads();
+  for (int off = kRedThreads / 2; off > 0; off >>= 1) {
+    if (threadIdx.x < off) {
+      red[0][threadIdx.x] += red[0][threadIdx.x + off];
+      red[1][threadIdx.x] += red[1][threadIdx.x + off];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double n = static_cast<double>(r) * d;
+    const double ms = red[0][0] / n, mt = red[1][0] / n;
+    mse[bh * 2 + 0] = static_cast<float>(ms);
+    mse[bh * 2 + 1] = static_cast<float>(mt);
+    kinds[bh] = mt < ms ? kTemporal : kSpatial;
+  }
+}
+
+template <int D, int BN>
+static cudaError_t launch_prof_attn(const CUtensorMap& tqs, const CUtensorMap& tk, const CUtensorMap& tv,
+                                    const ProfArgs& pa, int BH, cudaStream_t stream) {
+  using C = ProfCfg<D, BN>;
+  auto kern = profile_attn3_kernel<D, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(BH) * pa.tiles * pa.splits;
+  kern<<<grid, kProfThreads, C::SMEM_ALLOC, stream>>>(tqs, tk, tv, pa);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_profile(const void* q, const void* k, const void* v, const Geom& g, int BH, int d, int w_s,
+                           int w_t, float scale_log2, const ProfilePlan& plan, void* ws, uint8_t* kinds_out,
+                           float* mse_out, int* err, cudaStream_t stream) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(w + plan.off_qs);
+  int4* ranges = reinterpret_cast<int4*>(w + plan.off_ranges);
+  float* opart = reinterpret_cast<float*>(w + plan.off_opart);
+  float* ml = reinterpret_cast<float*>(w + plan.off_ml);
+  {
+    const int vpr = d / 8;
+    dim3 grid((plan.r_pad * vpr + 255) / 256, BH);
+    profile_prep_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), g, d, plan.r, plan.r_pad,
+                                                  w_s, w_t, qs, ranges);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tqs, tk, tv;
+  cudaError_t e = encode_rows_map(&tqs, qs, d, plan.r_pad, BH, kPM);
+  if (e == cudaSuccess) e = encode_rows_map(&tk, k, d, g.N, BH, g.block);
+  if (e == cudaSuccess) e = encode_rows_map(&tv, v, d, g.N, BH, g.block);
+  if (e != cudaSuccess) return e;
+  ProfArgs pa;
+  pa.ranges = ranges;
+  pa.opart = opart;
+  pa.ml = ml;
+  pa.err = err;
+  pa.r_pad = plan.r_pad;
+  pa.tiles = plan.tiles;
+  pa.splits = plan.splits;
+  const int nb = (g.N + g.block - 1) / g.block;
+  pa.per_split = (nb + plan.splits - 1) / plan.splits;
+  pa.scale_log2 = scale_log2;
+  pa.g = g;
+  if (d == 128 && g.block == 128) e = launch_prof_attn<128, 128>(tqs, tk, tv, pa, BH, stream);
+  else if (d == 64 && g.block == 128) e = launch_prof_attn<64, 128>(tqs, tk, tv, pa, BH, stream);
+  else if (d == 128 && g.block == 64) e = launch_prof_attn<128, 64>(tqs, tk, tv, pa, BH, stream);
+  else if (d == 64 && g.block == 64) e = launch_prof_attn<64, 64>(tqs, tk, tv, pa, BH, stream);
+  else return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  profile_reduce_kernel<<<BH, kRedThreads, 0, stream>>>(opart, ml, plan.r, plan.r_pad, plan.splits, d, kinds_out,
+                                                        mse_out);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

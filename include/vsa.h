@@ -1,0 +1,242 @@
+/*
+ * vsa.h -- C ABI of libvsa.so: spatial-temporal block-sparse self-attention for video
+ * diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * One attention call over a latent grid of F x Hl x Wl tokens (S = Hl*Wl tokens per frame,
+ * N = F*S, natural token t = (f*Hl + h)*Wl + w = f*S + s) runs these steps, each a CUDA
+ * kernel behind one entry point below:
+ *
+ *   vsa_profile_heads   pick a spatial or temporal pattern per head from ~1% of the query
+ *                       rows ("Sparse Video-Gen" summary page, section "Approach"; its
+ *                       "Measured effects" table gives the 1% profiling fraction)
+ *   vsa_permute         gather temporal heads into frame-major order (same page,
+ *                       "Approach": the token-major to frame-major layout transformation
+ *                       that makes temporal blocks contiguous), cube heads into cube-major
+ *                       order ("USV" page, Figure 2: local 3D cubes)
+ *   vsa_build_mask      block masks: spatial/temporal windows ("Sparse Video-Gen",
+ *                       "Approach" and "Limitations": hand-fixed ratios c_s, c_t), or the
+ *                       own cube plus the top-k cubes of mean-pooled Q K^T ("USV",
+ *                       Figure 2: top-k cube selection)
+ *   vsa_sparse_attn_fwd softmax(Q K^T * scale) V restricted to the kept KV blocks, online
+ *                       softmax ("OSP-Next" page, section "Method": sparse attention kept
+ *                       compatible with FlashAttention kernels)
+ *   vsa_unpermute       scatter the output back to natural order
+ *   vsa_attention       all of the above on one stream
+ *
+ * Conventions
+ *   - Tensors are [B, H, rows, d] row-major (d fastest), bf16 unless stated otherwise.
+ *     A head's buffer holds N rows in natural or frame-major order, or C*V rows in
+ *     cube-major order (C cubes of V = cube_f*cube_h*cube_w slots, padding slots zero).
+ *   - Ownership: the caller owns every buffer (inputs, outputs, workspace, error word).
+ *     The library never allocates or frees device memory and keeps no mutable global
+ *     state; every call is asynchronous on `stream` (NULL = legacy default stream) and
+ *     never synchronises, except vsa_get_device_error.
+ *   - All device pointers must be 16-byte aligned; tensors must be contiguous.
+ *   - Errors: arguments are validated on the host before any launch (VSA_ERR_INVALID_ARG,
+ *     VSA_ERR_UNSUPPORTED, VSA_ERR_WORKSPACE); a failed launch returns VSA_ERR_CUDA.
+ *     Kernels that detect a bad device-side input (an index or count out of range) or a
+ *     bounded wait that ran out set bits of the caller's device error word `d_err`
+ *     (VSA_DEVERR_*) and return without trapping; vsa_get_device_error reads it.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define VSA_API __attribute__((visibility("default")))
+#else
+#define VSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, bad enum */
+    VSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d not in {64,128}) */
+    VSA_ERR_WORKSPACE = 3,     /* workspace smaller than the matching *_workspace_size */
+    VSA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    VSA_ERR_DEVICE = 5,        /* the device error word holds an error bit */
+    VSA_ERR_TIMEOUT = 6        /* the device error word holds the timeout bit */
+} vsa_status;
+
+/* Bits of the device error word. */
+#define VSA_DEVERR_KV_RANGE 0x1   /* kv index outside [0, blocks) or count outside [0, max_kv] */
+#define VSA_DEVERR_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up */
+#define VSA_DEVERR_KIND 0x4       /* head kind byte not one of vsa_kind */
+#define VSA_DEVERR_OVERFLOW 0x8   /* a mask row kept more blocks than max_kv */
+
+typedef enum { VSA_F32 = 0, VSA_BF16 = 1 } vsa_dtype;
+
+typedef enum { VSA_SPATIAL = 0, VSA_TEMPORAL = 1, VSA_CUBE = 2 } vsa_kind;
+
+/* How vsa_attention chooses each head's kind. */
+typedef enum {
+    VSA_SELECT_PROFILE = 0,    /* run vsa_profile_heads (bf16 input only) */
+    VSA_SELECT_GIVEN = 1,      /* read the caller's kinds from d_kind */
+    VSA_SELECT_CUBE = 2        /* every head is a cube head (own cube + top-k) */
+} vsa_select;
+
+typedef struct {
+    int B, H;                     /* batch, heads */
+    int F, Hl, Wl;                /* latent grid: frames x height x width tokens */
+    int d;                        /* head dimension: 64 or 128 */
+    int block;                    /* tokens per query block and per key block: 64 or 128 */
+    int cube_f, cube_h, cube_w;   /* cube dims for cube heads, or all 0 when unused;
+                                     cube_f*cube_h*cube_w must equal block */
+} vsa_shape;
+
+typedef struct {
+    int w_s;                      /* spatial window in frames (blocks whose frame
+                                     intervals are at most w_s apart are kept) */
+    int w_t;                      /* temporal window in positions, frame-major order */
+    double profile_frac;          /* profiled share of query rows: r = ceil(frac*N) */
+    int topk;                     /* long-range cubes per query cube (cube heads) */
+    float scale;                  /* softmax scale; 0 selects 1/sqrt(d) */
+} vsa_params;
+
+/* Pointers of one attention problem; o and lse are written. lse may be NULL. */
+typedef struct {
+    const void *q, *k, *v;        /* [B, H, rows, d] */
+    void *o;                      /* [B, H, rows, d] */
+    float *lse;                   /* [B, H, rows] natural-log log-sum-exp, or NULL */
+} vsa_qkvo;
+
+VSA_API const char *vsa_status_string(vsa_status s);
+VSA_API int vsa_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * Host-side planning helpers (no device work)
+ * --------------------------------------------------------------------------------- */
+
+/* Rows of a permuted buffer per head: N, or C*V when cube dims are set. */
+VSA_API vsa_status vsa_layout_rows(const vsa_shape *shape, int64_t *rows);
+
+/* Blocks per head in the permuted buffers: ceil(rows / block). Masks are [B,H,nblk,...]. */
+VSA_API vsa_status vsa_num_blocks(const vsa_shape *shape, int *nblk);
+
+/* Smallest window whose kept-block fraction reaches `target` for a spatial or temporal
+ * head ("Sparse Video-Gen" summary, "Measured effects": sparsity given as kept fraction).
+ * Writes the window and its exact kept fraction (kept may be NULL). */
+VSA_API vsa_status vsa_pattern_window(const vsa_shape *shape, vsa_kind kind, double target, int *w, double *kept);
+
+/* Largest number of kept KV blocks of any query block: max over the spatial window w_s and
+ * the temporal window w_t, or topk + 1 for cube shapes (cube dims set). */
+VSA_API vsa_status vsa_max_kv(const vsa_shape *shape, const vsa_params *params, int *max_kv);
+
+/* Profiling rows r = ceil(profile_frac * N) clamped to [1, N]. */
+VSA_API vsa_status vsa_profile_rows(const vsa_shape *shape, const vsa_params *params, int *rows);
+
+/* Workspace bytes of vsa_profile_heads / vsa_build_mask / vsa_attention. */
+VSA_API size_t vsa_profile_workspace_size(const vsa_shape *shape, const vsa_params *params);
+VSA_API size_t vsa_mask_workspace_size(const vsa_shape *shape, const vsa_params *params);
+VSA_API size_t vsa_attention_workspace_size(const vsa_shape *shape, const vsa_params *params, vsa_dtype dtype,
+                                    vsa_select select);
+
+/* ---------------------------------------------------------------------------------
+ * Kernels (asynchronous on `stream`)
+ * --------------------------------------------------------------------------------- */
+
+/*
+ * Gather natural-order rows into each head's layout ("Sparse Video-Gen" summary,
+ * "Approach": token-major to frame-major transformation; "USV" Figure 2: 3D cubes).
+ *   src      [B, H, N, d] in src_dtype (VSA_F32 or VSA_BF16), natural order
+ *   dst      [B, H, R, d] bf16, R from vsa_layout_rows; temporal heads get frame-major
+ *            order (slot s*F + f), cube heads cube-major order with zeroed padding slots
+ *   d_kind   [B*H] device bytes (vsa_kind)
+ * Spatial heads are left untouched when src is bf16; when src is fp32 they are copied in
+ * natural order so that dst holds bf16 values (round to nearest even) for every head.
+ */
+VSA_API vsa_status vsa_permute(const void *src, vsa_dtype src_dtype, void *dst, const uint8_t *d_kind,
+                       const vsa_shape *shape, int *d_err, cudaStream_t stream);
+
+/*
+ * Inverse of vsa_permute for outputs: dst[b,h,t] = src[b,h,slot(t)].
+ *   src      [B, H, R, d] bf16 in each head's layout;  src_lse [B, H, R] fp32 or NULL
+ *   dst      [B, H, N, d] in dst_dtype, natural order;  dst_lse [B, H, N] or NULL
+ * Spatial heads are left untouched when dst is bf16 (their output is written in place by
+ * vsa_sparse_attn_fwd); when dst is fp32 every head is converted.
+ */
+VSA_API vsa_status vsa_unpermute(const void *src, const float *src_lse, void *dst, vsa_dtype dst_dtype, float *dst_lse,
+                         const uint8_t *d_kind, const vsa_shape *shape, int *d_err, cudaStream_t stream);
+
+/*
+ * Online profiling ("Sparse Video-Gen" summary, "Approach"; "Measured effects" rows on the
+ * profiling fraction).  For r = ceil(profile_frac*N) evenly strided query rows
+ * rho_i = floor((2i+1)N/(2r)) of every head it computes dense attention and attention
+ * under the spatial (w_s) and temporal (w_t) block masks, the mean squared difference of
+ * each to dense over the r*d outputs, and picks the smaller (ties: spatial).
+ *   q, k, v  [B, H, N, d] bf16, natural order
+ *   d_kind   [B*H] out: VSA_SPATIAL or VSA_TEMPORAL
+ *   d_mse    [B*H*2] out: (spatial, temporal) mean squared error, fp32
+ *   ws       at least vsa_profile_workspace_size bytes of device memory
+ */
+VSA_API vsa_status vsa_profile_heads(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                             const vsa_params *params, uint8_t *d_kind, float *d_mse, void *ws, size_t ws_bytes,
+                             int *d_err, cudaStream_t stream);
+
+/*
+ * Block masks in three equivalent forms, per (b, h, query block i):
+ *   d_bits   [B, H, nblk, ceil(nblk/32)] uint32: bit j%32 of word j/32 set when block j is kept
+ *   d_kv_idx [B, H, nblk, max_kv] int32: kept key blocks ascending, unused entries -1
+ *   d_kv_cnt [B, H, nblk] int32: number of kept key blocks
+ * Spatial head: blocks of the natural order, kept when their frame intervals are at most
+ * w_s apart.  Temporal head: blocks of the frame-major order, kept when their position
+ * intervals are at most w_t apart.  Cube head ("USV", Figure 2): the own cube plus the
+ * topk cubes with the largest fp64 score mean(Q over cube) . mean(K over cube'), ties to
+ * the smaller index; q_cube / k_cube are the cube-major bf16 Q and K from vsa_permute
+ * (required when cube dims are set, else ignored).  Rows past a head's own block count
+ * get count 0.  A row that keeps more than max_kv blocks sets VSA_DEVERR_OVERFLOW.
+ */
+VSA_API vsa_status vsa_build_mask(const uint8_t *d_kind, const void *q_cube, const void *k_cube, const vsa_shape *shape,
+                          const vsa_params *params, uint32_t *d_bits, int32_t *d_kv_idx, int32_t *d_kv_cnt,
+                          int max_kv, void *ws, size_t ws_bytes, int *d_err, cudaStream_t stream);
+
+/*
+ * Block-sparse attention forward ("OSP-Next", "Method"; "Sparse Video-Gen", "Approach"):
+ * for every query block i of every head, O_i = softmax(Q_i K_J^T * scale) V_J over the
+ * key blocks J = kv_idx[b,h,i,0..cnt), keys past the head's real rows (ragged tail,
+ * cube padding) excluded; fp32 accumulation, bf16 output, natural-log LSE.  A row with no
+ * key gets O = 0 and LSE = -inf.
+ *   natural   q, k, v, o, lse of spatial heads ([B, H, N, d], natural order)
+ *   permuted  q, k, v, o, lse of temporal and cube heads ([B, H, R, d]); may be NULL,
+ *             in which case every head uses `natural`
+ *   d_kind    [B*H] head kinds; d_kv_idx / d_kv_cnt from vsa_build_mask
+ *   scale     softmax scale, 0 selects 1/sqrt(d)
+ */
+VSA_API vsa_status vsa_sparse_attn_fwd(const vsa_qkvo *natural, const vsa_qkvo *permuted, const uint8_t *d_kind,
+                               const int32_t *d_kv_idx, const int32_t *d_kv_cnt, int max_kv,
+                               const vsa_shape *shape, float scale, int *d_err, cudaStream_t stream);
+
+/*
+ * The whole call: kinds (profiled, given or cube) -> permute -> masks -> sparse attention
+ * -> unpermute, all on `stream`.
+ *   io        natural q, k, v (dtype), o (dtype), lse (fp32, may be NULL)
+ *   d_kind    [B*H]: read for VSA_SELECT_GIVEN, written otherwise
+ *   d_mse     [B*H*2] written by profiling (may be NULL)
+ *   ws        vsa_attention_workspace_size bytes; the masks and permuted tensors live there
+ */
+VSA_API vsa_status vsa_attention(const vsa_qkvo *io, vsa_dtype dtype, const vsa_shape *shape, const vsa_params *params,
+                         vsa_select select, uint8_t *d_kind, float *d_mse, void *ws, size_t ws_bytes, int *d_err,
+                         cudaStream_t stream);
+
+/* Byte offsets of the mask arrays inside vsa_attention's workspace (for inspection). */
+VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const vsa_params *params, vsa_dtype dtype,
+                                          vsa_select select, size_t *off_bits, size_t *off_kv_idx,
+                                          size_t *off_kv_cnt, int *max_kv);
+
+/* Synchronise `stream`, copy the device error word to *host_err and map it to a status
+ * (VSA_OK when zero, VSA_ERR_TIMEOUT when the timeout bit is set, else VSA_ERR_DEVICE). */
+VSA_API vsa_status vsa_get_device_error(const int *d_err, cudaStream_t stream, int *host_err);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

@@ -1,0 +1,138 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared entry point, and its
+host-side planning helpers and argument validation behave as documented.  No kernel runs.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from block_sparse_attention_31_b200 import _lib
+
+FAKE = 0x10000  # 16-byte-aligned non-null address; never dereferenced (validation fails first)
+
+
+def test_every_declared_symbol_is_exported():
+    names = _lib.declared_symbols()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(_lib.lib, n), n
+    assert _lib.lib.vsa_version() >= 100
+    for s in range(7):
+        assert _lib.status_string(s)
+
+
+@pytest.mark.parametrize("wl", [synthetic.WAN, synthetic.HUNYUAN, synthetic.TINY,
+                                synthetic.Workload("ragged", 1, 1, 7, 5, 9, 64, 64, "bf16", "profiled")])
+@pytest.mark.parametrize("target", [1.0, 0.35, 0.18, 0.13, 0.05])
+def test_pattern_window_matches_oracle(wl, target):
+    shape = _lib.make_shape(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block)
+    for kind in (oracle.SPATIAL, oracle.TEMPORAL):
+        w, kept = _lib.vsa_pattern_window(shape, kind, target)
+        assert w == oracle.window_for_target(kind, wl.F, wl.Hl, wl.Wl, wl.block, target)
+        assert kept == pytest.approx(oracle.kept_fraction(kind, wl.F, wl.Hl, wl.Wl, wl.block, w), abs=1e-15)
+
+
+def test_survey_window_table():
+    # windows reached on the 21x30x52 grid (block 128), also listed in the design notes
+    shape = _lib.make_shape(1, 12, 21, 30, 52, 128, 128)
+    got = {t: (_lib.vsa_pattern_window(shape, 0, t)[0], _lib.vsa_pattern_window(shape, 1, t)[0])
+           for t in (1.0, 0.35, 0.18, 0.13, 0.05)}
+    assert got == {1.0: (20, 1548), 0.35: (4, 298), 0.18: (2, 140), 0.13: (1, 98), 0.05: (0, 31)}
+
+
+@pytest.mark.parametrize("F,Hl,Wl,block,w_s,w_t", [(21, 30, 52, 128, 2, 140), (4, 8, 8, 64, 0, 0),
+                                                   (7, 5, 9, 64, 1, 7), (33, 45, 80, 128, 3, 337)])
+def test_max_kv_matches_oracle(F, Hl, Wl, block, w_s, w_t):
+    shape = _lib.make_shape(1, 2, F, Hl, Wl, 128, block)
+    got = _lib.vsa_max_kv(shape, _lib.make_params(w_s, w_t))
+    ks = oracle.pattern_keep(oracle.SPATIAL, F, Hl, Wl, block, w_s).sum(axis=1).max()
+    kt = oracle.pattern_keep(oracle.TEMPORAL, F, Hl, Wl, block, w_t).sum(axis=1).max()
+    assert got == max(ks, kt)
+
+
+def test_cube_shape_helpers():
+    wl = synthetic.WAN_6X
+    shape = _lib.make_shape(1, 12, wl.F, wl.Hl, wl.Wl, 128, 128, wl.cube)
+    assert _lib.vsa_layout_rows(shape) == oracle.layout_rows(oracle.CUBE, wl.F, wl.Hl, wl.Wl, wl.cube) == 229376
+    assert _lib.vsa_num_blocks(shape) == 1792
+    assert _lib.vsa_max_kv(shape, _lib.make_params(0, 0, topk=32)) >= 33
+    assert _lib.vsa_mask_workspace_size(shape, _lib.make_params(topk=32)) == 2 * 8 * 12 * 1792 * 128
+
+
+@pytest.mark.parametrize("N", [256, 32760, 118800, 7 * 5 * 9])
+def test_profile_rows_matches_oracle(N):
+    shape = _lib.make_shape(1, 1, 1, 1, N, 64, 64)
+    assert _lib.vsa_profile_rows(shape, _lib.make_params(profile_frac=0.01)) == oracle.profile_rows(N, 0.01)
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_shape_validation():
+    p = _lib.make_params()
+    out = ctypes.c_int64()
+    lib = _lib.lib
+    assert lib.vsa_layout_rows(ctypes.byref(_lib.make_shape(1, 1, 4, 8, 8, 96, 64)), ctypes.byref(out)) == \
+        _lib.VSA_ERR_UNSUPPORTED
+    assert lib.vsa_layout_rows(ctypes.byref(_lib.make_shape(1, 1, 4, 8, 8, 64, 32)), ctypes.byref(out)) == \
+        _lib.VSA_ERR_UNSUPPORTED
+    assert lib.vsa_layout_rows(ctypes.byref(_lib.make_shape(0, 1, 4, 8, 8, 64, 64)), ctypes.byref(out)) == \
+        _lib.VSA_ERR_INVALID_ARG
+    # cube volume must equal the block
+    assert lib.vsa_layout_rows(ctypes.byref(_lib.make_shape(1, 1, 8, 8, 8, 64, 128, (4, 4, 2))),
+                               ctypes.byref(out)) == _lib.VSA_ERR_UNSUPPORTED
+    assert lib.vsa_layout_rows(None, ctypes.byref(out)) == _lib.VSA_ERR_INVALID_ARG
+    w = ctypes.c_int()
+    assert lib.vsa_pattern_window(ctypes.byref(_lib.make_shape(1, 1, 4, 8, 8, 64, 64)), 2, 0.5, ctypes.byref(w),
+                                  None) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_pattern_window(ctypes.byref(_lib.make_shape(1, 1, 4, 8, 8, 64, 64)), 0, 1.5, ctypes.byref(w),
+                                  None) == _lib.VSA_ERR_INVALID_ARG
+    assert p.profile_frac == 0.01
+
+
+def test_kernel_entry_points_validate_before_launch():
+    lib = _lib.lib
+    shape = _lib.make_shape(1, 2, 4, 8, 8, 64, 64)
+    params = _lib.make_params(0, 0)
+    s = ctypes.c_void_p(0)
+    # null / misaligned pointers
+    assert lib.vsa_permute(None, 1, FAKE, FAKE, ctypes.byref(shape), FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_permute(FAKE + 2, 1, FAKE, FAKE, ctypes.byref(shape), FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_permute(FAKE, 7, FAKE, FAKE, ctypes.byref(shape), FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_unpermute(FAKE, FAKE, FAKE, 1, None, FAKE, ctypes.byref(shape), FAKE, s) == \
+        _lib.VSA_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.vsa_profile_heads(FAKE, FAKE, FAKE, ctypes.byref(shape), ctypes.byref(params), FAKE, FAKE, FAKE, 16,
+                                 FAKE, s) == _lib.VSA_ERR_WORKSPACE
+    bad = _lib.make_params(0, 0, profile_frac=0.0)
+    assert lib.vsa_profile_heads(FAKE, FAKE, FAKE, ctypes.byref(shape), ctypes.byref(bad), FAKE, FAKE, FAKE, 1 << 30,
+                                 FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_build_mask(FAKE, None, None, ctypes.byref(shape), ctypes.byref(params), FAKE, FAKE, FAKE, 0,
+                              None, 0, FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    io = _lib.QKVO(FAKE, FAKE, None, FAKE, None)
+    assert lib.vsa_sparse_attn_fwd(ctypes.byref(io), None, FAKE, FAKE, FAKE, 4, ctypes.byref(shape), 0.0, FAKE,
+                                   s) == _lib.VSA_ERR_INVALID_ARG
+    io = _lib.QKVO(FAKE, FAKE, FAKE, FAKE, None)
+    assert lib.vsa_attention(ctypes.byref(io), 1, ctypes.byref(shape), ctypes.byref(params), 0, FAKE, None, FAKE, 8,
+                             FAKE, s) == _lib.VSA_ERR_WORKSPACE
+    # profiling needs bf16 input; cube selection needs cube dims
+    assert lib.vsa_attention(ctypes.byref(io), 0, ctypes.byref(shape), ctypes.byref(params), 0, FAKE, None, FAKE,
+                             1 << 40, FAKE, s) == _lib.VSA_ERR_UNSUPPORTED
+    assert lib.vsa_attention(ctypes.byref(io), 1, ctypes.byref(shape), ctypes.byref(params), 2, FAKE, None, FAKE,
+                             1 << 40, FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_get_device_error(None, s, None) == _lib.VSA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_monotone():
+    shape = _lib.make_shape(1, 12, 21, 30, 52, 128, 128)
+    p = _lib.make_params(2, 140)
+    a = _lib.vsa_attention_workspace_size(shape, p, 1, 0)
+    b = _lib.vsa_attention_workspace_size(shape, p, 1, 1)
+    assert a > b > 4 * 12 * 32760 * 128 * 2
+    assert _lib.vsa_profile_workspace_size(shape, p) > 12 * 384 * 128 * 2
+    ob, oi, oc, mk = _lib.vsa_attention_workspace_layout(shape, p, 1, 1)
+    assert ob == 0 and oi > ob and oc > oi and mk == _lib.vsa_max_kv(shape, p)
+    assert np.all(np.array([ob, oi, oc]) % 256 == 0)
