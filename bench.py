@@ -210,9 +210,28 @@ class Pipeline:
 STAGES = ("profile", "permute", "mask", "attention", "unpermute")
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of a per-rank scalar over the process group (identity without one)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank runs its own independent problem (weak scaling)."""
+    return base + rank
+
+
+def aggregate_tflops(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max / 1e3) / 1e12
+
+
 def gpu_arm(args, wl, rank, world, device):
     torch.cuda.set_device(device)
-    q, k, v = synthetic.make_qkv(wl, seed=wl.seed + rank)
+    q, k, v = synthetic.make_qkv(wl, seed=rank_seed(wl.seed, rank))
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     o = torch.empty_like(qd)
     pipe = Pipeline(wl, device)
@@ -245,17 +264,11 @@ def gpu_arm(args, wl, rank, world, device):
     stage_ms = {n: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, n in enumerate(STAGES)}
     if pipe.lib.vsa_get_device_error(pipe.err) != 0:
         raise RuntimeError("device error word set during the timed region")
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device)
     ms = total_ms / args.steps
     # end to end through the public API: pinned host inputs -> device -> vsa_attention -> host O
     e2e = e2e_arm(args, wl, q, k, v, device)
-    if world > 1:
-        t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(t.item())
+    e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], device)
     return dict(ms=ms, stage_ms=stage_ms, alg=alg, exe=exe, dense=dense, pairs=pairs, kept=kept_frac,
                 clocks=clk.summary(), launches=pipe.launches, e2e=e2e, w_s=pipe.params.w_s, w_t=pipe.params.w_t,
                 kinds=pipe.kinds.cpu().tolist())
@@ -412,7 +425,7 @@ def main():
     peak_burst = float(peaks["bf16_tflops"])
     attn_s = res["stage_ms"]["attention"] / 1e3
     achieved = res["alg"] / attn_s / 1e12
-    value = world * res["alg"] / (res["ms"] / 1e3) / 1e12
+    value = aggregate_tflops(res["alg"], res["ms"], world)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["ms"], "ms_per_call": res["ms"], "higher_is_better": True,
@@ -424,7 +437,7 @@ def main():
                          (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6)},
         "value_definition": "sparse-actual TFLOP/s of the whole call: algorithmic flops of the kept blocks "
                             "(4*d*valid_q*valid_k per kept pair) / ms per call, summed over ranks",
-        "dense_equiv_tflops": world * res["dense"] / (res["ms"] / 1e3) / 1e12,
+        "dense_equiv_tflops": aggregate_tflops(res["dense"], res["ms"], world),
         "stage_ms": res["stage_ms"],
         "roofline": {"kernel": "vsa_sparse_attn_fwd", "bound": "tensor", "achieved": achieved,
                      "peak": peak_sust, "unit": "TFLOP/s", "frac": achieved / peak_sust,
@@ -434,7 +447,7 @@ def main():
                      "traffic": None},
         "gpu_launches": res["launches"] * args.steps,
         "clocks": res["clocks"],
-        "e2e": {"value": world * res["alg"] / (res["e2e"]["ms_per_step"] / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": aggregate_tflops(res["alg"], res["e2e"]["ms_per_step"], world), "unit": "TFLOP/s",
                 "ms_per_step": res["e2e"]["ms_per_step"], "h2d_bytes_per_step": res["e2e"]["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"]},
     }

@@ -17,7 +17,8 @@ no model, weights or videos are used):
   shared per-position vector (u = u_pos[h, s(t)]), so half of the heads favour
   intra-frame attention and half same-position attention across frames;
 * Q = z_Q + 2*u, K = z_K + 2*u, V = noise; cast to bf16 with round-to-nearest-even
-  except for the fp32 tiny case.
+  except for the fp32 tiny case, whose Q/K/V are plain N(0,1) (no planted vector) with
+  fixed head kinds.
 
 The planted structure mirrors the two head families of the Sparse VideoGen summary page
 ("Approach": spatial heads attend within a frame, temporal heads to the same position
@@ -79,7 +80,7 @@ class Workload:
 
 
 TINY = Workload("tiny: B1 H2 4x8x8 d64 block64 fp32", 1, 2, 4, 8, 8, 64, 64, "f32", "fixed",
-                w_s=0, w_t=0, fixed_kinds=(SPATIAL, TEMPORAL))
+                w_s=0, w_t=0, fixed_kinds=(SPATIAL, TEMPORAL), structure_scale=0.0)  # plain N(0,1)
 WAN = Workload("wan2.1-1.3b: B1 H12 21x30x52 d128 block128 bf16", 1, 12, 21, 30, 52, 128, 128,
                "bf16", "profiled", target=0.18)
 HUNYUAN = Workload("hunyuanvideo-720p: B1 H24 33x45x80 d128 block128 bf16", 1, 24, 33, 45, 80, 128, 128,
