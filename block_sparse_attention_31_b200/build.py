@@ -1,6 +1,6 @@
 """Build libvsa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-Usage: python -m block_sparse_attention_31_b200.build [--force] [--verbose]
+Usage: python block_sparse_attention_31_b200/build.py [--force] [--verbose]
 """
 from __future__ import annotations
 
