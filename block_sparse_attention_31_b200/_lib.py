@@ -48,7 +48,7 @@ class QKVO(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libvsa.so is not built ({LIB_PATH}); run `python -m block_sparse_attention_31_b200.build`")
+        raise ImportError(f"libvsa.so is not built ({LIB_PATH}); run `python block_sparse_attention_31_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, vp, i32, i64, sz = ctypes.POINTER, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     st = ctypes.c_int
@@ -66,6 +66,8 @@ def _load():
         "vsa_permute": (st, [vp, i32, vp, vp, P(Shape), vp, vp]),
         "vsa_unpermute": (st, [vp, vp, vp, i32, vp, vp, P(Shape), vp, vp]),
         "vsa_profile_heads": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, sz, vp, vp]),
+        "vsa_profile_static_scratch_bytes": (sz, []),
+        "vsa_profile_heads_static": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, vp]),
         "vsa_build_mask": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, i32, vp, sz, vp, vp]),
         "vsa_sparse_attn_fwd": (st, [P(QKVO), P(QKVO), vp, vp, vp, i32, P(Shape), ctypes.c_float, vp, vp]),
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
@@ -195,6 +197,17 @@ def vsa_unpermute(src, src_lse, dst, dst_dtype, dst_lse, kinds, shape: Shape, er
 def vsa_profile_heads(q, k, v, shape: Shape, params: Params, kinds, mse, ws, ws_bytes, err, stream=None):
     _check(lib.vsa_profile_heads(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(params), _ptr(kinds),
                                  _ptr(mse), _ptr(ws), int(ws_bytes), _ptr(err), _stream(stream)), "vsa_profile_heads")
+
+
+def vsa_profile_static_scratch_bytes() -> int:
+    return int(lib.vsa_profile_static_scratch_bytes())
+
+
+def vsa_profile_heads_static(q, k, v, shape: Shape, params: Params, kinds, mse, err, stream=None):
+    """vsa_profile_heads with the library's own fixed scratch (no workspace argument)."""
+    _check(lib.vsa_profile_heads_static(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(params),
+                                        _ptr(kinds), _ptr(mse), _ptr(err), _stream(stream)),
+           "vsa_profile_heads_static")
 
 
 def vsa_build_mask(kinds, q_cube, k_cube, shape: Shape, params: Params, bits, kv_idx, kv_cnt, max_kv, ws, ws_bytes,

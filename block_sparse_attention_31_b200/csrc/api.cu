@@ -503,3 +503,71 @@ vsa_status vsa_get_device_error(const int* d_err, cudaStream_t stream, int* host
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Profiling without caller-provided scratch
+// ---------------------------------------------------------------------------------------
+// Some callers cannot allocate device memory for a workspace: a host framework that has
+// reserved all device memory for its own pool and hands out only the tensors it owns, or
+// a latency-critical path where cudaMalloc's implicit device synchronisation is not
+// acceptable.  For them vsa_profile_heads_static keeps its scratch in a fixed device array
+// of this file (kStaticProfileScratchBytes, held by every GPU that loads the library until
+// the process exits).  The array's host-side name is only a stand-in for the device
+// address, so the address is looked up once per device with cudaGetSymbolAddress and
+// passed to the kernels.
+namespace vsa {
+constexpr size_t kStaticProfileScratchBytes = size_t(16) << 20;
+constexpr int kStaticMaxDevices = 64;
+static __device__ __align__(256) uint8_t g_profile_scratch[kStaticProfileScratchBytes];
+static std::mutex g_profile_scratch_mu;
+static void* g_profile_scratch_ptr[kStaticMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use).
+static cudaError_t profile_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kStaticMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_profile_scratch_mu);
+  if (g_profile_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_profile_scratch);
+    if (e != cudaSuccess) return e;
+    g_profile_scratch_ptr[dev] = p;
+  }
+  *out = g_profile_scratch_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace vsa
+
+extern "C" {
+
+size_t vsa_profile_static_scratch_bytes(void) { return vsa::kStaticProfileScratchBytes; }
+
+vsa_status vsa_profile_heads_static(const void* q, const void* k, const void* v, const vsa_shape* shape,
+                                    const vsa_params* params, uint8_t* d_kind, float* d_mse, int* d_err,
+                                    cudaStream_t stream) {
+  Geom g;
+  vsa_status st = make_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!q || !k || !v || !params || !d_kind || !d_mse || !d_err) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return VSA_ERR_INVALID_ARG;
+  if (!(params->profile_frac > 0.0) || params->profile_frac > 1.0 || params->w_s < 0 || params->w_t < 0)
+    return VSA_ERR_INVALID_ARG;
+  const int BH = shape->B * shape->H;
+  // Fewer key-range splits need less scratch; use the largest count that fits.
+  ProfilePlan plan = profile_plan(g, BH, shape->d, params->profile_frac);
+  for (int s = plan.splits; s >= 1; --s) {
+    plan = profile_plan_splits(g, BH, shape->d, params->profile_frac, s);
+    if (plan.bytes <= kStaticProfileScratchBytes) break;
+  }
+  if (plan.bytes > kStaticProfileScratchBytes) return VSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (profile_scratch_address(&scratch) != cudaSuccess) return VSA_ERR_CUDA;
+  const cudaError_t e = launch_profile(q, k, v, g, BH, shape->d, params->w_s, params->w_t,
+                                       scale_log2_of(params->scale, shape->d), plan, scratch, d_kind, d_mse, d_err,
+                                       stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+}  // extern "C"

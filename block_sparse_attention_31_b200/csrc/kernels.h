@@ -54,6 +54,8 @@ struct ProfilePlan {
   size_t off_qs, off_ranges, off_opart, off_ml, bytes;
 };
 ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac);
+// Same layout as profile_plan but with an explicit number of key-range splits (>= 1).
+ProfilePlan profile_plan_splits(const Geom& g, int BH, int d, double frac, int splits);
 cudaError_t launch_profile(const void* q, const void* k, const void* v, const Geom& g, int BH, int d, int w_s,
                            int w_t, float scale_log2, const ProfilePlan& plan, void* ws, uint8_t* kinds_out,
                            float* mse_out, int* err, cudaStream_t stream);

@@ -59,6 +59,18 @@ ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
   return p;
 }
 
+ProfilePlan profile_plan_splits(const Geom& g, int BH, int d, double frac, int splits) {
+  ProfilePlan p = profile_plan(g, BH, d, frac);
+  const int nb = (g.N + g.block - 1) / g.block;
+  p.splits = splits < 1 ? 1 : (splits > nb ? nb : splits);
+  size_t off = p.off_opart;
+  off = align256(off + static_cast<size_t>(BH) * p.splits * 3 * p.r_pad * d * sizeof(float));
+  p.off_ml = off;
+  off = align256(off + static_cast<size_t>(BH) * p.splits * 3 * p.r_pad * 2 * sizeof(float));
+  p.bytes = off;
+  return p;
+}
+
 // Contiguous range [lo, hi] of key blocks kept for query block i, groups of G slots.
 __device__ __forceinline__ void kept_block_range(int i, int N, int B, int G, int w, int& lo, int& hi) {
   const int nb = (N + B - 1) / B;

@@ -182,6 +182,28 @@ VSA_API vsa_status vsa_profile_heads(const void *q, const void *k, const void *v
                              int *d_err, cudaStream_t stream);
 
 /*
+ * vsa_profile_heads without a workspace argument (the pages have no counterpart; this is
+ * an interface convenience).  For callers that cannot allocate device memory themselves,
+ * e.g. code running under a host framework that owns all device memory through its own
+ * pool, or a latency-critical path that must not call cudaMalloc.  The scratch lives in a
+ * fixed array of vsa_profile_static_scratch_bytes() (16 MiB) inside the library, held by
+ * every GPU that loads the library until the process exits; nothing is allocated.
+ *   - Same arguments and results as vsa_profile_heads, minus ws / ws_bytes.
+ *   - Shapes whose scratch does not fit (after lowering the number of key-range splits to
+ *     1) return VSA_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - Every call shares the one array per device and leaves its contents behind; each call
+ *     writes every scratch byte it reads, so no clearing is needed.  Calls that overlap on
+ *     the GPU (different streams, or different host threads on the same device) race on
+ *     the array: serialise them.
+ */
+VSA_API size_t vsa_profile_static_scratch_bytes(void);
+VSA_API vsa_status vsa_profile_heads_static(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                                            const vsa_params *params, uint8_t *d_kind, float *d_mse, int *d_err,
+                                            cudaStream_t stream);
+
+/*
  * Block masks in three equivalent forms, per (b, h, query block i):
  *   d_bits   [B, H, nblk, ceil(nblk/32)] uint32: bit j%32 of word j/32 set when block j is kept
  *   d_kv_idx [B, H, nblk, max_kv] int32: kept key blocks ascending, unused entries -1
