@@ -367,6 +367,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   a.scale_log2 = scale_log2_of(scale, shape->d);
   a.g = g;
   a.nat_rows = nat_rows;
+  a.ucap = std::min(g.nblk, 2 * max_kv);
   const cudaError_t e = launch_sparse_attn(nat, perm, a, shape->d, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }

@@ -5,20 +5,26 @@
 // compatible with FlashAttention kernels; "Sparse Video-Gen" summary, "Approach": block-wise
 // spatial and temporal masks).  Online softmax in the base-2 domain, fp32 accumulation.
 //
-// One CTA per (head, query block), 192 threads in three roles:
-//   warp 0  (one lane)  TMA producer: Q once, then K_j and V_j into a 2-stage ring
-//   warp 1  (one lane)  tcgen05 issuer: S = Q K_j^T into a double-buffered TMEM tile,
-//                       O += P_j V_j into a TMEM accumulator; warp 1 also owns TMEM
-//   warps 2-5           softmax: one query row per thread (TMEM lane = row); reads S from
-//                       TMEM, rescales O in TMEM when the running max grows, writes
-//                       P = exp2(S*scale*log2e - m) as bf16 into shared memory, and at the
-//                       end normalises O and stores it through shared memory with TMA
+// One CTA per pair of consecutive query blocks of a head (tiles 0 and 1), 320 threads:
+//   warp 0  (one lane)  TMA producer: both Q tiles once, then K and V of every key block in
+//                       the union of the two lists through a 2-stage ring (each K/V tile is
+//                       loaded once and serves both query tiles)
+//   warp 1  (one lane)  tcgen05 issuer, per union entry: P.V of tile 0's previous block, Q.K^T
+//                       of tile 0, then the same for tile 1; the tensor core works on one tile
+//                       while the other tile's softmax runs.  Warp 1 also owns TMEM.
+//   warps 2-5 / 6-9     softmax of tile 0 / tile 1, one query row per thread (TMEM lane = row):
+//                       S from TMEM, online max in the base-2 domain with lazy rescaling of O
+//                       (only when the max grows by more than 2^8), P = exp2(S*scale*log2e - m)
+//                       written as packed bf16 over the tile's S columns in TMEM, where the
+//                       P.V MMA reads it; at the end O / l goes through shared memory to a TMA
+//                       store.
+// TMEM: S0, S1 (BN columns each), O0, O1 (D columns each).
 //
-// All operand tiles use the 128-byte swizzle (TMA SWIZZLE_128B == UMMA SWIZZLE_128B):
+// Shared-memory operand tiles use the 128-byte swizzle (TMA SWIZZLE_128B == UMMA SWIZZLE_128B):
 // a tile of R rows x 64 bf16 is R*128 bytes, 16-byte chunk c of row r at ((c ^ r%8)*16).
-// QK^T: A = Q (K-major), B = K (K-major).  PV: A = P (K-major over keys), B = V (MN-major:
-// keys are rows, d contiguous).  Every wait is bounded; on a timeout the CTA raises its
-// abort flag, drains its in-flight copies and MMAs, frees TMEM and returns.
+// Q.K^T: A = Q (K-major), B = K (K-major).  P.V: A = P from TMEM, B = V (MN-major: keys are
+// rows, d contiguous).  Every wait is bounded; on a timeout the CTA raises its abort flag,
+// drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -28,43 +34,42 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 192;
-constexpr int kBM = 128;  // MMA M: query rows per tile
+constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1
+constexpr int kBM = 128;           // MMA M: query rows per tile
 
 template <int D, int BN>
 struct AttnCfg {
   static constexpr int NS = 2;  // K/V ring stages
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = kBM * BN * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_Q = 0;  // two Q tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int NBAR = 16;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int BYTES = OFF_MISC + 64;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
-  static constexpr int TMEM_S0 = 0, TMEM_S1 = BN, TMEM_O = 2 * BN;
-  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  static constexpr int OFF_UNION = OFF_MISC + 64;  // union list, then two bitsets
+  static constexpr int TMEM_S = 0;                  // S of tile t at t*BN (P aliases its first BN/2 columns)
+  static constexpr int TMEM_O = 2 * BN;             // O of tile t at 2*BN + t*D
+  static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, false, true);
+  static int smem_bytes(int ucap, int nwords) { return OFF_UNION + 4 * ucap + 8 * nwords + 1024; }
 };
 
 // Barrier slots.
 enum {
-  B_Q = 0,
-  B_FULL_K = 1,   // +stage
-  B_FULL_V = 3,   // +stage
-  B_EMPTY_K = 5,  // +stage
-  B_EMPTY_V = 7,  // +stage
-  B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer
-  B_P_FULL = 13,
-  B_O_DONE = 14,
-  B_DRAIN = 15
+  B_Q = 0,         // +tile
+  B_FULL_K = 2,    // +stage
+  B_FULL_V = 4,    // +stage
+  B_EMPTY_K = 6,   // +stage
+  B_EMPTY_V = 8,   // +stage
+  B_S_FULL = 10,   // +tile
+  B_P_FULL = 12,   // +tile
+  B_O_FINAL = 14,  // +tile
+  B_DRAIN = 16
 };
+constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kKbMask = (1u << 30) - 1u;
 
 // Validity of the key columns of block kb for one head: a ragged tail (natural and
 // frame-major layouts) or cube padding slots are not real tokens.
@@ -75,17 +80,18 @@ __device__ __forceinline__ void key_valid_bits(const Geom& g, int kind, int kb, 
     uint32_t m = 0;
     for (int c = 0; c < 32; ++c) {
       const int slot = kb * BN + w * 32 + c;
-      bool ok;
-      if (kind == kCube)
-        ok = token_of_slot(g, kCube, slot) >= 0;
-      else
-        ok = slot < g.N;
+      const bool ok = kind == kCube ? token_of_slot(g, kCube, slot) >= 0 : slot < g.N;
       m |= (ok ? 1u : 0u) << c;
     }
     vb[w] = m;
   }
 }
 
+// One CTA per pair of consecutive query blocks (tiles 0 and 1) of one head.  The K/V blocks
+// of the union of the two lists stream through a 2-stage ring once and serve both tiles; the
+// MMA issuer interleaves the tiles (P.V of one, then Q.K^T of the same tile, then the other
+// tile) so the tensor core works on one tile while the other tile's softmax runs.  P is
+// written as packed bf16 over the tile's S columns in TMEM and read from there by the P.V MMA.
 template <int D, int BN>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tq_n, const __grid_constant__ CUtensorMap tk_n,
@@ -98,26 +104,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw_u32);
-  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sP = sbase + C::OFF_P;
-  uint8_t* pP = smem + C::OFF_P;
-  uint8_t* pQ = smem + C::OFF_Q;
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
-  // misc[0]: TMEM base address, misc[1]: abort flag, misc[2]: bad-list flag
+  // misc[0]: TMEM base address, misc[1]: abort flag, misc[2]: union length
   volatile int* abort_flag = misc + 1;
+  const int nwords = (a.g.nblk + 31) >> 5;
+  uint32_t* uni = reinterpret_cast<uint32_t*>(smem + C::OFF_UNION);
+  uint32_t* bits0 = uni + a.ucap;
+  uint32_t* bits1 = bits0 + nwords;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Geom& g = a.g;
-  const int bh = blockIdx.x / g.nblk;
-  const int qb = blockIdx.x - bh * g.nblk;
+  const int npairs = (g.nblk + 1) >> 1;
+  const int bh = blockIdx.x / npairs;
+  const int pair = blockIdx.x - bh * npairs;
   const int kind = a.kinds[bh];
   if (kind > kCube) {
-    if (tid == 0 && qb == 0) atomicOr(a.err, kDevErrKind);
+    if (tid == 0 && pair == 0) atomicOr(a.err, kDevErrKind);
     return;
   }
   const int rows = layout_rows(g, kind);
   const int nb_head = (rows + BN - 1) / BN;
-  if (qb >= nb_head) return;
+  const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
+  if (qb0 >= nb_head) return;
+  const bool has1 = qb1 < nb_head;
   const bool use_perm = a.has_perm && kind != kSpatial;
   const CUtensorMap* tq = use_perm ? &tq_p : &tq_n;
   const CUtensorMap* tk = use_perm ? &tk_p : &tk_n;
@@ -126,40 +137,83 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* lse = use_perm ? a.lse_perm : a.lse_nat;
   const int lse_stride = use_perm ? g.R : a.nat_rows;
 
-  // ---- validate this row's list ----
-  const size_t mrow = static_cast<size_t>(bh) * g.nblk + qb;
-  const int32_t* kvl = a.kv_idx + mrow * a.max_kv;
-  int cnt = a.kv_cnt[mrow];
-  bool bad = cnt < 0 || cnt > a.max_kv;
-  if (!bad)
-    for (int j = tid; j < cnt; j += kAttnThreads) {
-      const int kb = kvl[j];
-      bad |= kb < 0 || kb >= nb_head;
-    }
-  bool stop = false;  // drain quickly once some CTA has timed out
+  // ---- the two lists: validate, then build their union in ascending order ----
+  const size_t mrow0 = static_cast<size_t>(bh) * g.nblk + qb0;
+  const int32_t* kvl0 = a.kv_idx + mrow0 * a.max_kv;
+  const int32_t* kvl1 = kvl0 + a.max_kv;
+  int cnt0 = a.kv_cnt[mrow0];
+  int cnt1 = has1 ? a.kv_cnt[mrow0 + 1] : 0;
+  bool bad0 = cnt0 < 0 || cnt0 > a.max_kv, bad1 = cnt1 < 0 || cnt1 > a.max_kv;
+  for (int x = tid; x < 2 * nwords; x += kAttnThreads) bits0[x] = 0u;  // bits1 follows bits0
+  bool stop = false;
   if (tid == 0) stop = (*reinterpret_cast<volatile int*>(a.err) & kDevErrTimeout) != 0;
   if (__syncthreads_or(stop)) return;
-  bad = __syncthreads_or(bad);
-  if (bad) {
+  // Lists must be strictly ascending block indices in [0, nb_head).
+  if (!bad0)
+    for (int j = tid; j < cnt0; j += kAttnThreads) {
+      const int kb = kvl0[j];
+      if (kb < 0 || kb >= nb_head || (j > 0 && kvl0[j - 1] >= kb)) bad0 = true;
+      else atomicOr(&bits0[kb >> 5], 1u << (kb & 31));
+    }
+  if (!bad1)
+    for (int j = tid; j < cnt1; j += kAttnThreads) {
+      const int kb = kvl1[j];
+      if (kb < 0 || kb >= nb_head || (j > 0 && kvl1[j - 1] >= kb)) bad1 = true;
+      else atomicOr(&bits1[kb >> 5], 1u << (kb & 31));
+    }
+  bad0 = __syncthreads_or(bad0);
+  bad1 = __syncthreads_or(bad1);
+  if (bad0 || bad1) {
     if (tid == 0) atomicOr(a.err, kDevErrKvRange);
-    cnt = 0;
+    if (bad0) {
+      cnt0 = 0;
+      for (int x = tid; x < nwords; x += kAttnThreads) bits0[x] = 0u;
+    }
+    if (bad1) {
+      cnt1 = 0;
+      for (int x = tid; x < nwords; x += kAttnThreads) bits1[x] = 0u;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t u0 = w < nwords ? bits0[w] : 0u, u1 = w < nwords ? bits1[w] : 0u;
+      uint32_t u = u0 | u1;
+      const int c = __popc(u);
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      int pos = base + incl - c;
+      while (u) {
+        const int b = __ffs(u) - 1;
+        u &= u - 1u;
+        uni[pos++] = static_cast<uint32_t>(w * 32 + b) | (((u0 >> b) & 1u) ? kInTile0 : 0u) |
+                     (((u1 >> b) & 1u) ? kInTile1 : 0u);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) misc[2] = base;
   }
 
   // ---- setup: barriers and TMEM ----
   if (tid == 0) {
-    mbar_init(bar(B_Q), 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar(B_FULL_K + s), 1);
-      mbar_init(bar(B_FULL_V + s), 1);
-      mbar_init(bar(B_EMPTY_K + s), 1);
-      mbar_init(bar(B_EMPTY_V + s), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(B_Q + t), 1);
+      mbar_init(bar(B_S_FULL + t), 1);
+      mbar_init(bar(B_P_FULL + t), 128);
+      mbar_init(bar(B_O_FINAL + t), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(B_S_FULL + s), 1);
-      mbar_init(bar(B_S_FREE + s), 128);
+    for (int st = 0; st < C::NS; ++st) {
+      mbar_init(bar(B_FULL_K + st), 1);
+      mbar_init(bar(B_FULL_V + st), 1);
+      mbar_init(bar(B_EMPTY_K + st), 1);
+      mbar_init(bar(B_EMPTY_V + st), 1);
     }
-    mbar_init(bar(B_P_FULL), 128);
-    mbar_init(bar(B_O_DONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0;
     mbar_init_fence();
@@ -176,215 +230,233 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int U = misc[2];
 
   if (warp == 0) {
     // ================= TMA producer =================
-    if (lane == 0 && cnt > 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(bar(B_Q), C::Q_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * kBM * 128, tq, bar(B_Q), c * 64, qb * BN, bh);
-      for (int j = 0; j < cnt; ++j) {
-        const int s = j % C::NS;
-        const uint32_t u = j / C::NS;
-        const int kb = kvl[j];
-        if (j >= C::NS && !mbar_wait(bar(B_EMPTY_K + s), (u - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(bar(B_FULL_K + s), C::KV_BYTES);
+    if (lane == 0 && U > 0) {
+      int nk = 0, nv = 0;  // copies issued
+      const int cnts[2] = {cnt0, cnt1};
+      for (int t = 0; t < 2; ++t) {
+        if (cnts[t] == 0) continue;
+        mbar_arrive_expect_tx(bar(B_Q + t), C::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK + s * C::KV_BYTES + c * BN * 128, tk, bar(B_FULL_K + s), c * 64, kb * BN, bh);
-        if (j >= C::NS && !mbar_wait(bar(B_EMPTY_V + s), (u - 1) & 1, abort_flag, a.err)) {
-          // K of this stage is in flight; account for it on the drain path below
-          issued = -(j + 1);
-          break;
-        }
-        mbar_arrive_expect_tx(bar(B_FULL_V + s), C::KV_BYTES);
+          tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * 64,
+                      (qb0 + t) * BN, bh);
+      }
+      for (int n = 0; n < U; ++n) {
+        const int st = n % C::NS;
+        const uint32_t u = n / C::NS;
+        const int kb = static_cast<int>(uni[n] & kKbMask);
+        if (n >= C::NS && !mbar_wait(bar(B_EMPTY_K + st), (u - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(B_FULL_K + st), C::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sV + s * C::KV_BYTES + c * BN * 128, tv, bar(B_FULL_V + s), c * 64, kb * BN, bh);
-        issued = j + 1;
+          tma_load_3d(sK + st * C::KV_BYTES + c * BN * 128, tk, bar(B_FULL_K + st), c * 64, kb * BN, bh);
+        nk = n + 1;
+        if (n >= C::NS && !mbar_wait(bar(B_EMPTY_V + st), (u - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(B_FULL_V + st), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sV + st * C::KV_BYTES + c * BN * 128, tv, bar(B_FULL_V + st), c * 64, kb * BN, bh);
+        nv = n + 1;
       }
       if (*abort_flag) {
-        // Drain: wait for every copy this thread issued that nobody may have consumed.
-        mbar_wait_drain(bar(B_Q), 0, a.err);
-        const int nk = issued >= 0 ? issued : -issued;        // K copies issued
-        const int nv = issued >= 0 ? issued : -issued - 1;    // V copies issued
-        for (int s = 0; s < C::NS; ++s) {
-          // last use of stage s among the first nk (nv) iterations
+        // Drain: every copy this thread issued must land before the CTA exits.
+        for (int t = 0; t < 2; ++t)
+          if (cnts[t] > 0) mbar_wait_drain(bar(B_Q + t), 0, a.err);
+        for (int st = 0; st < C::NS; ++st) {
           int lk = -1, lv = -1;
-          for (int j = s; j < nk; j += C::NS) lk = j;
-          for (int j = s; j < nv; j += C::NS) lv = j;
-          if (lk >= 0) mbar_wait_drain(bar(B_FULL_K + s), (lk / C::NS) & 1, a.err);
-          if (lv >= 0) mbar_wait_drain(bar(B_FULL_V + s), (lv / C::NS) & 1, a.err);
+          for (int n = st; n < nk; n += C::NS) lk = n;
+          for (int n = st; n < nv; n += C::NS) lv = n;
+          if (lk >= 0) mbar_wait_drain(bar(B_FULL_K + st), (lk / C::NS) & 1, a.err);
+          if (lv >= 0) mbar_wait_drain(bar(B_FULL_V + st), (lv / C::NS) & 1, a.err);
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ================= tcgen05 issuer =================
-    if (lane == 0 && cnt > 0) {
-      auto issue_pv = [&](int jp) -> bool {
-        const int sp = jp % C::NS;
-        if (!mbar_wait(bar(B_P_FULL), jp & 1, abort_flag, a.err)) return false;
-        if (!mbar_wait(bar(B_FULL_V + sp), (jp / C::NS) & 1, abort_flag, a.err)) return false;
+    if (lane == 0 && U > 0) {
+      const int cnts[2] = {cnt0, cnt1};
+      int pend[2] = {-1, -1};   // union entry whose Q.K^T is issued and P.V is not
+      int pvc[2] = {0, 0};      // P.V products issued per tile
+      bool qready[2] = {false, false};
+      bool ok = true;
+      auto issue_pv = [&](int t) -> bool {
+        const int np = pend[t];
+        if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
+        if (!mbar_wait(bar(B_FULL_V + np % C::NS), (np / C::NS) & 1, abort_flag, a.err)) return false;
         tc_fence_after();
+        const uint32_t vbase = sV + (np % C::NS) * C::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sV + sp * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024);
-          tc_mma_ss(tmem + C::TMEM_O, ad, bd, C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+          tc_mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * BN + kk * 8, bd, C::IDESC_PV,
+                    (pvc[t] > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(B_EMPTY_V + sp));
-        tc_commit(bar(B_O_DONE));
+        pend[t] = -1;
+        if (++pvc[t] == cnts[t]) tc_commit(bar(B_O_FINAL + t));
         return true;
       };
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, a.err);
-      for (int j = 0; ok && j < cnt; ++j) {
-        const int s = j % C::NS, sb = j & 1;
-        if (!mbar_wait(bar(B_FULL_K + s), (j / C::NS) & 1, abort_flag, a.err)) {
+      for (int n = 0; ok && n < U; ++n) {
+        const int st = n % C::NS;
+        if (!mbar_wait(bar(B_FULL_K + st), (n / C::NS) & 1, abort_flag, a.err)) {
           ok = false;
           break;
         }
-        if (j >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((j - 2) >> 1) & 1, abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        const uint32_t e = uni[n];
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
-          tc_mma_ss(tmem + (sb ? C::TMEM_S1 : C::TMEM_S0), ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        for (int t = 0; t < 2; ++t) {
+          if (pend[t] >= 0 && !issue_pv(t)) {
+            ok = false;
+            break;
+          }
+          if (!((e >> (30 + t)) & 1u)) continue;
+          if (!qready[t]) {
+            if (!mbar_wait(bar(B_Q + t), 0, abort_flag, a.err)) {
+              ok = false;
+              break;
+            }
+            qready[t] = true;
+          }
+          tc_fence_after();
+          const uint32_t qbase = sbase + C::OFF_Q + t * C::Q_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(qbase + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                sdesc_sw128(sK + st * C::KV_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+            tc_mma_ss(tmem + C::TMEM_S + t * BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(B_S_FULL + t));
+          pend[t] = n;
         }
-        tc_commit(bar(B_EMPTY_K + s));
-        tc_commit(bar(B_S_FULL + sb));
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
-        }
+        if (!ok) break;
+        tc_commit(bar(B_EMPTY_K + st));
+        if (n >= 1) tc_commit(bar(B_EMPTY_V + (n - 1) % C::NS));
       }
-      if (ok) issue_pv(cnt - 1);
+      for (int t = 0; ok && t < 2; ++t)
+        if (pend[t] >= 0 && !issue_pv(t)) ok = false;
       // Drain: all MMAs issued by this thread complete before TMEM is released.
       tc_commit(bar(B_DRAIN));
       mbar_wait_drain(bar(B_DRAIN), 0, a.err);
     }
     __syncwarp();
   } else {
-    // ================= softmax (warps 2..5, one row per thread) =================
-    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;  // query row within the tile
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < cnt; ++j) {
-      const int sb = j & 1;
-      ok = mbar_wait(bar(B_S_FULL + sb), (j >> 1) & 1, abort_flag, a.err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + (sb ? C::TMEM_S1 : C::TMEM_S0) + c * 32, s + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar(B_S_FREE + sb));
-      const int kb = kvl[j];
-      if (!block_full(g, kind, kb)) {
-        uint32_t vb[BN / 32];
-        key_valid_bits<BN>(g, kind, kb, vb);
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (!((vb[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m, mx * sl2);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      if (j >= 1) {
-        ok = mbar_wait(bar(B_O_DONE), (j - 1) & 1, abort_flag, a.err);
-        ok = __all_sync(0xffffffffu, ok);
+    // ================= softmax: warps 2-5 tile 0, warps 6-9 tile 1; one row per thread =================
+    const int t = (warp - 2) >> 2;
+    const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;   // query row within the tile
+    if (t == 0 || has1) {
+      const int cnt = t ? cnt1 : cnt0;
+      const int32_t* kvl = t ? kvl1 : kvl0;
+      const int qb = qb0 + t;
+      const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+      const uint32_t t_s = t_lane + C::TMEM_S + t * BN, t_o = t_lane + C::TMEM_O + t * D;
+      const float sl2 = a.scale_log2;
+      float m = -INFINITY, l = 0.f;  // m: the (lazily updated) max used for the exponentials
+      bool ok = true;
+      for (int k = 0; k < cnt; ++k) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), k & 1, abort_flag, a.err));
         if (!ok) break;
         tc_fence_after();
-        const float alpha = fast_exp2(m - m_use);
-        if (__any_sync(0xffffffffu, alpha < 1.f)) {
+        float s[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
+        const int kb = kvl[k];
+        if (!block_full(g, kind, kb)) {
+          uint32_t vb[BN / 32];
+          key_valid_bits<BN>(g, kind, kb, vb);
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (!((vb[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m, mx * sl2);
+        // Rescale only when the running max grows by more than 2^8; otherwise keep the old
+        // max (the exponentials stay below 256 and the final 1/l normalisation is exact).
+        const bool grow = m_new > m + 8.f;
+        if (k > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
+          const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            tmem_ld32(t_lane + C::TMEM_O + c * 32, o);
+            tmem_ld32(t_o + c * 32, o);
 #pragma unroll
             for (int x = 0; x < 32; ++x) o[x] *= alpha;
-            tmem_st32(t_lane + C::TMEM_O + c * 32, o);
+            tmem_st32(t_o + c * 32, o);
           }
         }
-        l *= alpha;
-      }
-      // P = exp2(S * scale * log2(e) - m), bf16 into the swizzled K-major P tile
-      float rs = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {
-        float p[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          p[x] = fast_exp2(fmaf(s[ch * 8 + x], sl2, -m_use));
-          rs += p[x];
+        if (grow) {
+          l *= fast_exp2(m - m_new);
+          m = m_new;
         }
-        uint4 pk;
-        pk.x = pack_bf16x2(p[0], p[1]);
-        pk.y = pack_bf16x2(p[2], p[3]);
-        pk.z = pack_bf16x2(p[4], p[5]);
-        pk.w = pack_bf16x2(p[6], p[7]);
-        const int kc = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(pP + kc * (kBM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = pk;
+        const float m_use = m == -INFINITY ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) {  // 64 probabilities -> 32 packed columns at a time
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = fast_exp2(fmaf(s[h * 64 + 2 * c], sl2, -m_use));
+            const float p1 = fast_exp2(fmaf(s[h * 64 + 2 * c + 1], sl2, -m_use));
+            rs += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32_u(t_s + h * 32, pk);
+        }
+        l += rs;
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL + t));
       }
-      l += rs;
-      m = m_new;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(B_P_FULL));
-    }
-    // ---- epilogue ----
-    if (ok && cnt > 0) {
-      ok = mbar_wait(bar(B_O_DONE), (cnt - 1) & 1, abort_flag, a.err);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-    }
-    const bool have = ok && cnt > 0 && l > 0.f;
-    const float inv = have ? 1.f / l : 0.f;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
+      // ---- epilogue: O / l -> bf16 -> swizzled smem (over this tile's Q) -> TMA store ----
       if (ok && cnt > 0) {
-        tmem_ld32(t_lane + C::TMEM_O + c * 32, o);
-      } else {
-#pragma unroll
-        for (int x = 0; x < 32; ++x) o[x] = 0.f;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FINAL + t), 0, abort_flag, a.err));
+        tc_fence_after();
       }
-      if (row < BN) {
+      const bool have = ok && cnt > 0 && l > 0.f;
+      const float inv = have ? 1.f / l : 0.f;
+      uint8_t* stage = smem + C::OFF_Q + t * C::Q_BYTES;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (ok && cnt > 0) {
+          tmem_ld32(t_o + c * 32, o);
+        } else {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 pk;
-          pk.x = pack_bf16x2(o[q4 * 8 + 0] * inv, o[q4 * 8 + 1] * inv);
-          pk.y = pack_bf16x2(o[q4 * 8 + 2] * inv, o[q4 * 8 + 3] * inv);
-          pk.z = pack_bf16x2(o[q4 * 8 + 4] * inv, o[q4 * 8 + 5] * inv);
-          pk.w = pack_bf16x2(o[q4 * 8 + 6] * inv, o[q4 * 8 + 7] * inv);
-          const int col = c * 32 + q4 * 8;  // element column
-          const int dc = col >> 6, cc = (col & 63) >> 3;
-          *reinterpret_cast<uint4*>(pQ + dc * (BN * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = pk;
+          for (int x = 0; x < 32; ++x) o[x] = 0.f;
+        }
+        if (row < BN) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v4;
+            v4.x = pack_bf16x2(o[q4 * 8 + 0] * inv, o[q4 * 8 + 1] * inv);
+            v4.y = pack_bf16x2(o[q4 * 8 + 2] * inv, o[q4 * 8 + 3] * inv);
+            v4.z = pack_bf16x2(o[q4 * 8 + 4] * inv, o[q4 * 8 + 5] * inv);
+            v4.w = pack_bf16x2(o[q4 * 8 + 6] * inv, o[q4 * 8 + 7] * inv);
+            const int col = c * 32 + q4 * 8;
+            const int dc = col >> 6, cc = (col & 63) >> 3;
+            *reinterpret_cast<uint4*>(stage + dc * (BN * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v4;
+          }
         }
       }
-    }
-    fence_proxy_async_smem();
-    named_barrier_sync(1, 128);
-    if (warp == 2 && lane == 0) {
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + t, 128);
+      if (quad == 2 && lane == 0) {
+        const uint32_t sstage = sbase + C::OFF_Q + t * C::Q_BYTES;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_store_3d(to, sQ + c * BN * 128, c * 64, qb * BN, bh);
-      tma_store_commit();
-      tma_store_wait_all();
+        for (int c = 0; c < D / 64; ++c) tma_store_3d(to, sstage + c * BN * 128, c * 64, qb * BN, bh);
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+      if (lse != nullptr && row < BN && qb * BN + row < rows)
+        lse[static_cast<size_t>(bh) * lse_stride + qb * BN + row] =
+            have ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
-    if (lse != nullptr && row < BN && qb * BN + row < rows)
-      lse[static_cast<size_t>(bh) * lse_stride + qb * BN + row] =
-          have ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
@@ -397,12 +469,15 @@ template <int D, int BN>
 static cudaError_t launch_attn_t(const AttnMaps& nat, const AttnMaps& perm, const AttnArgs& a, cudaStream_t stream) {
   using C = AttnCfg<D, BN>;
   auto kern = sparse_attn_fwd_kernel<D, BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  const int nwords = (a.g.nblk + 31) / 32;
+  const int smem = C::smem_bytes(a.ucap, nwords);
+  if (smem > 232448) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(a.BH) * a.g.nblk;
+  const long long grid = static_cast<long long>(a.BH) * ((a.g.nblk + 1) / 2);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kAttnThreads, C::SMEM_ALLOC, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
-                                                                              perm.v, perm.o, a);
+  kern<<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
+                                                                     perm.v, perm.o, a);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ struct AttnArgs {
   int max_kv;
   int has_perm;
   int nat_rows;  // rows per head of the natural buffers (N, or R when they hold every layout)
+  int ucap;      // capacity of the per-CTA union list: min(nblk, 2 * max_kv)
   float scale_log2;
   Geom g;
 };
@@ -51,7 +52,7 @@ struct ProfilePlan {
   int r_pad;    // rounded up to the 128-row tile
   int tiles;    // r_pad / 128
   int splits;   // key-range splits per tile
-  size_t off_qs, off_ranges, off_opart, off_ml, bytes;
+  size_t off_qs, off_ranges, off_opart, off_ml, off_rowerr, bytes;
 };
 ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac);
 // Same layout as profile_plan but with an explicit number of key-range splits (>= 1).

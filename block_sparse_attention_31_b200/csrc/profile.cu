@@ -16,10 +16,13 @@
 //            then three online softmaxes (dense, spatial-masked, temporal-masked) sharing
 //            that S, and three P V products into three TMEM accumulators; writes the
 //            partial (max, sum, unnormalised O) of each variant;
-//   reduce   one CTA per head: merges the splits, forms the three outputs, accumulates the
-//            two squared errors in fp64 in a fixed order and picks the kind.
+//   row_error one CTA per (sampled row, head): merges the splits, forms the three outputs and
+//            the row's two squared errors (fp64);
+//   reduce   one CTA per head: sums the rows' errors in a fixed order and picks the kind.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <cmath>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -29,6 +32,7 @@ namespace vsa {
 
 constexpr int kProfThreads = 192;
 constexpr int kPM = 128;  // rows per tile
+constexpr int kNumSMs = 148;
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -41,10 +45,24 @@ ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
   p.r_pad = (p.r + kPM - 1) / kPM * kPM;
   p.tiles = p.r_pad / kPM;
   const int nb = (g.N + g.block - 1) / g.block;
-  const long long ctas = static_cast<long long>(BH) * p.tiles;
-  int splits = static_cast<int>((2 * 148 + ctas - 1) / ctas);
-  if (splits < 1) splits = 1;
-  if (splits > nb) splits = nb;
+  // Key-range splits: the smallest count that fills at least one wave of 148 SMs with a last
+  // wave at least 90% full; otherwise the count (up to 16) with the fullest last wave.
+  const long long tiles = static_cast<long long>(BH) * p.tiles;
+  auto wave_eff = [&](int s) {
+    const double w = static_cast<double>(tiles * s) / kNumSMs;
+    return w / std::ceil(w);
+  };
+  int splits = 0;
+  for (int s = 1; s <= 16 && s <= nb; ++s)
+    if (tiles * s >= kNumSMs && wave_eff(s) >= 0.9) {
+      splits = s;
+      break;
+    }
+  if (splits == 0) {
+    splits = 1;
+    for (int s = 2; s <= 16 && s <= nb; ++s)
+      if (wave_eff(s) > wave_eff(splits) + 1e-9) splits = s;
+  }
   p.splits = splits;
   size_t off = 0;
   p.off_qs = off;
@@ -55,6 +73,8 @@ ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
   off = align256(off + static_cast<size_t>(BH) * splits * 3 * p.r_pad * d * sizeof(float));
   p.off_ml = off;
   off = align256(off + static_cast<size_t>(BH) * splits * 3 * p.r_pad * 2 * sizeof(float));
+  p.off_rowerr = off;
+  off = align256(off + static_cast<size_t>(BH) * p.r_pad * 2 * sizeof(double));
   p.bytes = off;
   return p;
 }
@@ -67,6 +87,8 @@ ProfilePlan profile_plan_splits(const Geom& g, int BH, int d, double frac, int s
   off = align256(off + static_cast<size_t>(BH) * p.splits * 3 * p.r_pad * d * sizeof(float));
   p.off_ml = off;
   off = align256(off + static_cast<size_t>(BH) * p.splits * 3 * p.r_pad * 2 * sizeof(float));
+  p.off_rowerr = off;
+  off = align256(off + static_cast<size_t>(BH) * p.r_pad * 2 * sizeof(double));
   p.bytes = off;
   return p;
 }
@@ -159,6 +181,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
+  volatile uint32_t* flags = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 16);  // [2][4]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Geom& g = a.g;
@@ -226,16 +249,21 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       auto issue_pv = [&](int jp) -> bool {
         if (!mbar_wait(bar(PB_P_FULL), jp & 1, abort_flag, a.err)) return false;
         if (!mbar_wait(bar(PB_FULL_V), jp & 1, abort_flag, a.err)) return false;
+        // variants that some row of the tile allows in this block (one word per softmax warp)
+        const uint32_t used = flags[(jp & 1) * 4 + 0] | flags[(jp & 1) * 4 + 1] | flags[(jp & 1) * 4 + 2] |
+                              flags[(jp & 1) * 4 + 3];
         tc_fence_after();
 #pragma unroll
-        for (int vv = 0; vv < 3; ++vv)
+        for (int vv = 0; vv < 3; ++vv) {
+          if (!((used >> vv) & 1u)) continue;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t ad =
                 sdesc_sw128(sP + vv * C::P_BYTES + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(sV + kk * 16 * 128, BN * 128, 1024);
-            tc_mma_ss(tmem + C::TMEM_O + vv * D, ad, bd, C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ss(tmem + C::TMEM_O + vv * D, ad, bd, C::IDESC_PV, 1u);
           }
+        }
         tc_commit(bar(PB_EMPTY_V));
         tc_commit(bar(PB_O_DONE));
         return true;
@@ -274,8 +302,21 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = a.scale_log2;
+    // Allowed keys of this row: spatial = natural tokens [rg.x, rg.y) (whole blocks),
+    // temporal = frame-major slots [rg.z, rg.w), i.e. (s, f) from (ts_lo, tf_lo) to (ts_hi, tf_hi).
     const int4 rg = a.ranges[tile * kPM + row];
+    const bool t_any = rg.w > rg.z;
+    const int ts_lo = rg.z / g.F, tf_lo = rg.z - (rg.z / g.F) * g.F;
+    const int ts_hi = t_any ? (rg.w - 1) / g.F : -1, tf_hi = t_any ? (rg.w - 1) - ((rg.w - 1) / g.F) * g.F : -1;
     float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f};
+    // Zero the accumulators: every P.V product accumulates, and skipped ones leave zeros.
+    {
+      float z[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) z[x] = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 3 * D / 32; ++c) tmem_st32(t_lane + C::TMEM_O + c * 32, z);
+    }
     bool ok = true;
     for (int j = 0; j < cnt; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_S_FULL), j & 1, abort_flag, a.err));
@@ -286,40 +327,50 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + C::TMEM_S + c * 32, s + c * 32);
       tc_fence_before();
       mbar_arrive(bar(PB_S_FREE));
-      // masks of the three variants for this block's key tokens t = kb*BN + c
       const int t0 = (kb0 + j) * BN;
-      uint32_t mk[3][BN / 32];
-      {
-        int f = t0 / g.S, sp = t0 - (t0 / g.S) * g.S;
+      const int nvalid = min(BN, g.N - t0);
+      // spatial: the block is either inside the row's token range or outside it
+      const bool sp_on = t0 >= rg.x && t0 < rg.y;
+      // temporal: quick reject on the block's position span, then an exact per-column mask
+      const int f_a = t0 / g.S, s_a = t0 - f_a * g.S;
+      const int f_b = (t0 + nvalid - 1) / g.S, s_b = (t0 + nvalid - 1) - f_b * g.S;
+      bool tp_on = t_any;
+      if (tp_on && f_a == f_b) tp_on = s_a <= ts_hi && s_b >= ts_lo;
+      else if (tp_on && f_b == f_a + 1) tp_on = (s_a <= ts_hi) || (s_b >= ts_lo);
+      uint32_t mt[BN / 32];
 #pragma unroll
-        for (int w = 0; w < BN / 32; ++w) {
-          uint32_t md = 0, ms = 0, mt = 0;
+      for (int w = 0; w < BN / 32; ++w) mt[w] = 0u;
+      if (tp_on) {
+        int f = f_a, sp = s_a;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int t = t0 + w * 32 + c;
-            const int p = sp * g.F + f;
-            const bool valid = t < g.N;
-            md |= (valid ? 1u : 0u) << c;
-            ms |= ((valid && t >= rg.x && t < rg.y) ? 1u : 0u) << c;
-            mt |= ((valid && p >= rg.z && p < rg.w) ? 1u : 0u) << c;
-            if (++sp == g.S) {
-              sp = 0;
-              ++f;
-            }
+        for (int c = 0; c < BN; ++c) {
+          const bool in = c < nvalid && (sp > ts_lo || (sp == ts_lo && f >= tf_lo)) &&
+                          (sp < ts_hi || (sp == ts_hi && f <= tf_hi));
+          mt[c >> 5] |= (in ? 1u : 0u) << (c & 31);
+          if (++sp == g.S) {
+            sp = 0;
+            ++f;
           }
-          mk[0][w] = md;
-          mk[1][w] = ms;
-          mk[2][w] = mt;
         }
+        uint32_t any = 0u;
+#pragma unroll
+        for (int w = 0; w < BN / 32; ++w) any |= mt[w];
+        tp_on = any != 0u;
       }
+      // per-variant row maxima (raw scores)
+      float mx0 = -INFINITY, mx2 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        const float v = c < nvalid ? s[c] : -INFINITY;
+        s[c] = v;
+        mx0 = fmaxf(mx0, v);
+        if ((mt[c >> 5] >> (c & 31)) & 1u) mx2 = fmaxf(mx2, v);
+      }
+      const float mx[3] = {mx0, sp_on ? mx0 : -INFINITY, tp_on ? mx2 : -INFINITY};
       float mnew[3], muse[3];
 #pragma unroll
       for (int vv = 0; vv < 3; ++vv) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if ((mk[vv][c >> 5] >> (c & 31)) & 1u) mx = fmaxf(mx, s[c]);
-        mnew[vv] = fmaxf(m[vv], mx * sl2);
+        mnew[vv] = fmaxf(m[vv], mx[vv] * sl2);
         muse[vv] = mnew[vv] == -INFINITY ? 0.f : mnew[vv];
       }
       if (j >= 1) {
@@ -329,7 +380,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
         for (int vv = 0; vv < 3; ++vv) {
           const float alpha = fast_exp2(m[vv] - muse[vv]);
-          if (__any_sync(0xffffffffu, alpha < 1.f)) {
+          if (__any_sync(0xffffffffu, alpha < 1.f && m[vv] != -INFINITY)) {
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
               float o[32];
@@ -342,8 +393,14 @@ __global__ void __launch_bounds__(kProfThreads, 1)
           l[vv] *= alpha;
         }
       }
+      // publish which variants this warp's rows use in this block (read by the MMA issuer)
+      {
+        const uint32_t use = 1u | (__any_sync(0xffffffffu, sp_on) ? 2u : 0u) | (__any_sync(0xffffffffu, tp_on) ? 4u : 0u);
+        if (lane == 0) flags[(j & 1) * 4 + quad] = use;
+      }
 #pragma unroll
       for (int vv = 0; vv < 3; ++vv) {
+        const bool on = vv == 0 || (vv == 1 ? sp_on : tp_on);
         float rs = 0.f;
         uint8_t* pv = pP + vv * C::P_BYTES;
 #pragma unroll
@@ -352,7 +409,8 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             const int c = ch * 8 + x;
-            p[x] = ((mk[vv][c >> 5] >> (c & 31)) & 1u) ? fast_exp2(fmaf(s[c], sl2, -muse[vv])) : 0.f;
+            const bool keep = vv == 2 ? ((mt[c >> 5] >> (c & 31)) & 1u) != 0u : true;
+            p[x] = (on && keep) ? fast_exp2(fmaf(s[c], sl2, -muse[vv])) : 0.f;
             rs += p[x];
           }
           uint4 pk;
@@ -403,39 +461,67 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+// Merge the key splits of one sampled row of one head and accumulate its two squared errors
+// (one CTA of d threads per (row, head)); the per-row sums are reduced in fixed order below.
+__global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __restrict__ opart,
+                                                                const float* __restrict__ ml, int r_pad,
+                                                                int splits, int d, double* __restrict__ row_err) {
+  __shared__ double red[2][4];
+  const int i = blockIdx.x, bh = blockIdx.y, x = threadIdx.x;
+  float o[3];
+#pragma unroll
+  for (int vv = 0; vv < 3; ++vv) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < splits; ++sp) {
+      const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
+      M = fmaxf(M, ml[prow * 2]);
+    }
+    float L = 0.f, acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
+      const float ms = ml[prow * 2];
+      if (ms == -INFINITY) continue;
+      const float w = exp2f(ms - M);
+      L += ml[prow * 2 + 1] * w;
+      acc += opart[prow * d + x] * w;
+    }
+    o[vv] = L > 0.f ? acc / L : 0.f;
+  }
+  const double ds = static_cast<double>(o[1]) - o[0], dt = static_cast<double>(o[2]) - o[0];
+  double es = ds * ds, et = dt * dt;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    es += __shfl_xor_sync(0xffffffffu, es, off);
+    et += __shfl_xor_sync(0xffffffffu, et, off);
+  }
+  if ((x & 31) == 0) {
+    red[0][x >> 5] = es;
+    red[1][x >> 5] = et;
+  }
+  __syncthreads();
+  if (x == 0) {
+    double a = 0.0, b = 0.0;
+    for (int w = 0; w < d / 32; ++w) {
+      a += red[0][w];
+      b += red[1][w];
+    }
+    row_err[(static_cast<size_t>(bh) * r_pad + i) * 2 + 0] = a;
+    row_err[(static_cast<size_t>(bh) * r_pad + i) * 2 + 1] = b;
+  }
+}
+
 constexpr int kRedThreads = 256;
 
-__global__ void __launch_bounds__(kRedThreads) profile_reduce_kernel(const float* __restrict__ opart,
-                                                                     const float* __restrict__ ml, int r, int r_pad,
-                                                                     int splits, int d, uint8_t* __restrict__ kinds,
+// Sum the per-row errors of one head in a fixed order, form the two MSEs, pick the kind.
+__global__ void __launch_bounds__(kRedThreads) profile_reduce_kernel(const double* __restrict__ row_err, int r,
+                                                                     int r_pad, int d, uint8_t* __restrict__ kinds,
                                                                      float* __restrict__ mse) {
   __shared__ double red[2][kRedThreads];
   const int bh = blockIdx.x;
   double es = 0.0, et = 0.0;
-  for (int idx = threadIdx.x; idx < r * d; idx += kRedThreads) {
-    const int i = idx / d, x = idx - (idx / d) * d;
-    float o[3];
-#pragma unroll
-    for (int vv = 0; vv < 3; ++vv) {
-      float M = -INFINITY;
-      for (int sp = 0; sp < splits; ++sp) {
-        const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-        M = fmaxf(M, ml[prow * 2]);
-      }
-      float L = 0.f, acc = 0.f;
-      for (int sp = 0; sp < splits; ++sp) {
-        const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-        const float ms = ml[prow * 2];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
-        L += ml[prow * 2 + 1] * w;
-        acc += opart[prow * d + x] * w;
-      }
-      o[vv] = L > 0.f ? acc / L : 0.f;
-    }
-    const double ds = static_cast<double>(o[1]) - o[0], dt = static_cast<double>(o[2]) - o[0];
-    es += ds * ds;
-    et += dt * dt;
+  for (int i = threadIdx.x; i < r; i += kRedThreads) {
+    es += row_err[(static_cast<size_t>(bh) * r_pad + i) * 2 + 0];
+    et += row_err[(static_cast<size_t>(bh) * r_pad + i) * 2 + 1];
   }
   red[0][threadIdx.x] = es;
   red[1][threadIdx.x] = et;
@@ -507,8 +593,11 @@ cudaError_t launch_profile(const void* q, const void* k, const void* v, const Ge
   else if (d == 64 && g.block == 64) e = launch_prof_attn<64, 64>(tqs, tk, tv, pa, BH, stream);
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;
-  profile_reduce_kernel<<<BH, kRedThreads, 0, stream>>>(opart, ml, plan.r, plan.r_pad, plan.splits, d, kinds_out,
-                                                        mse_out);
+  double* row_err = reinterpret_cast<double*>(w + plan.off_rowerr);
+  profile_row_error_kernel<<<dim3(plan.r, BH), d, 0, stream>>>(opart, ml, plan.r_pad, plan.splits, d, row_err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  profile_reduce_kernel<<<BH, kRedThreads, 0, stream>>>(row_err, plan.r, plan.r_pad, d, kinds_out, mse_out);
   return cudaGetLastError();
 }
 

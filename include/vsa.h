@@ -229,7 +229,8 @@ VSA_API vsa_status vsa_build_mask(const uint8_t *d_kind, const void *q_cube, con
  *   natural   q, k, v, o, lse of spatial heads ([B, H, N, d], natural order)
  *   permuted  q, k, v, o, lse of temporal and cube heads ([B, H, R, d]); may be NULL,
  *             in which case every head uses `natural`
- *   d_kind    [B*H] head kinds; d_kv_idx / d_kv_cnt from vsa_build_mask
+ *   d_kind    [B*H] head kinds; d_kv_idx / d_kv_cnt from vsa_build_mask (each list strictly
+ *             ascending; a malformed list sets VSA_DEVERR_KV_RANGE and its rows are zero)
  *   scale     softmax scale, 0 selects 1/sqrt(d)
  */
 VSA_API vsa_status vsa_sparse_attn_fwd(const vsa_qkvo *natural, const vsa_qkvo *permuted, const uint8_t *d_kind,
