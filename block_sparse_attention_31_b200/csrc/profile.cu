@@ -13,8 +13,9 @@
 //            and, per sampled row, the contiguous key range each pattern allows (spatial:
 //            a natural-order token range; temporal: a frame-major slot range);
 //   attn3    one CTA per (head, 128-row tile, key split): S = Q K^T on tcgen05 into TMEM,
-//            then three online softmaxes (dense, spatial-masked, temporal-masked) sharing
-//            that S, and three P V products into three TMEM accumulators; writes the
+//            one online softmax whose probabilities serve the dense, spatial-masked and
+//            temporal-masked variants, and three P.V products into three TMEM accumulators
+//            (the masked ones with rows switched off by the MMA's lane mask); writes the
 //            partial (max, sum, unnormalised O) of each variant;
 //   row_error one CTA per (sampled row, head): merges the splits, forms the three outputs and
 //            the row's two squared errors (fp64);
@@ -142,20 +143,22 @@ struct ProfCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int P_BYTES = kPM * BN * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_P = OFF_V + KV_BYTES;  // three P tiles
-  static constexpr int OFF_BAR = OFF_P + 3 * P_BYTES;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;      // 2 stages
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES; // 2 stages
+  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES; // temporal-masked P
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
-  static constexpr int BYTES = OFF_MISC + 64;
+  static constexpr int BYTES = OFF_MISC + 128;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
+  // TMEM: S (dense P packed over its first BN/2 columns), then O of dense, spatial, temporal
   static constexpr int TMEM_S = 0, TMEM_O = BN;
   static constexpr int TMEM_COLS = (BN + 3 * D) <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kPM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kPM, D, false, true);
 };
 
-enum { PB_Q = 0, PB_FULL_K, PB_FULL_V, PB_EMPTY_K, PB_EMPTY_V, PB_S_FULL, PB_S_FREE, PB_P_FULL, PB_O_DONE, PB_DRAIN };
+enum { PB_Q = 0, PB_FULL_K = 1, PB_FULL_V = 3, PB_EMPTY_K = 5, PB_EMPTY_V = 7, PB_S_FULL = 9, PB_P_FULL = 10,
+       PB_O_FINAL = 11, PB_DRAIN = 12 };
 
 struct ProfArgs {
   const int4* ranges;
@@ -167,6 +170,23 @@ struct ProfArgs {
   Geom g;
 };
 
+// Set bits [lo, hi] (inclusive, columns) of a BN-bit mask.
+template <int BN>
+__device__ __forceinline__ void set_bit_range(uint32_t (&m)[BN / 32], int lo, int hi) {
+#pragma unroll
+  for (int w = 0; w < BN / 32; ++w) {
+    const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 31);
+    if (a <= b) m[w] |= (0xffffffffu >> (31 - b)) & (0xffffffffu << a);
+  }
+}
+
+// Three attention variants of 128 sampled query rows over a range of natural key blocks:
+// dense, spatial (the row's kept natural blocks: whole blocks on or off) and temporal (the
+// row's kept frame-major slots).  All three use the dense running max, so their
+// probabilities are masked copies of the dense ones and each score is exponentiated once:
+// the spatial P.V reads the dense P from TMEM with the rows outside the window disabled, the
+// temporal P.V reads a masked copy from shared memory with rows that have no allowed key in
+// the block disabled.  Contributions more than 2^126 below the dense maximum flush to zero.
 template <int D, int BN>
 __global__ void __launch_bounds__(kProfThreads, 1)
     profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
@@ -181,7 +201,8 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
-  volatile uint32_t* flags = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 16);  // [2][4]
+  // per block parity: [slot][variant 0 = spatial, 1 = temporal][quad] ballots of rows using it
+  volatile uint32_t* rowuse = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 32);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Geom& g = a.g;
@@ -197,14 +218,15 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 
   if (tid == 0) {
     mbar_init(bar(PB_Q), 1);
-    mbar_init(bar(PB_FULL_K), 1);
-    mbar_init(bar(PB_FULL_V), 1);
-    mbar_init(bar(PB_EMPTY_K), 1);
-    mbar_init(bar(PB_EMPTY_V), 1);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(bar(PB_FULL_K + st), 1);
+      mbar_init(bar(PB_FULL_V + st), 1);
+      mbar_init(bar(PB_EMPTY_K + st), 1);
+      mbar_init(bar(PB_EMPTY_V + st), 1);
+    }
     mbar_init(bar(PB_S_FULL), 1);
-    mbar_init(bar(PB_S_FREE), 128);
     mbar_init(bar(PB_P_FULL), 128);
-    mbar_init(bar(PB_O_DONE), 1);
+    mbar_init(bar(PB_O_FINAL), 1);
     mbar_init(bar(PB_DRAIN), 1);
     misc[1] = 0;
     mbar_init_fence();
@@ -225,22 +247,30 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * kPM * 128, &tqs, bar(PB_Q), c * 64, tile * kPM, bh);
       for (int j = 0; j < cnt; ++j) {
-        const int kb = kb0 + j;
-        if (j >= 1 && !mbar_wait(bar(PB_EMPTY_K), (j - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(bar(PB_FULL_K), C::KV_BYTES);
+        const int kb = kb0 + j, st = j & 1;
+        const uint32_t u = j >> 1;
+        if (j >= 2 && !mbar_wait(bar(PB_EMPTY_K + st), (u - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(PB_FULL_K + st), C::KV_BYTES);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_load_3d(sK + c * BN * 128, &tk, bar(PB_FULL_K), c * 64, kb * BN, bh);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sK + st * C::KV_BYTES + c * BN * 128, &tk, bar(PB_FULL_K + st), c * 64, kb * BN, bh);
         nk = j + 1;
-        if (j >= 1 && !mbar_wait(bar(PB_EMPTY_V), (j - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(bar(PB_FULL_V), C::KV_BYTES);
+        if (j >= 2 && !mbar_wait(bar(PB_EMPTY_V + st), (u - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(bar(PB_FULL_V + st), C::KV_BYTES);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_load_3d(sV + c * BN * 128, &tv, bar(PB_FULL_V), c * 64, kb * BN, bh);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sV + st * C::KV_BYTES + c * BN * 128, &tv, bar(PB_FULL_V + st), c * 64, kb * BN, bh);
         nv = j + 1;
       }
       if (*abort_flag) {
         mbar_wait_drain(bar(PB_Q), 0, a.err);
-        if (nk > 0) mbar_wait_drain(bar(PB_FULL_K), (nk - 1) & 1, a.err);
-        if (nv > 0) mbar_wait_drain(bar(PB_FULL_V), (nv - 1) & 1, a.err);
+        for (int st = 0; st < 2; ++st) {
+          int lk = -1, lv = -1;
+          for (int j = st; j < nk; j += 2) lk = j;
+          for (int j = st; j < nv; j += 2) lv = j;
+          if (lk >= 0) mbar_wait_drain(bar(PB_FULL_K + st), (lk >> 1) & 1, a.err);
+          if (lv >= 0) mbar_wait_drain(bar(PB_FULL_V + st), (lv >> 1) & 1, a.err);
+        }
       }
     }
     __syncwarp();
@@ -248,33 +278,51 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     if (lane == 0 && cnt > 0) {
       auto issue_pv = [&](int jp) -> bool {
         if (!mbar_wait(bar(PB_P_FULL), jp & 1, abort_flag, a.err)) return false;
-        if (!mbar_wait(bar(PB_FULL_V), jp & 1, abort_flag, a.err)) return false;
-        // variants that some row of the tile allows in this block (one word per softmax warp)
-        const uint32_t used = flags[(jp & 1) * 4 + 0] | flags[(jp & 1) * 4 + 1] | flags[(jp & 1) * 4 + 2] |
-                              flags[(jp & 1) * 4 + 3];
-        tc_fence_after();
+        if (!mbar_wait(bar(PB_FULL_V + (jp & 1)), (jp >> 1) & 1, abort_flag, a.err)) return false;
+        uint32_t dis_sp[4], dis_tp[4];
+        uint32_t any_sp = 0u, any_tp = 0u;
 #pragma unroll
-        for (int vv = 0; vv < 3; ++vv) {
-          if (!((used >> vv) & 1u)) continue;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t us = rowuse[(jp & 1) * 8 + q], ut = rowuse[(jp & 1) * 8 + 4 + q];
+          dis_sp[q] = ~us;
+          dis_tp[q] = ~ut;
+          any_sp |= us;
+          any_tp |= ut;
+        }
+        tc_fence_after();
+        const uint32_t vbase = sV + (jp & 1) * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+          tc_mma_ts(tmem + C::TMEM_O, tmem + C::TMEM_S + kk * 8, bd, C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (any_sp) {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t ad =
-                sdesc_sw128(sP + vv * C::P_BYTES + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sV + kk * 16 * 128, BN * 128, 1024);
-            tc_mma_ss(tmem + C::TMEM_O + vv * D, ad, bd, C::IDESC_PV, 1u);
+            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+            tc_mma_ts_masked(tmem + C::TMEM_O + D, tmem + C::TMEM_S + kk * 8, bd, C::IDESC_PV, dis_sp, 1u);
           }
         }
-        tc_commit(bar(PB_EMPTY_V));
-        tc_commit(bar(PB_O_DONE));
+        if (any_tp) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sP + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+            tc_mma_ss_masked(tmem + C::TMEM_O + 2 * D, ad, bd, C::IDESC_PV, dis_tp, 1u);
+          }
+        }
+        tc_commit(bar(PB_EMPTY_V + (jp & 1)));
         return true;
       };
       bool ok = mbar_wait(bar(PB_Q), 0, abort_flag, a.err);
       for (int j = 0; ok && j < cnt; ++j) {
-        if (!mbar_wait(bar(PB_FULL_K), j & 1, abort_flag, a.err)) {
+        const int st = j & 1;
+        if (!mbar_wait(bar(PB_FULL_K + st), (j >> 1) & 1, abort_flag, a.err)) {
           ok = false;
           break;
         }
-        if (j >= 1 && !mbar_wait(bar(PB_S_FREE), (j - 1) & 1, abort_flag, a.err)) {
+        // P of the previous block lives over S: its P.V products go first (in-order pipe)
+        if (j >= 1 && !issue_pv(j - 1)) {
           ok = false;
           break;
         }
@@ -282,17 +330,13 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + st * C::KV_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
           tc_mma_ss(tmem + C::TMEM_S, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(PB_EMPTY_K));
+        tc_commit(bar(PB_EMPTY_K + st));
         tc_commit(bar(PB_S_FULL));
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
-        }
       }
-      if (ok) issue_pv(cnt - 1);
+      if (ok && issue_pv(cnt - 1)) tc_commit(bar(PB_O_FINAL));
       tc_commit(bar(PB_DRAIN));
       mbar_wait_drain(bar(PB_DRAIN), 0, a.err);
     }
@@ -301,6 +345,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t t_s = t_lane + C::TMEM_S, t_o = t_lane + C::TMEM_O;
     const float sl2 = a.scale_log2;
     // Allowed keys of this row: spatial = natural tokens [rg.x, rg.y) (whole blocks),
     // temporal = frame-major slots [rg.z, rg.w), i.e. (s, f) from (ts_lo, tf_lo) to (ts_hi, tf_hi).
@@ -308,14 +353,13 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     const bool t_any = rg.w > rg.z;
     const int ts_lo = rg.z / g.F, tf_lo = rg.z - (rg.z / g.F) * g.F;
     const int ts_hi = t_any ? (rg.w - 1) / g.F : -1, tf_hi = t_any ? (rg.w - 1) - ((rg.w - 1) / g.F) * g.F : -1;
-    float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f};
-    // Zero the accumulators: every P.V product accumulates, and skipped ones leave zeros.
-    {
+    float m = -INFINITY, l[3] = {0.f, 0.f, 0.f};
+    {  // the spatial and temporal accumulators only ever accumulate: start them at zero
       float z[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x) z[x] = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 3 * D / 32; ++c) tmem_st32(t_lane + C::TMEM_O + c * 32, z);
+      for (int c = 0; c < 2 * D / 32; ++c) tmem_st32(t_o + D + c * 32, z);
     }
     bool ok = true;
     for (int j = 0; j < cnt; ++j) {
@@ -324,112 +368,105 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       tc_fence_after();
       float s[BN];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + C::TMEM_S + c * 32, s + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar(PB_S_FREE));
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
       const int t0 = (kb0 + j) * BN;
       const int nvalid = min(BN, g.N - t0);
-      // spatial: the block is either inside the row's token range or outside it
+      if (nvalid < BN) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (c >= nvalid) s[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m, mx * sl2);
+      const bool grow = m_new > m + 8.f;
+      // The S_FULL wait also covers the previous block's P.V products (in-order pipe): O is stable.
+      if (j > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
+        const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 3 * D / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] *= alpha;
+          tmem_st32(t_o + c * 32, o);
+        }
+      }
+      if (grow) {
+        const float alpha = fast_exp2(m - m_new);
+        l[0] *= alpha;
+        l[1] *= alpha;
+        l[2] *= alpha;
+        m = m_new;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
+      // masks: spatial whole block; temporal as contiguous column ranges per frame segment
       const bool sp_on = t0 >= rg.x && t0 < rg.y;
-      // temporal: quick reject on the block's position span, then an exact per-column mask
-      const int f_a = t0 / g.S, s_a = t0 - f_a * g.S;
-      const int f_b = (t0 + nvalid - 1) / g.S, s_b = (t0 + nvalid - 1) - f_b * g.S;
-      bool tp_on = t_any;
-      if (tp_on && f_a == f_b) tp_on = s_a <= ts_hi && s_b >= ts_lo;
-      else if (tp_on && f_b == f_a + 1) tp_on = (s_a <= ts_hi) || (s_b >= ts_lo);
       uint32_t mt[BN / 32];
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) mt[w] = 0u;
-      if (tp_on) {
-        int f = f_a, sp = s_a;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const bool in = c < nvalid && (sp > ts_lo || (sp == ts_lo && f >= tf_lo)) &&
-                          (sp < ts_hi || (sp == ts_hi && f <= tf_hi));
-          mt[c >> 5] |= (in ? 1u : 0u) << (c & 31);
-          if (++sp == g.S) {
-            sp = 0;
-            ++f;
-          }
+      if (t_any) {
+        int f = t0 / g.S, s0 = t0 - (t0 / g.S) * g.S;
+        for (int c = 0; c < nvalid;) {
+          const int seg = min(nvalid - c, g.S - s0);
+          const int lo_s = ts_lo + (f < tf_lo ? 1 : 0), hi_s = ts_hi - (f > tf_hi ? 1 : 0);
+          const int x0 = max(lo_s, s0), x1 = min(hi_s, s0 + seg - 1);
+          if (x0 <= x1) set_bit_range<BN>(mt, c + x0 - s0, c + x1 - s0);
+          c += seg;
+          ++f;
+          s0 = 0;
         }
-        uint32_t any = 0u;
-#pragma unroll
-        for (int w = 0; w < BN / 32; ++w) any |= mt[w];
-        tp_on = any != 0u;
       }
-      // per-variant row maxima (raw scores)
-      float mx0 = -INFINITY, mx2 = -INFINITY;
+      uint32_t tany = 0u;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        const float v = c < nvalid ? s[c] : -INFINITY;
-        s[c] = v;
-        mx0 = fmaxf(mx0, v);
-        if ((mt[c >> 5] >> (c & 31)) & 1u) mx2 = fmaxf(mx2, v);
-      }
-      const float mx[3] = {mx0, sp_on ? mx0 : -INFINITY, tp_on ? mx2 : -INFINITY};
-      float mnew[3], muse[3];
+      for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
+      const bool tp_on = tany != 0u;
+      float rs = 0.f, rt = 0.f;
 #pragma unroll
-      for (int vv = 0; vv < 3; ++vv) {
-        mnew[vv] = fmaxf(m[vv], mx[vv] * sl2);
-        muse[vv] = mnew[vv] == -INFINITY ? 0.f : mnew[vv];
-      }
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (j - 1) & 1, abort_flag, a.err));
-        if (!ok) break;
-        tc_fence_after();
+      for (int h = 0; h < BN / 64; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int vv = 0; vv < 3; ++vv) {
-          const float alpha = fast_exp2(m[vv] - muse[vv]);
-          if (__any_sync(0xffffffffu, alpha < 1.f && m[vv] != -INFINITY)) {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              float o[32];
-              tmem_ld32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+        for (int c = 0; c < 32; ++c) {
+          const int col = h * 64 + 2 * c;
+          const float p0 = fast_exp2(fmaf(s[col], sl2, -m_use));
+          const float p1 = fast_exp2(fmaf(s[col + 1], sl2, -m_use));
+          rs += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+          const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
+          rt += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+        }
+        if (tp_on) {  // masked copy for the temporal P.V (K-major, 128-byte swizzle)
 #pragma unroll
-              for (int x = 0; x < 32; ++x) o[x] *= alpha;
-              tmem_st32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 v4;
+            uint32_t* w4 = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const int col = h * 64 + ch * 8 + 2 * x;
+              const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
+              w4[x] = pk[ch * 4 + x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
             }
+            const int kc = (h * 8 + ch) >> 3, cc = (h * 8 + ch) & 7;
+            *reinterpret_cast<uint4*>(pP + kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v4;
           }
-          l[vv] *= alpha;
         }
+        tmem_st32_u(t_s + h * 32, pk);
       }
-      // publish which variants this warp's rows use in this block (read by the MMA issuer)
-      {
-        const uint32_t use = 1u | (__any_sync(0xffffffffu, sp_on) ? 2u : 0u) | (__any_sync(0xffffffffu, tp_on) ? 4u : 0u);
-        if (lane == 0) flags[(j & 1) * 4 + quad] = use;
-      }
-#pragma unroll
-      for (int vv = 0; vv < 3; ++vv) {
-        const bool on = vv == 0 || (vv == 1 ? sp_on : tp_on);
-        float rs = 0.f;
-        uint8_t* pv = pP + vv * C::P_BYTES;
-#pragma unroll
-        for (int ch = 0; ch < BN / 8; ++ch) {
-          float p[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const int c = ch * 8 + x;
-            const bool keep = vv == 2 ? ((mt[c >> 5] >> (c & 31)) & 1u) != 0u : true;
-            p[x] = (on && keep) ? fast_exp2(fmaf(s[c], sl2, -muse[vv])) : 0.f;
-            rs += p[x];
-          }
-          uint4 pk;
-          pk.x = pack_bf16x2(p[0], p[1]);
-          pk.y = pack_bf16x2(p[2], p[3]);
-          pk.z = pack_bf16x2(p[4], p[5]);
-          pk.w = pack_bf16x2(p[6], p[7]);
-          const int kc = ch >> 3, cc = ch & 7;
-          *reinterpret_cast<uint4*>(pv + kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = pk;
-        }
-        l[vv] += rs;
-        m[vv] = mnew[vv];
+      l[0] += rs;
+      if (sp_on) l[1] += rs;
+      l[2] += rt;
+      const uint32_t bs = __ballot_sync(0xffffffffu, sp_on), bt = __ballot_sync(0xffffffffu, tp_on);
+      if (lane == 0) {
+        rowuse[(j & 1) * 8 + quad] = bs;
+        rowuse[(j & 1) * 8 + 4 + quad] = bt;
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(PB_P_FULL));
     }
     if (ok && cnt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_FINAL), 0, abort_flag, a.err));
       tc_fence_after();
     }
     // partials: (m, l) and unnormalised O of each variant
@@ -438,14 +475,14 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     for (int vv = 0; vv < 3; ++vv) {
       const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
       const bool have = ok && cnt > 0;
-      a.ml[prow * 2 + 0] = have ? m[vv] : -INFINITY;
+      a.ml[prow * 2 + 0] = have ? m : -INFINITY;
       a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
       float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
         if (have) {
-          tmem_ld32(t_lane + C::TMEM_O + vv * D + c * 32, o);
+          tmem_ld32(t_o + vv * D + c * 32, o);
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] = 0.f;

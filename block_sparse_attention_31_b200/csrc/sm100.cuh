@@ -159,6 +159,27 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Lane-masked forms: rows (TMEM lanes) whose bit is set in `disable` (lane i -> word i/32,
+// bit i%32) keep their old accumulator values.
+__device__ __forceinline__ void tc_mma_ts_masked(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 const uint32_t (&disable)[4], uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %8, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%4, %5, %6, %7}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(disable[0]), "r"(disable[1]), "r"(disable[2]), "r"(disable[3]),
+      "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_ss_masked(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 const uint32_t (&disable)[4], uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %8, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%4, %5, %6, %7}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(disable[0]), "r"(disable[1]), "r"(disable[2]), "r"(disable[3]),
+      "r"(accumulate)
+      : "memory");
+}
+
 // Store 32 consecutive 32-bit columns of raw bits (one row per thread), waits for completion.
 __device__ __forceinline__ void tmem_st32_u(uint32_t taddr, const uint32_t* r) {
   asm volatile(
