@@ -73,6 +73,7 @@ def _load():
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
+        "vsa_selftest_exp2": (st, [vp, vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -241,3 +242,8 @@ def vsa_get_device_error(err, stream=None) -> int:
     if st not in (VSA_OK, VSA_ERR_DEVICE, VSA_ERR_TIMEOUT):
         raise VsaError(st, "vsa_get_device_error")
     return h.value
+
+
+def vsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
+    _check(lib.vsa_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), int(x.numel()), _stream(stream)),
+           "vsa_selftest_exp2")

@@ -48,13 +48,13 @@ struct AttnCfg {
   static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
   static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_UNION = OFF_MISC + 64;  // union list, then two bitsets
+  static constexpr int OFF_UNION = OFF_MISC + 64;  // union list, two bitsets, key-validity masks
   static constexpr int TMEM_S = 0;                  // S of tile t at t*BN (P aliases its first BN/2 columns)
   static constexpr int TMEM_O = 2 * BN;             // O of tile t at 2*BN + t*D
   static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, false, true);
-  static int smem_bytes(int ucap, int nwords) { return OFF_UNION + 4 * ucap + 8 * nwords + 1024; }
+  static int smem_bytes(int ucap, int nwords) { return OFF_UNION + 4 * ucap + 8 * nwords + 4 * ucap * (BN / 32) + 1024; }
 };
 
 // Barrier slots.
@@ -69,23 +69,9 @@ enum {
   B_O_FINAL = 14,  // +tile
   B_DRAIN = 16
 };
-constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kKbMask = (1u << 30) - 1u;
-
-// Validity of the key columns of block kb for one head: a ragged tail (natural and
-// frame-major layouts) or cube padding slots are not real tokens.
-template <int BN>
-__device__ __forceinline__ void key_valid_bits(const Geom& g, int kind, int kb, uint32_t (&vb)[BN / 32]) {
-#pragma unroll
-  for (int w = 0; w < BN / 32; ++w) {
-    uint32_t m = 0;
-    for (int c = 0; c < 32; ++c) {
-      const int slot = kb * BN + w * 32 + c;
-      const bool ok = kind == kCube ? token_of_slot(g, kCube, slot) >= 0 : slot < g.N;
-      m |= (ok ? 1u : 0u) << c;
-    }
-    vb[w] = m;
-  }
-}
+constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kPartial = 1u << 29, kKbMask = (1u << 29) - 1u;
+// Probability pairs (2 columns) whose exponentials run on the FMA pipe: 1 pair in 8.
+constexpr int kPolyPairMask = 7;
 
 // One CTA per pair of consecutive query blocks (tiles 0 and 1) of one head.  The K/V blocks
 // of the union of the two lists stream through a 2-stage ring once and serve both tiles; the
@@ -113,6 +99,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* uni = reinterpret_cast<uint32_t*>(smem + C::OFF_UNION);
   uint32_t* bits0 = uni + a.ucap;
   uint32_t* bits1 = bits0 + nwords;
+  uint32_t* uvalid = bits1 + nwords;  // [ucap][BN/32] valid-key bits of partial union entries
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Geom& g = a.g;
@@ -192,12 +179,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       while (u) {
         const int b = __ffs(u) - 1;
         u &= u - 1u;
-        uni[pos++] = static_cast<uint32_t>(w * 32 + b) | (((u0 >> b) & 1u) ? kInTile0 : 0u) |
-                     (((u1 >> b) & 1u) ? kInTile1 : 0u);
+        const int kb = w * 32 + b;
+        uni[pos++] = static_cast<uint32_t>(kb) | (((u0 >> b) & 1u) ? kInTile0 : 0u) |
+                     (((u1 >> b) & 1u) ? kInTile1 : 0u) | (block_full(g, kind, kb) ? 0u : kPartial);
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) misc[2] = base;
+    __syncwarp();
+    // valid-key bits of the blocks that are not full (ragged tail, cube padding)
+    for (int n = 0; n < base; ++n) {
+      const uint32_t e = uni[n];
+      if (!(e & kPartial)) continue;
+      const int kb = static_cast<int>(e & kKbMask);
+#pragma unroll
+      for (int w = 0; w < BN / 32; ++w) {
+        const int slot = kb * BN + w * 32 + lane;
+        const bool ok = kind == kCube ? token_of_slot(g, kCube, slot) >= 0 : slot < g.N;
+        const uint32_t m = __ballot_sync(0xffffffffu, ok);
+        if (lane == 0) uvalid[n * (BN / 32) + w] = m;
+      }
+    }
   }
 
   // ---- setup: barriers and TMEM ----
@@ -284,18 +286,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int pvc[2] = {0, 0};      // P.V products issued per tile
       bool qready[2] = {false, false};
       bool ok = true;
+      // Descriptor bases; each K step adds a compile-time offset (in 16-byte units) to the
+      // start-address field, which never carries out of its 14 bits (shared memory < 256 KB).
+      static_assert(C::NS == 2, "descriptor selection below assumes two stages");
+      const uint64_t dq0 = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t dq1 = sdesc_sw128(sbase + C::OFF_Q + C::Q_BYTES, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::KV_BYTES, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::KV_BYTES, BN * 128, 1024);
       auto issue_pv = [&](int t) -> bool {
         const int np = pend[t];
         if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
         if (!mbar_wait(bar(B_FULL_V + np % C::NS), (np / C::NS) & 1, abort_flag, a.err)) return false;
         tc_fence_after();
-        const uint32_t vbase = sV + (np % C::NS) * C::KV_BYTES;
+        const uint64_t vd = (np & 1) ? dv1 : dv0;
+        const uint32_t d_o = tmem + C::TMEM_O + t * D, a_p = tmem + C::TMEM_S + t * BN;
+        tc_mma_ts(d_o, a_p, vd, C::IDESC_PV, pvc[t] > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-          tc_mma_ts(tmem + C::TMEM_O + t * D, tmem + C::TMEM_S + t * BN + kk * 8, bd, C::IDESC_PV,
-                    (pvc[t] > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < BN / 16; ++kk)
+          tc_mma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV, 1u);
         pend[t] = -1;
         if (++pvc[t] == cnts[t]) tc_commit(bar(B_O_FINAL + t));
         return true;
@@ -322,14 +330,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             qready[t] = true;
           }
           tc_fence_after();
-          const uint32_t qbase = sbase + C::OFF_Q + t * C::Q_BYTES;
+          const uint32_t d_s = tmem + C::TMEM_S + t * BN;
+          const uint64_t qd = t ? dq1 : dq0, kd = st ? dk1 : dk0;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(qbase + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                sdesc_sw128(sK + st * C::KV_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
-            tc_mma_ss(tmem + C::TMEM_S + t * BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc_mma_ss(d_s, qd + static_cast<uint64_t>(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) / 16),
+                      kd + static_cast<uint64_t>(((kk >> 2) * (BN * 128) + (kk & 3) * 32) / 16), C::IDESC_QK,
+                      kk > 0 ? 1u : 0u);
           tc_commit(bar(B_S_FULL + t));
           pend[t] = n;
         }
@@ -351,31 +358,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quad * 32 + lane;   // query row within the tile
     if (t == 0 || has1) {
       const int cnt = t ? cnt1 : cnt0;
-      const int32_t* kvl = t ? kvl1 : kvl0;
       const int qb = qb0 + t;
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
       const uint32_t t_s = t_lane + C::TMEM_S + t * BN, t_o = t_lane + C::TMEM_O + t * D;
       const float sl2 = a.scale_log2;
       float m = -INFINITY, l = 0.f;  // m: the (lazily updated) max used for the exponentials
       bool ok = true;
+      int cur = 0;  // cursor into the union list (this tile's entries are the ones with its bit)
+      const uint32_t tbit = t ? kInTile1 : kInTile0;
       for (int k = 0; k < cnt; ++k) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), k & 1, abort_flag, a.err));
         if (!ok) break;
         tc_fence_after();
-        float s[BN];
+        while (!(uni[cur] & tbit)) ++cur;
+        const uint32_t ent = uni[cur];
+        if (ent & kPartial) {  // same block for every row: mask invalid key columns to -inf in TMEM
+#pragma unroll 1
+          for (int w = 0; w < BN / 32; ++w) {
+            const uint32_t vb = uvalid[cur * (BN / 32) + w];
+            if (vb == 0xffffffffu) continue;
+            float v[32];
+            tmem_ld32(t_s + w * 32, v);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
-        const int kb = kvl[k];
-        if (!block_full(g, kind, kb)) {
-          uint32_t vb[BN / 32];
-          key_valid_bits<BN>(g, kind, kb, vb);
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (!((vb[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+            for (int x = 0; x < 32; ++x) v[x] = ((vb >> x) & 1u) ? v[x] : -INFINITY;
+            tmem_st32(t_s + w * 32, v);
+          }
         }
+        ++cur;
+        // pass 1: row max, 64 columns per wait
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int h = 0; h < BN / 64; ++h) {
+          uint32_t r[64];
+          tmem_ld32_async(t_s + h * 64, r);
+          tmem_ld32_async(t_s + h * 64 + 32, r + 32);
+          tmem_wait_ld();
+          reg_fence<64>(r);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+        }
         const float m_new = fmaxf(m, mx * sl2);
         // Rescale only when the running max grows by more than 2^8; otherwise keep the old
         // max (the exponentials stay below 256 and the final 1/l normalisation is exact).
@@ -396,14 +417,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = m_new;
         }
         const float m_use = m == -INFINITY ? 0.f : m;
+        // pass 2: 64 scores at a time -> 32 packed bf16 pairs written over the consumed S columns
         float rs = 0.f;
 #pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {  // 64 probabilities -> 32 packed columns at a time
+        for (int h = 0; h < BN / 64; ++h) {
+          uint32_t r[64];
+          tmem_ld32_async(t_s + h * 64, r);
+          tmem_ld32_async(t_s + h * 64 + 32, r + 32);
+          tmem_wait_ld();
+          reg_fence<64>(r);
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = fast_exp2(fmaf(s[h * 64 + 2 * c], sl2, -m_use));
-            const float p1 = fast_exp2(fmaf(s[h * 64 + 2 * c + 1], sl2, -m_use));
+            const float x0 = fmaf(__uint_as_float(r[2 * c]), sl2, -m_use);
+            const float x1 = fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m_use);
+            const bool poly = (c & kPolyPairMask) == kPolyPairMask;
+            const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
+            const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
             rs += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }

@@ -1,0 +1,26 @@
+// selftest.cu -- device-side checks exposed for the test suite (not part of an attention call).
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+#include "vsa.h"
+
+namespace vsa {
+
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                     float* __restrict__ y_mufu, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    y_poly[i] = exp2_poly(x[i]);
+    y_mufu[i] = fast_exp2(x[i]);
+  }
+}
+
+}  // namespace vsa
+
+extern "C" vsa_status vsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int n, cudaStream_t stream) {
+  if (x == nullptr || y_poly == nullptr || y_mufu == nullptr || n < 0) return VSA_ERR_INVALID_ARG;
+  if (n == 0) return VSA_OK;
+  vsa::exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y_poly, y_mufu, n);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}

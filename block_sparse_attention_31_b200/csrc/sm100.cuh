@@ -226,6 +226,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Issue a 32-column TMEM load without waiting; the registers are valid only after
+// tmem_wait_ld() followed by reg_fence() on them.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Tell the compiler that registers filled by asynchronous loads change at this point, so no
+// use of them is scheduled before the preceding wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   uint32_t r[32];
 #pragma unroll
@@ -241,11 +263,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// Per-warpgroup register rebalancing (all four warps of a warpgroup execute the same one).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+
 // Hardware base-2 exponential (MUFU), flushes denormals; ex2(-inf) = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes, to offload part of the exponentials from the MUFU unit.
+// x = n + f with n = round(x) (adding 1.5*2^23 leaves n in the low mantissa bits) and
+// f in [-0.5, 0.5]; 2^f is a minimax cubic (coefficients from csrc/fit_exp2_poly.py, max
+// relative error 7.5e-5) and 2^n is added to the exponent field.  Returns 0 for x < -125;
+// valid up to x = 127.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float magic = 12582912.0f;
+  const float xc = fmaxf(x, -125.0f);
+  const float t = __fadd_rn(xc, magic);
+  const float f = __fsub_rn(xc, __fsub_rn(t, magic));
+  const float p = fmaf(fmaf(fmaf(0.05517149344086647f, f, 0.24261093139648438f), f, 0.6932609677314758f), f,
+                       0.9999280571937561f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -125.0f ? 0.0f : r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -254,6 +254,11 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
                                           vsa_select select, size_t *off_bits, size_t *off_kv_idx,
                                           size_t *off_kv_cnt, int *max_kv);
 
+/* Self-test hook (the pages have no counterpart): evaluates the kernels' two base-2
+ * exponentials, the FMA-pipe polynomial (y_poly) and the hardware approximation (y_mufu),
+ * on n device floats, so that tests can bound the polynomial's error. */
+VSA_API vsa_status vsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, cudaStream_t stream);
+
 /* Synchronise `stream`, copy the device error word to *host_err and map it to a status
  * (VSA_OK when zero, VSA_ERR_TIMEOUT when the timeout bit is set, else VSA_ERR_DEVICE). */
 VSA_API vsa_status vsa_get_device_error(const int *d_err, cudaStream_t stream, int *host_err);
