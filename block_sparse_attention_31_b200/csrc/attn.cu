@@ -369,9 +369,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int k = 0; k < cnt; ++k) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), k & 1, abort_flag, a.err));
         if (!ok) break;
-        tc_fence_after();
         while (!(uni[cur] & tbit)) ++cur;
         const uint32_t ent = uni[cur];
+        tc_fence_after();
         if (ent & kPartial) {  // same block for every row: mask invalid key columns to -inf in TMEM
 #pragma unroll 1
           for (int w = 0; w < BN / 32; ++w) {
@@ -385,8 +385,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         ++cur;
-        // pass 1: row max, 64 columns per wait
-        float mx = -INFINITY;
+        // pass 1: row max, 64 columns per wait; eight independent partial maxima keep the
+        // dependency chains short
+        float mx8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
 #pragma unroll
         for (int h = 0; h < BN / 64; ++h) {
           uint32_t r[64];
@@ -395,8 +398,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_ld();
           reg_fence<64>(r);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m, mx * sl2);
         // Rescale only when the running max grows by more than 2^8; otherwise keep the old
         // max (the exponentials stay below 256 and the final 1/l normalisation is exact).
@@ -417,8 +422,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = m_new;
         }
         const float m_use = m == -INFINITY ? 0.f : m;
-        // pass 2: 64 scores at a time -> 32 packed bf16 pairs written over the consumed S columns
-        float rs = 0.f;
+        // pass 2: 64 scores at a time -> 32 packed bf16 pairs written over the consumed S columns;
+        // the row sum is kept in eight partial sums
+        float rs8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) rs8[x] = 0.f;
 #pragma unroll
         for (int h = 0; h < BN / 64; ++h) {
           uint32_t r[64];
@@ -434,12 +442,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const bool poly = (c & kPolyPairMask) == kPolyPairMask;
             const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
             const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
-            rs += p0 + p1;
+            rs8[(2 * c) & 7] += p0;
+            rs8[(2 * c + 1) & 7] += p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st32_u(t_s + h * 32, pk);
         }
-        l += rs;
+        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL + t));
       }

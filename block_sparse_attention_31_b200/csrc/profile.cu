@@ -376,9 +376,13 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         for (int c = 0; c < BN; ++c)
           if (c >= nvalid) s[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx * sl2);
       const bool grow = m_new > m + 8.f;
       // The S_FULL wait also covers the previous block's P.V products (in-order pipe): O is stable.
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
       const bool tp_on = tany != 0u;
-      float rs = 0.f, rt = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f}, rt4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < BN / 64; ++h) {
         uint32_t pk[32];
@@ -431,10 +435,10 @@ __global__ void __launch_bounds__(kProfThreads, 1)
           const int col = h * 64 + 2 * c;
           const float p0 = fast_exp2(fmaf(s[col], sl2, -m_use));
           const float p1 = fast_exp2(fmaf(s[col + 1], sl2, -m_use));
-          rs += p0 + p1;
+          rs4[c & 3] += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
           const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-          rt += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+          rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
         }
         if (tp_on) {  // masked copy for the temporal P.V (K-major, 128-byte swizzle)
 #pragma unroll
@@ -453,6 +457,8 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         }
         tmem_st32_u(t_s + h * 32, pk);
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      const float rt = (rt4[0] + rt4[1]) + (rt4[2] + rt4[3]);
       l[0] += rs;
       if (sp_on) l[1] += rs;
       l[2] += rt;
