@@ -89,7 +89,8 @@ cudaError_t launch_pattern_mask(const uint8_t* kinds, const Geom& g, int BH, int
 // ---------------------------------------------------------------------------------------
 constexpr int kPoolThreads = 64;
 
-// One CTA per (cube, head); thread x owns dimensions 2x, 2x+1 (+128 per pass).
+// One CTA per (cube, head); thread x owns dimensions 2x, 2x+1 (+128 per pass).  The sums run
+// over the cube's real tokens in slot order, i.e. increasing natural token index.
 __global__ void __launch_bounds__(kPoolThreads) cube_pool_kernel(const __nv_bfloat16* __restrict__ qc,
                                                                  const __nv_bfloat16* __restrict__ kc,
                                                                  const uint8_t* __restrict__ kinds, Geom g, int d,
@@ -97,21 +98,24 @@ __global__ void __launch_bounds__(kPoolThreads) cube_pool_kernel(const __nv_bflo
                                                                  double* __restrict__ kbar) {
   const int cube = blockIdx.x, bh = blockIdx.y;
   if (kinds[bh] != kCube) return;
-  const int count = cube_tokens(g, cube);
+  const int cw_i = cube % g.ncw, ch_i = (cube / g.ncw) % g.nch, cf_i = cube / (g.ncw * g.nch);
+  const int nf = min(g.cf, g.F - cf_i * g.cf), nh = min(g.ch, g.Hl - ch_i * g.ch), nw = min(g.cw, g.Wl - cw_i * g.cw);
+  const double n = static_cast<double>(nf * nh * nw);
   const size_t base = (static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol) * d;
   const size_t out = (static_cast<size_t>(bh) * g.ncubes + cube) * d;
   for (int x = threadIdx.x * 2; x < d; x += kPoolThreads * 2) {
     double sq0 = 0.0, sq1 = 0.0, sk0 = 0.0, sk1 = 0.0;
-    for (int r = 0; r < g.vol; ++r) {
-      if (token_of_slot(g, kCube, cube * g.vol + r) < 0) continue;
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(qc + base + static_cast<size_t>(r) * d + x);
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(kc + base + static_cast<size_t>(r) * d + x);
-      sq0 = __dadd_rn(sq0, static_cast<double>(__low2float(a)));
-      sq1 = __dadd_rn(sq1, static_cast<double>(__high2float(a)));
-      sk0 = __dadd_rn(sk0, static_cast<double>(__low2float(b)));
-      sk1 = __dadd_rn(sk1, static_cast<double>(__high2float(b)));
-    }
-    const double n = static_cast<double>(count);
+    for (int df = 0; df < nf; ++df)
+      for (int dh = 0; dh < nh; ++dh)
+        for (int dw = 0; dw < nw; ++dw) {
+          const size_t r = static_cast<size_t>((df * g.ch + dh) * g.cw + dw);
+          const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(qc + base + r * d + x);
+          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(kc + base + r * d + x);
+          sq0 = __dadd_rn(sq0, static_cast<double>(__low2float(a)));
+          sq1 = __dadd_rn(sq1, static_cast<double>(__high2float(a)));
+          sk0 = __dadd_rn(sk0, static_cast<double>(__low2float(b)));
+          sk1 = __dadd_rn(sk1, static_cast<double>(__high2float(b)));
+        }
     qbar[out + x] = __ddiv_rn(sq0, n);
     qbar[out + x + 1] = __ddiv_rn(sq1, n);
     kbar[out + x] = __ddiv_rn(sk0, n);
@@ -119,63 +123,94 @@ __global__ void __launch_bounds__(kPoolThreads) cube_pool_kernel(const __nv_bflo
   }
 }
 
-constexpr int kTopkRows = 8;       // query cubes per CTA (one warp each for the selection)
-constexpr int kTopkChunk = 32;     // key cubes staged per pass
-constexpr int kTopkThreads = 256;  // kTopkRows * 32
+// Coarse scores S[c][c'] = qbar_c . kbar_c' of one head: 64 x 64 outputs per CTA, 4 x 4 per
+// thread (rows ty + 16i, columns tx + 16j), dimensions staged 32 at a time in shared memory
+// (transposed, so a warp's column reads are consecutive).  Every output accumulates its
+// products in dimension order with separately rounded multiply and add.
+constexpr int kScoreTile = 64, kScoreK = 32;
 
-static size_t topk_smem_bytes(int C, int d, int nwords) {
-  return sizeof(double) * (static_cast<size_t>(kTopkRows) * C + static_cast<size_t>(kTopkRows) * d +
-                           static_cast<size_t>(kTopkChunk) * (d + 1)) +
-         sizeof(uint32_t) * static_cast<size_t>(kTopkRows) * nwords;
+__global__ void __launch_bounds__(256) cube_score_kernel(const double* __restrict__ qbar,
+                                                         const double* __restrict__ kbar,
+                                                         const uint8_t* __restrict__ kinds, int C, int d,
+                                                         double* __restrict__ scores) {
+  __shared__ double sq[kScoreK][kScoreTile + 1];
+  __shared__ double sk[kScoreK][kScoreTile + 1];
+  const int bh = blockIdx.z;
+  if (kinds[bh] != kCube) return;
+  const int r0 = blockIdx.y * kScoreTile, c0 = blockIdx.x * kScoreTile;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const double* qh = qbar + static_cast<size_t>(bh) * C * d;
+  const double* kh = kbar + static_cast<size_t>(bh) * C * d;
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int e0 = 0; e0 < d; e0 += kScoreK) {
+    __syncthreads();
+    for (int x = tid; x < kScoreTile * kScoreK; x += 256) {
+      const int r = x / kScoreK, e = x - r * kScoreK;
+      sq[e][r] = r0 + r < C ? qh[static_cast<size_t>(r0 + r) * d + e0 + e] : 0.0;
+      sk[e][r] = c0 + r < C ? kh[static_cast<size_t>(c0 + r) * d + e0 + e] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int e = 0; e < kScoreK; ++e) {
+      double a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = sq[e][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = sk[e][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __dadd_rn(acc[i][j], __dmul_rn(a[i], b[j]));
+    }
+  }
+  double* sh = scores + static_cast<size_t>(bh) * C * C;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty + 16 * i;
+    if (r >= C) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx + 16 * j;
+      if (c < C) sh[static_cast<size_t>(r) * C + c] = acc[i][j];
+    }
+  }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) cube_topk_kernel(const double* __restrict__ qbar,
-                                                                 const double* __restrict__ kbar,
-                                                                 const uint8_t* __restrict__ kinds, Geom g, int d,
-                                                                 int topk, uint32_t* __restrict__ bits,
-                                                                 int32_t* __restrict__ kv_idx,
-                                                                 int32_t* __restrict__ kv_cnt, int max_kv, int* err) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+// Top-k of one score row per warp (score descending, ties to the smaller index) plus the own
+// cube; emits the bitset, the ascending list and the count.
+constexpr int kTopkWarps = 4;
+
+__global__ void __launch_bounds__(kTopkWarps * 32) cube_topk_kernel(const double* __restrict__ scores,
+                                                                    const uint8_t* __restrict__ kinds, Geom g,
+                                                                    int topk, uint32_t* __restrict__ bits,
+                                                                    int32_t* __restrict__ kv_idx,
+                                                                    int32_t* __restrict__ kv_cnt, int max_kv,
+                                                                    int* err) {
+  extern __shared__ __align__(16) uint8_t topk_smem[];  // [kTopkWarps][C] doubles, then [kTopkWarps][nwords]
   const int bh = blockIdx.y;
   if (kinds[bh] != kCube) return;
   const int C = g.ncubes;
   const int nwords = (g.nblk + 31) >> 5;
-  const int row0 = blockIdx.x * kTopkRows;
-  double* sc = reinterpret_cast<double*>(smem_raw);  // [kTopkRows][C]
-  double* qs = sc + static_cast<size_t>(kTopkRows) * C;  // [kTopkRows][d]
-  double* ks = qs + static_cast<size_t>(kTopkRows) * d;  // [kTopkChunk][d + 1]
-  uint32_t* sel = reinterpret_cast<uint32_t*>(ks + static_cast<size_t>(kTopkChunk) * (d + 1));  // [rows][nwords]
-  const int tid = threadIdx.x;
-  for (int x = tid; x < kTopkRows * d; x += kTopkThreads) {
-    const int r = x / d, c = x - r * d;
-    qs[x] = row0 + r < C ? qbar[(static_cast<size_t>(bh) * C + row0 + r) * d + c] : 0.0;
-  }
-  for (int x = tid; x < kTopkRows * nwords; x += kTopkThreads) sel[x] = 0u;
-  const int r = tid >> 5, lane = tid & 31;
-  for (int c0 = 0; c0 < C; c0 += kTopkChunk) {
-    __syncthreads();
-    for (int x = tid; x < kTopkChunk * d; x += kTopkThreads) {
-      const int c = x / d, e = x - c * d;
-      ks[c * (d + 1) + e] = c0 + c < C ? kbar[(static_cast<size_t>(bh) * C + c0 + c) * d + e] : 0.0;
-    }
-    __syncthreads();
-    if (c0 + lane < C) {
-      double acc = 0.0;
-      for (int e = 0; e < d; ++e) acc = __dadd_rn(acc, __dmul_rn(qs[r * d + e], ks[lane * (d + 1) + e]));
-      sc[static_cast<size_t>(r) * C + c0 + lane] = acc;
-    }
-  }
-  __syncthreads();
-  const int row = row0 + r;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kTopkWarps + warp;
+  double* srow = reinterpret_cast<double*>(topk_smem) + static_cast<size_t>(warp) * C;
+  uint32_t* sel = reinterpret_cast<uint32_t*>(reinterpret_cast<double*>(topk_smem) + static_cast<size_t>(kTopkWarps) * C) +
+                  warp * nwords;
+  for (int x = lane; x < nwords; x += 32) sel[x] = 0u;
   if (row >= C) return;
-  const double* srow = sc + static_cast<size_t>(r) * C;
-  uint32_t* srow_sel = sel + r * nwords;
+  const double* grow = scores + (static_cast<size_t>(bh) * C + row) * C;
+  for (int c = lane; c < C; c += 32) srow[c] = __ldg(grow + c);
+  __syncwarp();
   const int picks = topk < C ? topk : C;
   for (int p = 0; p < picks; ++p) {
     double best = -DBL_MAX;
     int best_c = 0x7fffffff;
     for (int c = lane; c < C; c += 32) {
-      if ((srow_sel[c >> 5] >> (c & 31)) & 1u) continue;
+      if ((sel[c >> 5] >> (c & 31)) & 1u) continue;
       const double s = srow[c];
       if (s > best || (s == best && c < best_c)) {
         best = s;
@@ -191,54 +226,73 @@ __global__ void __launch_bounds__(kTopkThreads) cube_topk_kernel(const double* _
         best_c = oc;
       }
     }
-    if (lane == 0 && best_c < C) srow_sel[best_c >> 5] |= 1u << (best_c & 31);
+    if (lane == 0 && best_c < C) sel[best_c >> 5] |= 1u << (best_c & 31);
     __syncwarp();
   }
-  if (lane == 0) srow_sel[row >> 5] |= 1u << (row & 31);
+  if (lane == 0) sel[row >> 5] |= 1u << (row & 31);
   __syncwarp();
   const size_t orow = static_cast<size_t>(bh) * g.nblk + row;
-  for (int x = lane; x < nwords; x += 32) bits[orow * nwords + x] = srow_sel[x];
-  if (lane == 0) {
-    int n = 0;
-    int32_t* irow = kv_idx + orow * max_kv;
-    for (int wd = 0; wd < nwords; ++wd) {
-      uint32_t m = srow_sel[wd];
-      while (m) {
-        const int b = __ffs(m) - 1;
-        m &= m - 1u;
-        if (n < max_kv) irow[n] = wd * 32 + b;
-        ++n;
-      }
+  for (int x = lane; x < nwords; x += 32) bits[orow * nwords + x] = sel[x];
+  // ascending list: per word prefix counts across the warp
+  int32_t* irow = kv_idx + orow * max_kv;
+  int base = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t m = w < nwords ? sel[w] : 0u;
+    const int c = __popc(m);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += n;
     }
-    for (int x = n; x < max_kv; ++x) irow[x] = -1;
-    kv_cnt[orow] = n;
-    if (n > max_kv) atomicOr(err, kDevErrOverflow);
+    int pos = base + incl - c;
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1u;
+      if (pos < max_kv) irow[pos] = w * 32 + b;
+      ++pos;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  for (int x = base + lane; x < max_kv; x += 32) irow[x] = -1;
+  if (lane == 0) {
+    kv_cnt[orow] = base;
+    if (base > max_kv) atomicOr(err, kDevErrOverflow);
   }
 }
 
 size_t cube_mask_workspace_bytes(const Geom& g, int BH, int d) {
-  return 2 * sizeof(double) * static_cast<size_t>(BH) * g.ncubes * d;
+  return sizeof(double) * (2 * static_cast<size_t>(BH) * g.ncubes * d +
+                           static_cast<size_t>(BH) * g.ncubes * g.ncubes);
 }
 
 cudaError_t launch_cube_mask(const uint8_t* kinds, const void* q_cube, const void* k_cube, const Geom& g, int BH, int d,
                              int topk, uint32_t* bits, int32_t* kv_idx, int32_t* kv_cnt, int max_kv, void* ws,
                              int* err, cudaStream_t stream) {
+  const int C = g.ncubes;
   double* qbar = static_cast<double*>(ws);
-  double* kbar = qbar + static_cast<size_t>(BH) * g.ncubes * d;
-  cube_pool_kernel<<<dim3(g.ncubes, BH), kPoolThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q_cube),
-                                                                     static_cast<const __nv_bfloat16*>(k_cube), kinds,
-                                                                     g, d, qbar, kbar);
+  double* kbar = qbar + static_cast<size_t>(BH) * C * d;
+  double* scores = kbar + static_cast<size_t>(BH) * C * d;
+  cube_pool_kernel<<<dim3(C, BH), kPoolThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q_cube),
+                                                              static_cast<const __nv_bfloat16*>(k_cube), kinds, g, d,
+                                                              qbar, kbar);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nwords = (g.nblk + 31) >> 5;
-  const size_t smem = topk_smem_bytes(g.ncubes, d, nwords);
-  e = cudaFuncSetAttribute(cube_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const int nt = (C + kScoreTile - 1) / kScoreTile;
+  cube_score_kernel<<<dim3(nt, nt, BH), 256, 0, stream>>>(qbar, kbar, kinds, C, d, scores);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  cube_topk_kernel<<<dim3((g.ncubes + kTopkRows - 1) / kTopkRows, BH), kTopkThreads, smem, stream>>>(
-      qbar, kbar, kinds, g, d, topk, bits, kv_idx, kv_cnt, max_kv, err);
+  const int nwords = (g.nblk + 31) >> 5;
+  const size_t smem = sizeof(double) * kTopkWarps * C + sizeof(uint32_t) * kTopkWarps * nwords;
+  if (smem > 232448) return cudaErrorInvalidConfiguration;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(cube_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  cube_topk_kernel<<<dim3((C + kTopkWarps - 1) / kTopkWarps, BH), kTopkWarps * 32, smem, stream>>>(
+      scores, kinds, g, topk, bits, kv_idx, kv_cnt, max_kv, err);
   return cudaGetLastError();
 }
-
-size_t cube_topk_smem_bytes(const Geom& g, int d) { return topk_smem_bytes(g.ncubes, d, (g.nblk + 31) >> 5); }
 
 }  // namespace vsa

@@ -133,7 +133,8 @@ VSA_API vsa_status vsa_max_kv(const vsa_shape *shape, const vsa_params *params, 
 /* Profiling rows r = ceil(profile_frac * N) clamped to [1, N]. */
 VSA_API vsa_status vsa_profile_rows(const vsa_shape *shape, const vsa_params *params, int *rows);
 
-/* Workspace bytes of vsa_profile_heads / vsa_build_mask / vsa_attention. */
+/* Workspace bytes of vsa_profile_heads / vsa_build_mask / vsa_attention.  For cube shapes the
+ * mask workspace holds the fp64 pooled means (2*B*H*C*d) and coarse scores (B*H*C*C). */
 VSA_API size_t vsa_profile_workspace_size(const vsa_shape *shape, const vsa_params *params);
 VSA_API size_t vsa_mask_workspace_size(const vsa_shape *shape, const vsa_params *params);
 VSA_API size_t vsa_attention_workspace_size(const vsa_shape *shape, const vsa_params *params, vsa_dtype dtype,

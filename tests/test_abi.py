@@ -58,7 +58,7 @@ def test_cube_shape_helpers():
     assert _lib.vsa_layout_rows(shape) == oracle.layout_rows(oracle.CUBE, wl.F, wl.Hl, wl.Wl, wl.cube) == 229376
     assert _lib.vsa_num_blocks(shape) == 1792
     assert _lib.vsa_max_kv(shape, _lib.make_params(0, 0, topk=32)) >= 33
-    assert _lib.vsa_mask_workspace_size(shape, _lib.make_params(topk=32)) == 2 * 8 * 12 * 1792 * 128
+    assert _lib.vsa_mask_workspace_size(shape, _lib.make_params(topk=32)) == 8 * (2 * 12 * 1792 * 128 + 12 * 1792 * 1792)
 
 
 @pytest.mark.parametrize("N", [256, 32760, 118800, 7 * 5 * 9])
