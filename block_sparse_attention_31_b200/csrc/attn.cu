@@ -14,7 +14,7 @@
 //                       while the other tile's softmax runs.  Warp 1 also owns TMEM.
 //   warps 2-5 / 6-9     softmax of tile 0 / tile 1, one query row per thread (TMEM lane = row):
 //                       S from TMEM, online max in the base-2 domain with lazy rescaling of O
-//                       (only when the max grows by more than 2^8), P = exp2(S*scale*log2e - m)
+//                       (only when the max grows by more than 2^16), P = exp2(S*scale*log2e - m)
 //                       written as packed bf16 over the tile's S columns in TMEM, where the
 //                       P.V MMA reads it; at the end O / l goes through shared memory to a TMA
 //                       store.
@@ -403,9 +403,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m, mx * sl2);
-        // Rescale only when the running max grows by more than 2^8; otherwise keep the old
-        // max (the exponentials stay below 256 and the final 1/l normalisation is exact).
-        const bool grow = m_new > m + 8.f;
+        // Rescale only when the running max grows by more than 2^kRescaleLog2; otherwise keep the
+        // old max (the final 1/l normalisation is exact either way).
+        const bool grow = m_new > m + kRescaleLog2;
         if (k > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
           const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
 #pragma unroll 1

@@ -143,22 +143,23 @@ struct ProfCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int P_BYTES = kPM * BN * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;      // 2 stages
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES; // 2 stages
-  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES; // temporal-masked P
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;       // 2 stages
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // 2 stages
+  static constexpr int OFF_PD = OFF_V + 2 * KV_BYTES; // dense P
+  static constexpr int OFF_PT = OFF_PD + P_BYTES;     // temporal-masked P
+  static constexpr int OFF_BAR = OFF_PT + P_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
   static constexpr int BYTES = OFF_MISC + 128;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
-  // TMEM: S (dense P packed over its first BN/2 columns), then O of dense, spatial, temporal
+  // TMEM: S, then O of dense, spatial, temporal
   static constexpr int TMEM_S = 0, TMEM_O = BN;
   static constexpr int TMEM_COLS = (BN + 3 * D) <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kPM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kPM, D, false, true);
 };
 
-enum { PB_Q = 0, PB_FULL_K = 1, PB_FULL_V = 3, PB_EMPTY_K = 5, PB_EMPTY_V = 7, PB_S_FULL = 9, PB_P_FULL = 10,
-       PB_O_FINAL = 11, PB_DRAIN = 12 };
+enum { PB_Q = 0, PB_FULL_K = 1, PB_FULL_V = 3, PB_EMPTY_K = 5, PB_EMPTY_V = 7, PB_S_FULL = 9, PB_S_FREE = 10,
+       PB_P_FULL = 11, PB_O_DONE = 12, PB_DRAIN = 13 };
 
 struct ProfArgs {
   const int4* ranges;
@@ -183,10 +184,12 @@ __device__ __forceinline__ void set_bit_range(uint32_t (&m)[BN / 32], int lo, in
 // Three attention variants of 128 sampled query rows over a range of natural key blocks:
 // dense, spatial (the row's kept natural blocks: whole blocks on or off) and temporal (the
 // row's kept frame-major slots).  All three use the dense running max, so their
-// probabilities are masked copies of the dense ones and each score is exponentiated once:
-// the spatial P.V reads the dense P from TMEM with the rows outside the window disabled, the
-// temporal P.V reads a masked copy from shared memory with rows that have no allowed key in
-// the block disabled.  Contributions more than 2^126 below the dense maximum flush to zero.
+// probabilities are masked copies of the dense ones and each score is exponentiated once.
+// The spatial P.V reads the dense P with the rows outside the window disabled (the MMA's
+// output-lane mask); the temporal P.V reads a masked copy with rows that allow no key of the
+// block disabled.  Contributions more than 2^126 below the dense maximum flush to zero.
+// Both P tiles live in shared memory so that Q.K^T of block j+1 runs while the softmax of
+// block j computes.
 template <int D, int BN>
 __global__ void __launch_bounds__(kProfThreads, 1)
     profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
@@ -196,8 +199,10 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw_u32);
-  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sP = sbase + C::OFF_P;
-  uint8_t* pP = smem + C::OFF_P;
+  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+  const uint32_t sPD = sbase + C::OFF_PD, sPT = sbase + C::OFF_PT;
+  uint8_t* pPD = smem + C::OFF_PD;
+  uint8_t* pPT = smem + C::OFF_PT;
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
@@ -225,8 +230,9 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       mbar_init(bar(PB_EMPTY_V + st), 1);
     }
     mbar_init(bar(PB_S_FULL), 1);
+    mbar_init(bar(PB_S_FREE), 128);
     mbar_init(bar(PB_P_FULL), 128);
-    mbar_init(bar(PB_O_FINAL), 1);
+    mbar_init(bar(PB_O_DONE), 1);
     mbar_init(bar(PB_DRAIN), 1);
     misc[1] = 0;
     mbar_init_fence();
@@ -276,6 +282,24 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && cnt > 0) {
+      const uint64_t dq = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::KV_BYTES, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::KV_BYTES, BN * 128, 1024);
+      const uint64_t dpd = sdesc_sw128(sPD, 16, 1024), dpt = sdesc_sw128(sPT, 16, 1024);
+      auto issue_qk = [&](int j) -> bool {
+        if (!mbar_wait(bar(PB_FULL_K + (j & 1)), (j >> 1) & 1, abort_flag, a.err)) return false;
+        if (j >= 1 && !mbar_wait(bar(PB_S_FREE), (j - 1) & 1, abort_flag, a.err)) return false;
+        tc_fence_after();
+        const uint64_t kd = (j & 1) ? dk1 : dk0;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ss(tmem + C::TMEM_S, dq + static_cast<uint64_t>(((kk >> 2) * (kPM * 128) + (kk & 3) * 32) / 16),
+                    kd + static_cast<uint64_t>(((kk >> 2) * (BN * 128) + (kk & 3) * 32) / 16), C::IDESC_QK,
+                    kk > 0 ? 1u : 0u);
+        tc_commit(bar(PB_EMPTY_K + (j & 1)));
+        tc_commit(bar(PB_S_FULL));
+        return true;
+      };
       auto issue_pv = [&](int jp) -> bool {
         if (!mbar_wait(bar(PB_P_FULL), jp & 1, abort_flag, a.err)) return false;
         if (!mbar_wait(bar(PB_FULL_V + (jp & 1)), (jp >> 1) & 1, abort_flag, a.err)) return false;
@@ -290,53 +314,42 @@ __global__ void __launch_bounds__(kProfThreads, 1)
           any_tp |= ut;
         }
         tc_fence_after();
-        const uint32_t vbase = sV + (jp & 1) * C::KV_BYTES;
+        const uint64_t vd = (jp & 1) ? dv1 : dv0;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-          tc_mma_ts(tmem + C::TMEM_O, tmem + C::TMEM_S + kk * 8, bd, C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t poff = static_cast<uint64_t>(((kk >> 2) * (kPM * 128) + (kk & 3) * 32) / 16);
+          tc_mma_ss(tmem + C::TMEM_O, dpd + poff, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV,
+                    (jp > 0 || kk > 0) ? 1u : 0u);
         }
         if (any_sp) {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-            tc_mma_ts_masked(tmem + C::TMEM_O + D, tmem + C::TMEM_S + kk * 8, bd, C::IDESC_PV, dis_sp, 1u);
+            const uint64_t poff = static_cast<uint64_t>(((kk >> 2) * (kPM * 128) + (kk & 3) * 32) / 16);
+            tc_mma_ss_masked(tmem + C::TMEM_O + D, dpd + poff, vd + static_cast<uint64_t>(kk * 16 * 128 / 16),
+                             C::IDESC_PV, dis_sp, 1u);
           }
         }
         if (any_tp) {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sP + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-            tc_mma_ss_masked(tmem + C::TMEM_O + 2 * D, ad, bd, C::IDESC_PV, dis_tp, 1u);
+            const uint64_t poff = static_cast<uint64_t>(((kk >> 2) * (kPM * 128) + (kk & 3) * 32) / 16);
+            tc_mma_ss_masked(tmem + C::TMEM_O + 2 * D, dpt + poff, vd + static_cast<uint64_t>(kk * 16 * 128 / 16),
+                             C::IDESC_PV, dis_tp, 1u);
           }
         }
         tc_commit(bar(PB_EMPTY_V + (jp & 1)));
+        tc_commit(bar(PB_O_DONE));
         return true;
       };
-      bool ok = mbar_wait(bar(PB_Q), 0, abort_flag, a.err);
+      bool ok = mbar_wait(bar(PB_Q), 0, abort_flag, a.err) && issue_qk(0);
       for (int j = 0; ok && j < cnt; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(bar(PB_FULL_K + st), (j >> 1) & 1, abort_flag, a.err)) {
+        // Q.K^T of the next block first: it overlaps this block's softmax
+        if (j + 1 < cnt && !issue_qk(j + 1)) {
           ok = false;
           break;
         }
-        // P of the previous block lives over S: its P.V products go first (in-order pipe)
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kPM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + st * C::KV_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
-          tc_mma_ss(tmem + C::TMEM_S, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(PB_EMPTY_K + st));
-        tc_commit(bar(PB_S_FULL));
+        if (!issue_pv(j)) ok = false;
       }
-      if (ok && issue_pv(cnt - 1)) tc_commit(bar(PB_O_FINAL));
       tc_commit(bar(PB_DRAIN));
       mbar_wait_drain(bar(PB_DRAIN), 0, a.err);
     }
@@ -369,6 +382,8 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       float s[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
+      tc_fence_before();
+      mbar_arrive(bar(PB_S_FREE));  // S may be overwritten by the next block's Q.K^T
       const int t0 = (kb0 + j) * BN;
       const int nvalid = min(BN, g.N - t0);
       if (nvalid < BN) {
@@ -384,27 +399,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx * sl2);
-      const bool grow = m_new > m + 8.f;
-      // The S_FULL wait also covers the previous block's P.V products (in-order pipe): O is stable.
-      if (j > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
-        const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < 3 * D / 32; ++c) {
-          float o[32];
-          tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] *= alpha;
-          tmem_st32(t_o + c * 32, o);
-        }
-      }
-      if (grow) {
-        const float alpha = fast_exp2(m - m_new);
-        l[0] *= alpha;
-        l[1] *= alpha;
-        l[2] *= alpha;
-        m = m_new;
-      }
-      const float m_use = m == -INFINITY ? 0.f : m;
+      const bool grow = m_new > m + kRescaleLog2;
       // masks: spatial whole block; temporal as contiguous column ranges per frame segment
       const bool sp_on = t0 >= rg.x && t0 < rg.y;
       uint32_t mt[BN / 32];
@@ -426,36 +421,63 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
       const bool tp_on = tany != 0u;
+      // the previous block's P.V products must be done: O stable, P tiles free
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (j - 1) & 1, abort_flag, a.err));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
+        const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 3 * D / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] *= alpha;
+          tmem_st32(t_o + c * 32, o);
+        }
+      }
+      if (grow) {
+        const float alpha = fast_exp2(m - m_new);
+        l[0] *= alpha;
+        l[1] *= alpha;
+        l[2] *= alpha;
+        m = m_new;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
+      const bool warp_tp = __any_sync(0xffffffffu, tp_on);
       float rs4[4] = {0.f, 0.f, 0.f, 0.f}, rt4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < BN / 64; ++h) {
-        uint32_t pk[32];
+      for (int ch = 0; ch < BN / 8; ++ch) {  // 8 probabilities -> one 16-byte chunk of each P tile
+        uint4 v4;
+        uint32_t* w4 = reinterpret_cast<uint32_t*>(&v4);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = h * 64 + 2 * c;
+        for (int x = 0; x < 4; ++x) {
+          const int col = ch * 8 + 2 * x;
           const float p0 = fast_exp2(fmaf(s[col], sl2, -m_use));
           const float p1 = fast_exp2(fmaf(s[col + 1], sl2, -m_use));
-          rs4[c & 3] += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-          const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-          rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
-        }
-        if (tp_on) {  // masked copy for the temporal P.V (K-major, 128-byte swizzle)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 v4;
-            uint32_t* w4 = reinterpret_cast<uint32_t*>(&v4);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const int col = h * 64 + ch * 8 + 2 * x;
-              const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-              w4[x] = pk[ch * 4 + x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
-            }
-            const int kc = (h * 8 + ch) >> 3, cc = (h * 8 + ch) & 7;
-            *reinterpret_cast<uint4*>(pP + kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v4;
+          rs4[x] += p0 + p1;
+          w4[x] = pack_bf16x2(p0, p1);
+          if (warp_tp) {
+            const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
+            rt4[x] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
           }
         }
-        tmem_st32_u(t_s + h * 32, pk);
+        const int kc = ch >> 3, cc = ch & 7;
+        const int off = kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(pPD + off) = v4;
+        if (tp_on) {
+          uint4 t4;
+          uint32_t* m4 = reinterpret_cast<uint32_t*>(&t4);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const int col = ch * 8 + 2 * x;
+            const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
+            m4[x] = w4[x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
+          }
+          *reinterpret_cast<uint4*>(pPT + off) = t4;
+        }
       }
       const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       const float rt = (rt4[0] + rt4[1]) + (rt4[2] + rt4[3]);
@@ -472,7 +494,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       mbar_arrive(bar(PB_P_FULL));
     }
     if (ok && cnt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_FINAL), 0, abort_flag, a.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
       tc_fence_after();
     }
     // partials: (m, l) and unnormalised O of each variant

@@ -23,6 +23,10 @@ constexpr int kDevErrKvRange = 0x1;
 constexpr int kDevErrTimeout = 0x2;
 constexpr int kDevErrKind = 0x4;
 constexpr int kDevErrOverflow = 0x8;
+// Lazy softmax rescaling: the accumulators are rescaled only when the running row max (base 2)
+// grows by more than this; otherwise the stale max is kept and probabilities may reach
+// 2^kRescaleLog2, far inside fp32 and bf16 range, with the final 1/l normalisation exact.
+constexpr float kRescaleLog2 = 16.0f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
