@@ -179,7 +179,10 @@ class Pipeline:
         self.mask_bytes = _lib.vsa_mask_workspace_size(self.shape, self.params)
         self.prof_ws = torch.empty(max(self.prof_bytes, 256), dtype=torch.uint8, device=device)
         self.mask_ws = torch.empty(max(self.mask_bytes, 256), dtype=torch.uint8, device=device)
-        self.launches = ((3 if wl.mode == "profiled" else 0) + 3 + (3 if wl.mode == "cube" else 1) + 1 + 1)
+        # work order for cube heads, as the whole call builds it
+        self.order = (torch.empty(wl.B * wl.H * self.nblk, dtype=torch.int32, device=device)
+                      if wl.mode == "cube" else None)
+        self.launches = ((3 if wl.mode == "profiled" else 0) + 3 + (4 if wl.mode == "cube" else 1) + 1 + 1)
 
     def step(self, q, k, v, o, ev=None):
         L, s = self.lib, None
@@ -196,10 +199,12 @@ class Pipeline:
             ev[2].record()
         L.vsa_build_mask(self.kinds, self.qp, self.kp, self.shape, self.params, self.bits, self.kv_idx, self.kv_cnt,
                          self.max_kv, self.mask_ws, self.mask_bytes, self.err, s)
+        if self.order is not None:
+            L.vsa_block_order(self.kinds, self.kv_idx, self.kv_cnt, self.max_kv, self.shape, self.order, s)
         if ev is not None:
             ev[3].record()
         L.vsa_sparse_attn_fwd(L.qkvo(q, k, v, o), L.qkvo(self.qp, self.kp, self.vp, self.op), self.kinds,
-                              self.kv_idx, self.kv_cnt, self.max_kv, self.shape, 0.0, self.err, s)
+                              self.kv_idx, self.kv_cnt, self.max_kv, self.shape, 0.0, self.err, s, order=self.order)
         if ev is not None:
             ev[4].record()
         L.vsa_unpermute(self.op, None, o, L.VSA_BF16, None, self.kinds, self.shape, self.err, s)

@@ -14,8 +14,8 @@ import torch
 from . import _lib
 from ._lib import (VSA_BF16, VSA_CUBE, VSA_F32, VSA_SELECT_CUBE, VSA_SELECT_GIVEN, VSA_SELECT_PROFILE, VSA_SPATIAL,
                    VSA_TEMPORAL, Params, QKVO, Shape, VsaError, make_params, make_shape, qkvo, vsa_attention,
-                   vsa_attention_workspace_layout, vsa_attention_workspace_size, vsa_build_mask,
-                   vsa_get_device_error, vsa_layout_rows, vsa_mask_workspace_size, vsa_max_kv, vsa_num_blocks,
+                   vsa_attention_workspace_layout, vsa_attention_workspace_size, vsa_block_order,
+                   vsa_build_mask, vsa_get_device_error, vsa_layout_rows, vsa_mask_workspace_size, vsa_max_kv, vsa_num_blocks,
                    vsa_pattern_window, vsa_permute, vsa_profile_heads, vsa_profile_rows, vsa_profile_workspace_size,
                    vsa_sparse_attn_fwd, vsa_unpermute)
 
@@ -105,7 +105,7 @@ def attention(q, k, v, F: int, Hl: int, Wl: int, **kw):
 
 
 __all__ = ["SparseAttention", "attention", "VsaError", "Shape", "Params", "QKVO", "make_shape", "make_params", "qkvo",
-           "vsa_attention", "vsa_attention_workspace_layout", "vsa_attention_workspace_size", "vsa_build_mask",
+           "vsa_attention", "vsa_attention_workspace_layout", "vsa_attention_workspace_size", "vsa_block_order", "vsa_build_mask",
            "vsa_get_device_error", "vsa_layout_rows", "vsa_mask_workspace_size", "vsa_max_kv", "vsa_num_blocks",
            "vsa_pattern_window", "vsa_permute", "vsa_profile_heads", "vsa_profile_rows",
            "vsa_profile_workspace_size", "vsa_sparse_attn_fwd", "vsa_unpermute", "VSA_SPATIAL", "VSA_TEMPORAL",

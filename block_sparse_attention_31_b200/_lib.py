@@ -69,7 +69,8 @@ def _load():
         "vsa_profile_static_scratch_bytes": (sz, []),
         "vsa_profile_heads_static": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, vp]),
         "vsa_build_mask": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, i32, vp, sz, vp, vp]),
-        "vsa_sparse_attn_fwd": (st, [P(QKVO), P(QKVO), vp, vp, vp, i32, P(Shape), ctypes.c_float, vp, vp]),
+        "vsa_block_order": (st, [vp, vp, vp, i32, P(Shape), vp, vp]),
+        "vsa_sparse_attn_fwd": (st, [P(QKVO), P(QKVO), vp, vp, vp, i32, vp, P(Shape), ctypes.c_float, vp, vp]),
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
@@ -222,11 +223,17 @@ def qkvo(q, k, v, o, lse=None) -> QKVO:
     return QKVO(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse))
 
 
+def vsa_block_order(kinds, kv_idx, kv_cnt, max_kv, shape: Shape, order, stream=None):
+    _check(lib.vsa_block_order(_ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt), int(max_kv), ctypes.byref(shape),
+                               _ptr(order), _stream(stream)), "vsa_block_order")
+
+
 def vsa_sparse_attn_fwd(natural: QKVO, permuted, kinds, kv_idx, kv_cnt, max_kv, shape: Shape, scale, err,
-                        stream=None):
+                        stream=None, order=None):
     _check(lib.vsa_sparse_attn_fwd(ctypes.byref(natural), ctypes.byref(permuted) if permuted is not None else None,
-                                   _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt), int(max_kv), ctypes.byref(shape),
-                                   float(scale), _ptr(err), _stream(stream)), "vsa_sparse_attn_fwd")
+                                   _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt), int(max_kv), _ptr(order),
+                                   ctypes.byref(shape), float(scale), _ptr(err), _stream(stream)),
+           "vsa_sparse_attn_fwd")
 
 
 def vsa_attention(io: QKVO, dtype: int, shape: Shape, params: Params, select: int, kinds, mse, ws, ws_bytes, err,

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <vector>
 
@@ -55,6 +56,21 @@ cudaError_t encode_rows_map(CUtensorMap* map, const void* base, int d, int rows,
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Every non-null pointer is device (or managed) memory.  Kernels and TMA copies fault on a
+// pageable host address, so a host pointer is refused here, before anything is launched.
+static bool on_device(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (p == nullptr) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return false;
+  }
+  return true;
+}
 
 // Validate the shape and derive the geometry.
 static vsa_status make_geom(const vsa_shape* s, Geom* g) {
@@ -261,6 +277,7 @@ vsa_status vsa_permute(const void* src, vsa_dtype src_dtype, void* dst, const ui
   if (st != VSA_OK) return st;
   if (!src || !dst || !d_kind || !d_err || !aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
   if (src_dtype != VSA_F32 && src_dtype != VSA_BF16) return VSA_ERR_INVALID_ARG;
+  if (!on_device({src, dst, d_kind, d_err})) return VSA_ERR_INVALID_ARG;
   const cudaError_t e =
       launch_permute(src, src_dtype == VSA_F32, dst, d_kind, g, shape->B * shape->H, shape->d, d_err, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
@@ -274,6 +291,7 @@ vsa_status vsa_unpermute(const void* src, const float* src_lse, void* dst, vsa_d
   if (!src || !dst || !d_kind || !d_err || !aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
   if ((src_lse == nullptr) != (dst_lse == nullptr)) return VSA_ERR_INVALID_ARG;
   if (dst_dtype != VSA_F32 && dst_dtype != VSA_BF16) return VSA_ERR_INVALID_ARG;
+  if (!on_device({src, src_lse, dst, dst_lse, d_kind, d_err})) return VSA_ERR_INVALID_ARG;
   const cudaError_t e = launch_unpermute(src, src_lse, dst, dst_dtype == VSA_F32, dst_lse, d_kind, g,
                                          shape->B * shape->H, shape->d, d_err, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
@@ -292,6 +310,7 @@ vsa_status vsa_profile_heads(const void* q, const void* k, const void* v, const 
   const int BH = shape->B * shape->H;
   const ProfilePlan plan = profile_plan(g, BH, shape->d, params->profile_frac);
   if (ws_bytes < plan.bytes) return VSA_ERR_WORKSPACE;
+  if (!on_device({q, k, v, d_kind, d_mse, ws, d_err})) return VSA_ERR_INVALID_ARG;
   const cudaError_t e = launch_profile(q, k, v, g, BH, shape->d, params->w_s, params->w_t,
                                        scale_log2_of(params->scale, shape->d), plan, ws, d_kind, d_mse, d_err, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
@@ -306,6 +325,8 @@ vsa_status vsa_build_mask(const uint8_t* d_kind, const void* q_cube, const void*
   if (!d_kind || !params || !d_bits || !d_kv_idx || !d_kv_cnt || !d_err || max_kv <= 0) return VSA_ERR_INVALID_ARG;
   if (params->w_s < 0 || params->w_t < 0) return VSA_ERR_INVALID_ARG;
   const int BH = shape->B * shape->H;
+  if (!on_device({d_kind, d_bits, d_kv_idx, d_kv_cnt, d_err})) return VSA_ERR_INVALID_ARG;
+  if (g.ncubes > 0 && !on_device({q_cube, k_cube, ws})) return VSA_ERR_INVALID_ARG;
   cudaError_t e = launch_pattern_mask(d_kind, g, BH, params->w_s, params->w_t, d_bits, d_kv_idx, d_kv_cnt, max_kv,
                                       d_err, stream);
   if (e != cudaSuccess) return VSA_ERR_CUDA;
@@ -334,9 +355,23 @@ static vsa_status encode_set(AttnMaps* m, const vsa_qkvo* t, const Geom& g, int 
   return VSA_OK;
 }
 
+vsa_status vsa_block_order(const uint8_t* d_kind, const int32_t* d_kv_idx, const int32_t* d_kv_cnt, int max_kv,
+                           const vsa_shape* shape, int32_t* d_order, cudaStream_t stream) {
+  Geom g;
+  vsa_status st = make_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!d_kind || !d_kv_idx || !d_kv_cnt || !d_order || max_kv <= 0) return VSA_ERR_INVALID_ARG;
+  if (g.nblk > 32768) return VSA_ERR_UNSUPPORTED;
+  if (!on_device({d_kind, d_kv_idx, d_kv_cnt, d_order})) return VSA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_block_order(d_kind, g, shape->B * shape->H, d_kv_idx, d_kv_cnt, max_kv, d_order,
+                                           stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
 vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted, const uint8_t* d_kind,
-                               const int32_t* d_kv_idx, const int32_t* d_kv_cnt, int max_kv, const vsa_shape* shape,
-                               float scale, int* d_err, cudaStream_t stream) {
+                               const int32_t* d_kv_idx, const int32_t* d_kv_cnt, int max_kv,
+                               const int32_t* d_order, const vsa_shape* shape, float scale, int* d_err,
+                               cudaStream_t stream) {
   Geom g;
   vsa_status st = make_geom(shape, &g);
   if (st != VSA_OK) return st;
@@ -344,6 +379,12 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   if (permuted != nullptr && (st = check_qkvo(permuted)) != VSA_OK) return st;
   if (!d_kind || !d_kv_idx || !d_kv_cnt || !d_err || max_kv <= 0 || !(scale >= 0.f)) return VSA_ERR_INVALID_ARG;
   const int BH = shape->B * shape->H;
+  if (!on_device({natural->q, natural->k, natural->v, natural->o, natural->lse, d_kind, d_kv_idx, d_kv_cnt, d_order,
+                  d_err}))
+    return VSA_ERR_INVALID_ARG;
+  if (permuted != nullptr &&
+      !on_device({permuted->q, permuted->k, permuted->v, permuted->o, permuted->lse}))
+    return VSA_ERR_INVALID_ARG;
   AttnMaps nat, perm;
   // Without a permuted set every head reads the `natural` buffers, whose rows must then
   // cover every head's layout (R rows per head).
@@ -358,6 +399,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   a.kinds = d_kind;
   a.kv_idx = d_kv_idx;
   a.kv_cnt = d_kv_cnt;
+  a.order = d_order;
   a.lse_nat = natural->lse;
   a.lse_perm = permuted != nullptr ? permuted->lse : natural->lse;
   a.err = d_err;
@@ -376,7 +418,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
 // Whole call
 // ---------------------------------------------------------------------------------------
 struct AttnLayout {
-  size_t off_bits, off_idx, off_cnt, off_q, off_k, off_v, off_o, off_lse, off_prof, off_mask, bytes;
+  size_t off_bits, off_idx, off_cnt, off_order, off_q, off_k, off_v, off_o, off_lse, off_prof, off_mask, bytes;
   int max_kv;
 };
 
@@ -402,6 +444,8 @@ static vsa_status attention_layout(const vsa_shape* shape, const vsa_params* par
   off = align256(off + BH * g.nblk * max_kv * 4);
   L->off_cnt = off;
   off = align256(off + BH * g.nblk * 4);
+  L->off_order = off;
+  if (g.ncubes > 0) off = align256(off + BH * g.nblk * 4);
   const size_t tbytes = BH * g.R * d * 2;
   L->off_q = off;
   off = align256(off + tbytes);
@@ -451,6 +495,7 @@ vsa_status vsa_attention(const vsa_qkvo* io, vsa_dtype dtype, const vsa_shape* s
   if (!d_kind || !ws || !d_err || !aligned16(ws)) return VSA_ERR_INVALID_ARG;
   if (ws_bytes < L.bytes) return VSA_ERR_WORKSPACE;
   if (dtype != VSA_F32 && dtype != VSA_BF16) return VSA_ERR_INVALID_ARG;
+  if (!on_device({io->q, io->k, io->v, io->o, io->lse, d_kind, d_mse, ws, d_err})) return VSA_ERR_INVALID_ARG;
   Geom g;
   make_geom(shape, &g);
   const int BH = shape->B * shape->H;
@@ -480,13 +525,20 @@ vsa_status vsa_attention(const vsa_qkvo* io, vsa_dtype dtype, const vsa_shape* s
   if ((st = vsa_build_mask(d_kind, pq, pk, shape, params, bits, kv_idx, kv_cnt, L.max_kv, w + L.off_mask,
                            ws_bytes - L.off_mask, d_err, stream)) != VSA_OK)
     return st;
-  // 4. attention: fp32 inputs run every head from the converted buffers
+  // 4. attention: fp32 inputs run every head from the converted buffers.  With cube heads
+  // possible, query blocks are paired and scheduled by their first kept key block.
+  int32_t* order = nullptr;
+  if (g.ncubes > 0) {
+    order = reinterpret_cast<int32_t*>(w + L.off_order);
+    if ((st = vsa_block_order(d_kind, kv_idx, kv_cnt, L.max_kv, shape, order, stream)) != VSA_OK) return st;
+  }
   const vsa_qkvo perm_set{pq, pk, pv, po, plse};
   if (dtype == VSA_F32) {
-    st = vsa_sparse_attn_fwd(&perm_set, nullptr, d_kind, kv_idx, kv_cnt, L.max_kv, shape, params->scale, d_err,
-                             stream);
+    st = vsa_sparse_attn_fwd(&perm_set, nullptr, d_kind, kv_idx, kv_cnt, L.max_kv, order, shape, params->scale,
+                             d_err, stream);
   } else {
-    st = vsa_sparse_attn_fwd(io, &perm_set, d_kind, kv_idx, kv_cnt, L.max_kv, shape, params->scale, d_err, stream);
+    st = vsa_sparse_attn_fwd(io, &perm_set, d_kind, kv_idx, kv_cnt, L.max_kv, order, shape, params->scale, d_err,
+                             stream);
   }
   if (st != VSA_OK) return st;
   // 5. back to natural order
@@ -563,6 +615,7 @@ vsa_status vsa_profile_heads_static(const void* q, const void* k, const void* v,
     if (plan.bytes <= kStaticProfileScratchBytes) break;
   }
   if (plan.bytes > kStaticProfileScratchBytes) return VSA_ERR_WORKSPACE;
+  if (!on_device({q, k, v, d_kind, d_mse, d_err})) return VSA_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if (profile_scratch_address(&scratch) != cudaSuccess) return VSA_ERR_CUDA;
   const cudaError_t e = launch_profile(q, k, v, g, BH, shape->d, params->w_s, params->w_t,

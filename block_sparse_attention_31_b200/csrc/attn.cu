@@ -113,9 +113,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const int rows = layout_rows(g, kind);
   const int nb_head = (rows + BN - 1) / BN;
-  const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
-  if (qb0 >= nb_head) return;
-  const bool has1 = qb1 < nb_head;
+  if (2 * pair >= nb_head) return;
+  const bool has1 = 2 * pair + 1 < nb_head;
+  int qb0 = 2 * pair, qb1 = 2 * pair + 1;
+  if (a.order != nullptr) {  // locality-aware pairing from vsa_build_mask
+    const int32_t* ord = a.order + static_cast<size_t>(bh) * g.nblk;
+    qb0 = ord[2 * pair];
+    qb1 = has1 ? ord[2 * pair + 1] : nb_head;
+    if (qb0 < 0 || qb0 >= nb_head || (has1 && (qb1 < 0 || qb1 >= nb_head || qb1 == qb0))) {
+      if (tid == 0) atomicOr(a.err, kDevErrKvRange);
+      return;
+    }
+  }
   const bool use_perm = a.has_perm && kind != kSpatial;
   const CUtensorMap* tq = use_perm ? &tq_p : &tq_n;
   const CUtensorMap* tk = use_perm ? &tk_p : &tk_n;
@@ -126,10 +135,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ---- the two lists: validate, then build their union in ascending order ----
   const size_t mrow0 = static_cast<size_t>(bh) * g.nblk + qb0;
+  const size_t mrow1 = static_cast<size_t>(bh) * g.nblk + (has1 ? qb1 : qb0);
   const int32_t* kvl0 = a.kv_idx + mrow0 * a.max_kv;
-  const int32_t* kvl1 = kvl0 + a.max_kv;
+  const int32_t* kvl1 = a.kv_idx + mrow1 * a.max_kv;
   int cnt0 = a.kv_cnt[mrow0];
-  int cnt1 = has1 ? a.kv_cnt[mrow0 + 1] : 0;
+  int cnt1 = has1 ? a.kv_cnt[mrow1] : 0;
   bool bad0 = cnt0 < 0 || cnt0 > a.max_kv, bad1 = cnt1 < 0 || cnt1 > a.max_kv;
   for (int x = tid; x < 2 * nwords; x += kAttnThreads) bits0[x] = 0u;  // bits1 follows bits0
   bool stop = false;
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * 64,
-                      (qb0 + t) * BN, bh);
+                      (t ? qb1 : qb0) * BN, bh);
       }
       for (int n = 0; n < U; ++n) {
         const int st = n % C::NS;
@@ -358,7 +368,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quad * 32 + lane;   // query row within the tile
     if (t == 0 || has1) {
       const int cnt = t ? cnt1 : cnt0;
-      const int qb = qb0 + t;
+      const int qb = t ? qb1 : qb0;
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
       const uint32_t t_s = t_lane + C::TMEM_S + t * BN, t_o = t_lane + C::TMEM_O + t * D;
       const float sl2 = a.scale_log2;

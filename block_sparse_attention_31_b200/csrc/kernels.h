@@ -22,6 +22,10 @@ cudaError_t launch_cube_mask(const uint8_t* kinds, const void* q_cube, const voi
                              int topk, uint32_t* bits, int32_t* kv_idx, int32_t* kv_cnt, int max_kv, void* ws,
                              int* err, cudaStream_t stream);
 
+// Attention work order per head (query blocks sorted by their first kept key block).
+cudaError_t launch_block_order(const uint8_t* kinds, const Geom& g, int BH, const int32_t* kv_idx,
+                               const int32_t* kv_cnt, int max_kv, int32_t* order, cudaStream_t stream);
+
 // Tensor maps of one attention problem (3D: d, rows, B*H).
 struct AttnMaps {
   CUtensorMap q, k, v, o;
@@ -31,6 +35,7 @@ struct AttnArgs {
   const uint8_t* kinds;
   const int32_t* kv_idx;
   const int32_t* kv_cnt;
+  const int32_t* order;  // [B*H, nblk] query-block order, or null for natural order
   float* lse_nat;
   float* lse_perm;
   int* err;

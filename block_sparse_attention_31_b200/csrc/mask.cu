@@ -262,6 +262,71 @@ __global__ void __launch_bounds__(kTopkWarps * 32) cube_topk_kernel(const double
   }
 }
 
+// Work order for the attention kernel, per head: the query blocks sorted by (smallest kept key
+// block, block index); rows of a head past its own block count, then empty rows, go last.
+// Consecutive entries then share most key blocks (neighbouring windows for pattern heads,
+// the same cube slab or position for cube heads), which the attention kernel turns into
+// shared K/V loads within a CTA and L2 reuse across concurrently running CTAs.
+constexpr int kOrderThreads = 1024;
+
+__global__ void __launch_bounds__(kOrderThreads) block_order_kernel(const uint8_t* __restrict__ kinds, Geom g,
+                                                                    const int32_t* __restrict__ kv_idx,
+                                                                    const int32_t* __restrict__ kv_cnt, int max_kv,
+                                                                    int n2, int32_t* __restrict__ order) {
+  extern __shared__ uint32_t keys[];  // n2 = next power of two >= nblk
+  const int bh = blockIdx.x;
+  const int kind = kinds[bh];
+  const int rows = kind <= kCube ? layout_rows(g, kind) : 0;
+  const int nb_head = (rows + g.block - 1) / g.block;
+  for (int i = threadIdx.x; i < n2; i += kOrderThreads) {
+    uint32_t key = 0xffffffffu;
+    if (i < g.nblk) {
+      const size_t row = static_cast<size_t>(bh) * g.nblk + i;
+      const int cnt = kv_cnt[row];
+      uint32_t hi;
+      if (i >= nb_head) hi = 0xffffu;
+      else if (cnt <= 0) hi = 0xfffeu;
+      else hi = min(static_cast<uint32_t>(kv_idx[row * max_kv]), 0xfffdu);
+      key = (hi << 16) | static_cast<uint32_t>(i);
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += kOrderThreads) {
+        const int p = i ^ j;
+        if (p > i) {
+          const uint32_t a = keys[i], b = keys[p];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[p] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  for (int i = threadIdx.x; i < g.nblk; i += kOrderThreads)
+    order[static_cast<size_t>(bh) * g.nblk + i] = static_cast<int32_t>(keys[i] & 0xffffu);
+}
+
+cudaError_t launch_block_order(const uint8_t* kinds, const Geom& g, int BH, const int32_t* kv_idx,
+                               const int32_t* kv_cnt, int max_kv, int32_t* order, cudaStream_t stream) {
+  if (g.nblk > 0xffff) return cudaErrorInvalidValue;
+  int n2 = 1;
+  while (n2 < g.nblk) n2 <<= 1;
+  const size_t smem = sizeof(uint32_t) * n2;
+  if (smem > 232448) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(block_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  block_order_kernel<<<BH, kOrderThreads, smem, stream>>>(kinds, g, kv_idx, kv_cnt, max_kv, n2, order);
+  return cudaGetLastError();
+}
+
 size_t cube_mask_workspace_bytes(const Geom& g, int BH, int d) {
   return sizeof(double) * (2 * static_cast<size_t>(BH) * g.ncubes * d +
                            static_cast<size_t>(BH) * g.ncubes * g.ncubes);

@@ -31,7 +31,9 @@
  *     The library never allocates or frees device memory and keeps no mutable global
  *     state; every call is asynchronous on `stream` (NULL = legacy default stream) and
  *     never synchronises, except vsa_get_device_error.
- *   - All device pointers must be 16-byte aligned; tensors must be contiguous.
+ *   - All device pointers must be 16-byte aligned; tensors must be contiguous.  Each one
+ *     must be device (or managed) memory: a host address is refused with
+ *     VSA_ERR_INVALID_ARG before any launch.
  *   - Errors: arguments are validated on the host before any launch (VSA_ERR_INVALID_ARG,
  *     VSA_ERR_UNSUPPORTED, VSA_ERR_WORKSPACE); a failed launch returns VSA_ERR_CUDA.
  *     Kernels that detect a bad device-side input (an index or count out of range) or a
@@ -222,6 +224,19 @@ VSA_API vsa_status vsa_build_mask(const uint8_t *d_kind, const void *q_cube, con
                           int max_kv, void *ws, size_t ws_bytes, int *d_err, cudaStream_t stream);
 
 /*
+ * Work order for vsa_sparse_attn_fwd (no counterpart in the pages; it changes only which
+ * query blocks share a CTA and which run at the same time, never a result): per head, the
+ * query blocks 0..nb-1 sorted by (first kept key block, block index), where nb is the
+ * head's own block count; blocks past nb follow in ascending order.  Query blocks that
+ * keep the same key blocks (a cube slab for per-frame heads, a cube position across
+ * slabs for per-position heads) then land in the same CTA and in CTAs that run together.
+ *   d_kind, d_kv_idx, d_kv_cnt, max_kv   as for vsa_sparse_attn_fwd (device)
+ *   d_order  [B, H, nblk] int32 out (device, caller-owned); nblk <= 32768
+ */
+VSA_API vsa_status vsa_block_order(const uint8_t *d_kind, const int32_t *d_kv_idx, const int32_t *d_kv_cnt,
+                                   int max_kv, const vsa_shape *shape, int32_t *d_order, cudaStream_t stream);
+
+/*
  * Block-sparse attention forward ("OSP-Next", "Method"; "Sparse Video-Gen", "Approach"):
  * for every query block i of every head, O_i = softmax(Q_i K_J^T * scale) V_J over the
  * key blocks J = kv_idx[b,h,i,0..cnt), keys past the head's real rows (ragged tail,
@@ -232,11 +247,15 @@ VSA_API vsa_status vsa_build_mask(const uint8_t *d_kind, const void *q_cube, con
  *             in which case every head uses `natural`
  *   d_kind    [B*H] head kinds; d_kv_idx / d_kv_cnt from vsa_build_mask (each list strictly
  *             ascending; a malformed list sets VSA_DEVERR_KV_RANGE and its rows are zero)
+ *   d_order   NULL (query blocks paired as 2i, 2i+1) or the [B, H, nblk] permutation from
+ *             vsa_block_order (its first nb entries per head must be distinct blocks < nb,
+ *             else VSA_DEVERR_KV_RANGE)
  *   scale     softmax scale, 0 selects 1/sqrt(d)
  */
 VSA_API vsa_status vsa_sparse_attn_fwd(const vsa_qkvo *natural, const vsa_qkvo *permuted, const uint8_t *d_kind,
                                const int32_t *d_kv_idx, const int32_t *d_kv_cnt, int max_kv,
-                               const vsa_shape *shape, float scale, int *d_err, cudaStream_t stream);
+                               const int32_t *d_order, const vsa_shape *shape, float scale, int *d_err,
+                               cudaStream_t stream);
 
 /*
  * The whole call: kinds (profiled, given or cube) -> permute -> masks -> sparse attention

@@ -113,8 +113,10 @@ def test_kernel_entry_points_validate_before_launch():
     assert lib.vsa_build_mask(FAKE, None, None, ctypes.byref(shape), ctypes.byref(params), FAKE, FAKE, FAKE, 0,
                               None, 0, FAKE, s) == _lib.VSA_ERR_INVALID_ARG
     io = _lib.QKVO(FAKE, FAKE, None, FAKE, None)
-    assert lib.vsa_sparse_attn_fwd(ctypes.byref(io), None, FAKE, FAKE, FAKE, 4, ctypes.byref(shape), 0.0, FAKE,
-                                   s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_sparse_attn_fwd(ctypes.byref(io), None, FAKE, FAKE, FAKE, 4, None, ctypes.byref(shape), 0.0,
+                                   FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_block_order(FAKE, FAKE, FAKE, 4, ctypes.byref(shape), None, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_block_order(FAKE, FAKE, FAKE, 0, ctypes.byref(shape), FAKE, s) == _lib.VSA_ERR_INVALID_ARG
     io = _lib.QKVO(FAKE, FAKE, FAKE, FAKE, None)
     assert lib.vsa_attention(ctypes.byref(io), 1, ctypes.byref(shape), ctypes.byref(params), 0, FAKE, None, FAKE, 8,
                              FAKE, s) == _lib.VSA_ERR_WORKSPACE

@@ -161,7 +161,16 @@ def test_mask_overflow_flag():
 # sparse attention kernel (masks from the oracle, so the kernel is tested on its own)
 # ------------------------------------------------------------------------------------
 
-def _attention_case(wl, kinds_list, keeps, q, k, v, perm, rows=None, lse_check=True):
+def _check_block_order(order, kinds_list, wl, idx, cnt, nblk):
+    """The work order is, per head, the head's blocks sorted by (first kept block, index)."""
+    for h, kind in enumerate(kinds_list):
+        nb = -(-oracle.layout_rows(kind, wl.F, wl.Hl, wl.Wl, wl.cube) // wl.block)
+        first = [int(idx[0, h, i, 0]) if cnt[0, h, i] > 0 else 1 << 20 for i in range(nb)]
+        want = sorted(range(nb), key=lambda i: (first[i], i)) + list(range(nb, nblk))
+        assert order[h].tolist() == want, f"head {h}"
+
+
+def _attention_case(wl, kinds_list, keeps, q, k, v, perm, rows=None, lse_check=True, ordered=False):
     H = len(kinds_list)
     shape = _lib.make_shape(1, H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, wl.cube if C_ in kinds_list else None)
     nblk = _lib.vsa_num_blocks(shape)
@@ -185,8 +194,24 @@ def _attention_case(wl, kinds_list, keeps, q, k, v, perm, rows=None, lse_check=T
         lsep = torch.empty(1, H, R, dtype=torch.float32, device="cuda")
         for src, dst in ((qd, qp), (kd, kp_), (vd, vp)):
             _lib.vsa_permute(src, _lib.VSA_BF16, dst, kinds, shape, err)
+        idx_d, cnt_d = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+        order = None
+        if ordered:
+            order = torch.full((H, nblk), -5, dtype=torch.int32, device="cuda")
+            _lib.vsa_block_order(kinds, idx_d, cnt_d, max_kv, shape, order)
+            _check_block_order(order.cpu(), kinds_list, wl, idx, cnt, nblk)
+            # pairing changes no result: natural pairing gives the same bits
+            op_nat, lsep_nat = torch.empty_like(op), torch.empty_like(lsep)
+            _lib.vsa_sparse_attn_fwd(_lib.qkvo(qd, kd, vd, o, lse), _lib.qkvo(qp, kp_, vp, op_nat, lsep_nat), kinds,
+                                     idx_d, cnt_d, max_kv, shape, 0.0, err)
         _lib.vsa_sparse_attn_fwd(_lib.qkvo(qd, kd, vd, o, lse), _lib.qkvo(qp, kp_, vp, op, lsep), kinds,
-                                 torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), max_kv, shape, 0.0, err)
+                                 idx_d, cnt_d, max_kv, shape, 0.0, err, order=order)
+        if ordered:
+            for h, kind in enumerate(kinds_list):
+                if kind != S_:  # rows past a head's own layout are never written
+                    r = oracle.layout_rows(kind, wl.F, wl.Hl, wl.Wl, wl.cube)
+                    assert torch.equal(op[0, h, :r], op_nat[0, h, :r]), f"head {h}"
+                    assert torch.equal(lsep[0, h, :r], lsep_nat[0, h, :r]), f"head {h}"
         _lib.vsa_unpermute(op, lsep, o, _lib.VSA_BF16, lse, kinds, shape, err)
     else:
         _lib.vsa_sparse_attn_fwd(_lib.qkvo(qd, kd, vd, o, lse), None, kinds, torch.from_numpy(idx).cuda(),
@@ -248,6 +273,20 @@ def test_attention_cube_padding():
     _attention_case(wl.with_(H=1), [C_], [kp], q, k, v, perm=True)
 
 
+@pytest.mark.parametrize("F,Hl,Wl", [(9, 9, 17), (12, 16, 16)])
+def test_attention_block_order(F, Hl, Wl):
+    """Cube and pattern heads run in the locality order of vsa_block_order: the order is the
+    documented sort, results equal natural pairing bit for bit and match the oracle."""
+    wl = _wl(F, Hl, Wl, 128, 128, H=3, topk=4)
+    q, k, v = synthetic.make_qkv(wl)
+    C = oracle.num_cubes(F, Hl, Wl)
+    rng = np.random.default_rng(F)
+    kc = rng.random((C, C)) < 0.15
+    kc[rng.random(C) < 0.1] = False           # a few query cubes with nothing kept
+    keeps = [kc, keep_for_head(S_, wl, 1, 0), keep_for_head(T_, wl, 0, 20)]
+    _attention_case(wl, [C_, S_, T_], keeps, q, k, v, perm=True, ordered=True)
+
+
 def test_attention_large_scores_stable():
     """Inputs scaled x8: logits up to a few hundred must not overflow the online softmax."""
     wl = _wl(3, 8, 16, 128, 128, H=1)
@@ -272,6 +311,20 @@ def test_attention_bad_lists_flag_error():
     o = o.cpu().float()
     assert (o[0, 0, 64:128] == 0).all() and (o[0, 0, 192:256] == 0).all()   # rejected rows are zero
     assert torch.isfinite(o).all()
+    # a host address anywhere is refused before any launch
+    o_host = torch.empty(1, 1, wl.N, 64, dtype=torch.bfloat16)
+    with pytest.raises(_lib.VsaError) as ex:
+        _lib.vsa_sparse_attn_fwd(_lib.qkvo(q, q, q, o_host), None, kinds, idx, cnt, 2, shape, 0.0, err)
+    assert ex.value.status == _lib.VSA_ERR_INVALID_ARG
+    # a work order that is not a permutation of the head's blocks
+    o = torch.empty_like(q)
+    good = torch.tensor([[[[0, -1], [1, -1], [2, -1], [3, -1]]]], dtype=torch.int32, device="cuda")
+    ones = torch.ones(1, 1, 4, dtype=torch.int32, device="cuda")
+    for bad in ([0, 0, 1, 2], [0, 1, 2, 7], [-1, 1, 2, 3]):
+        err.zero_()
+        order = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        _lib.vsa_sparse_attn_fwd(_lib.qkvo(q, q, q, o), None, kinds, good, ones, 2, shape, 0.0, err, order=order)
+        assert _lib.vsa_get_device_error(err) & _lib.VSA_DEVERR_KV_RANGE, bad
     # a bad kind byte
     err.zero_()
     kinds.fill_(9)
