@@ -9,9 +9,9 @@
 // Cube heads ("USV" page, Figure 2: top-k cube selection on coarse attention): every cube
 // is pooled to the fp64 mean of its real tokens' Q and K; the coarse score of (c, c') is
 // their dot product; each query cube keeps itself plus the top-k key cubes by score
-// (ties to the smaller index).  The pooled sums are accumulated in slot order and the dot
-// products in dimension order with separately rounded multiply and add, so the scores are
-// reproducible to the last bit.
+// (ties to the smaller index).  The pooled sums are accumulated in slot order with one
+// rounded add per token and the dot products in dimension order with one fused multiply-add
+// per term, so the scores are reproducible to the last bit.
 //
 // Every mask row is written three ways: a bitset, an ascending index list padded with -1,
 // and a count.
@@ -87,52 +87,87 @@ cudaError_t launch_pattern_mask(const uint8_t* kinds, const Geom& g, int BH, int
 // ---------------------------------------------------------------------------------------
 // Cube heads
 // ---------------------------------------------------------------------------------------
-constexpr int kPoolThreads = 64;
-
-// One CTA per (cube, head); thread x owns dimensions 2x, 2x+1 (+128 per pass).  The sums run
-// over the cube's real tokens in slot order, i.e. increasing natural token index.
-__global__ void __launch_bounds__(kPoolThreads) cube_pool_kernel(const __nv_bfloat16* __restrict__ qc,
-                                                                 const __nv_bfloat16* __restrict__ kc,
-                                                                 const uint8_t* __restrict__ kinds, Geom g, int d,
-                                                                 double* __restrict__ qbar,
-                                                                 double* __restrict__ kbar) {
-  const int cube = blockIdx.x, bh = blockIdx.y;
-  if (kinds[bh] != kCube) return;
-  const int cw_i = cube % g.ncw, ch_i = (cube / g.ncw) % g.nch, cf_i = cube / (g.ncw * g.nch);
-  const int nf = min(g.cf, g.F - cf_i * g.cf), nh = min(g.ch, g.Hl - ch_i * g.ch), nw = min(g.cw, g.Wl - cw_i * g.cw);
-  const double n = static_cast<double>(nf * nh * nw);
-  const size_t base = (static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol) * d;
-  const size_t out = (static_cast<size_t>(bh) * g.ncubes + cube) * d;
-  for (int x = threadIdx.x * 2; x < d; x += kPoolThreads * 2) {
-    double sq0 = 0.0, sq1 = 0.0, sk0 = 0.0, sk1 = 0.0;
-    for (int df = 0; df < nf; ++df)
-      for (int dh = 0; dh < nh; ++dh)
-        for (int dw = 0; dw < nw; ++dw) {
-          const size_t r = static_cast<size_t>((df * g.ch + dh) * g.cw + dw);
-          const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(qc + base + r * d + x);
-          const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(kc + base + r * d + x);
-          sq0 = __dadd_rn(sq0, static_cast<double>(__low2float(a)));
-          sq1 = __dadd_rn(sq1, static_cast<double>(__high2float(a)));
-          sk0 = __dadd_rn(sk0, static_cast<double>(__low2float(b)));
-          sk1 = __dadd_rn(sk1, static_cast<double>(__high2float(b)));
-        }
-    qbar[out + x] = __ddiv_rn(sq0, n);
-    qbar[out + x + 1] = __ddiv_rn(sq1, n);
-    kbar[out + x] = __ddiv_rn(sk0, n);
-    kbar[out + x + 1] = __ddiv_rn(sk1, n);
-  }
+// Exact widening of a bf16 bit pattern to double.  Normal numbers are rebuilt with integer
+// operations (exponent rebias 127 -> 1023, mantissa moved to the top of the 52-bit field);
+// zero, subnormals, infinities and NaN take the float path.  Both are exact.
+__device__ __forceinline__ double bf16_bits_to_double(uint32_t x) {
+  const uint32_t e = x & 0x7F80u;
+  if (e != 0u && e != 0x7F80u)
+    return __hiloint2double(static_cast<int>(((x & 0x8000u) << 16) | (((x & 0x7FFFu) << 13) + (896u << 20))), 0);
+  return static_cast<double>(__uint_as_float(x << 16));
 }
 
-// Coarse scores S[c][c'] = qbar_c . kbar_c' of one head: 64 x 64 outputs per CTA, 4 x 4 per
-// thread (rows ty + 16i, columns tx + 16j), dimensions staged 32 at a time in shared memory
-// (transposed, so a warp's column reads are consecutive).  Every output accumulates its
-// products in dimension order with separately rounded multiply and add.
-constexpr int kScoreTile = 64, kScoreK = 32;
+constexpr int kPoolWarps = 4;  // one cube per warp
+constexpr int kPoolBatch = 8;  // rows loaded ahead of the sequential adds
 
-__global__ void __launch_bounds__(256) cube_score_kernel(const double* __restrict__ qbar,
-                                                         const double* __restrict__ kbar,
-                                                         const uint8_t* __restrict__ kinds, int C, int d,
-                                                         double* __restrict__ scores) {
+// Pooled means of one cube per warp: lanes 0-15 own Q, lanes 16-31 own K, each lane eight
+// consecutive dimensions (one 16-byte load per row).  Per dimension the sum runs over the
+// cube's real tokens in slot order, i.e. increasing natural token index, one rounded add per
+// token; kPoolBatch rows are loaded before they are added so that the loads overlap.
+__global__ void __launch_bounds__(kPoolWarps * 32) cube_pool_kernel(const __nv_bfloat16* __restrict__ qc,
+                                                                   const __nv_bfloat16* __restrict__ kc,
+                                                                   const uint8_t* __restrict__ kinds, Geom g, int d,
+                                                                   double* __restrict__ qbar,
+                                                                   double* __restrict__ kbar) {
+  const int bh = blockIdx.y;
+  if (kinds[bh] != kCube) return;
+  const int lane = threadIdx.x & 31;
+  const int cube = blockIdx.x * kPoolWarps + (threadIdx.x >> 5);
+  const int x = (lane & 15) * 8;  // first dimension of this lane
+  if (cube >= g.ncubes || x >= d) return;
+  const __nv_bfloat16* src = lane < 16 ? qc : kc;
+  double* dst = lane < 16 ? qbar : kbar;
+  const int cw_i = cube % g.ncw, ch_i = (cube / g.ncw) % g.nch, cf_i = cube / (g.ncw * g.nch);
+  const int nf = min(g.cf, g.F - cf_i * g.cf), nh = min(g.ch, g.Hl - ch_i * g.ch), nw = min(g.cw, g.Wl - cw_i * g.cw);
+  const int cnt = nf * nh * nw;
+  const bool full = cnt == g.vol;
+  const __nv_bfloat16* base = src + (static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol) * d + x;
+  double acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+  for (int i0 = 0; i0 < cnt; i0 += kPoolBatch) {
+    uint4 buf[kPoolBatch];
+#pragma unroll
+    for (int u = 0; u < kPoolBatch; ++u) {
+      const int i = i0 + u;
+      if (i < cnt) {
+        int slot = i;
+        if (!full) {  // token i of the cube's nf x nh x nw real tokens -> slot (df*ch + dh)*cw + dw
+          const int dw = i % nw, t = i / nw;
+          slot = ((t / nh) * g.ch + t % nh) * g.cw + dw;
+        }
+        buf[u] = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(slot) * d);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPoolBatch; ++u) {
+      if (i0 + u < cnt) {
+        const uint32_t w[4] = {buf[u].x, buf[u].y, buf[u].z, buf[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * j] = __dadd_rn(acc[2 * j], bf16_bits_to_double(w[j] & 0xFFFFu));
+          acc[2 * j + 1] = __dadd_rn(acc[2 * j + 1], bf16_bits_to_double(w[j] >> 16));
+        }
+      }
+    }
+  }
+  const double n = static_cast<double>(cnt);
+  double* out = dst + (static_cast<size_t>(bh) * g.ncubes + cube) * d + x;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) out[j] = __ddiv_rn(acc[j], n);
+}
+
+// Coarse scores S[c][c'] = qbar_c . kbar_c' of one head: 128 x 128 outputs per CTA, 8 x 8
+// per thread (rows ty + 16i, columns tx + 16j), dimensions staged 16 at a time in shared
+// memory (transposed, so a warp's column reads are consecutive).  Every output accumulates
+// its products in dimension order, one fused multiply-add per term.  Eight outputs per
+// operand load keep the FP64 pipe, not shared memory, the limit.
+constexpr int kScoreTile = 128, kScoreK = 16, kScoreThreads = 256;
+
+__global__ void __launch_bounds__(kScoreThreads, 1) cube_score_kernel(const double* __restrict__ qbar,
+                                                                      const double* __restrict__ kbar,
+                                                                      const uint8_t* __restrict__ kinds, int C,
+                                                                      int d, double* __restrict__ scores) {
   __shared__ double sq[kScoreK][kScoreTile + 1];
   __shared__ double sk[kScoreK][kScoreTile + 1];
   const int bh = blockIdx.z;
@@ -141,93 +176,173 @@ __global__ void __launch_bounds__(256) cube_score_kernel(const double* __restric
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const double* qh = qbar + static_cast<size_t>(bh) * C * d;
   const double* kh = kbar + static_cast<size_t>(bh) * C * d;
-  double acc[4][4];
+  double acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
   for (int e0 = 0; e0 < d; e0 += kScoreK) {
     __syncthreads();
-    for (int x = tid; x < kScoreTile * kScoreK; x += 256) {
-      const int r = x / kScoreK, e = x - r * kScoreK;
+#pragma unroll
+    for (int it = 0; it < kScoreTile * kScoreK / kScoreThreads; ++it) {
+      const int x = tid + it * kScoreThreads;
+      const int r = x / kScoreK, e = x % kScoreK;
       sq[e][r] = r0 + r < C ? qh[static_cast<size_t>(r0 + r) * d + e0 + e] : 0.0;
       sk[e][r] = c0 + r < C ? kh[static_cast<size_t>(c0 + r) * d + e0 + e] : 0.0;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 2
     for (int e = 0; e < kScoreK; ++e) {
-      double a[4], b[4];
+      double a[8], b[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = sq[e][ty + 16 * i];
+      for (int i = 0; i < 8; ++i) a[i] = sq[e][ty + 16 * i];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = sk[e][tx + 16 * j];
+      for (int j = 0; j < 8; ++j) b[j] = sk[e][tx + 16 * j];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __dadd_rn(acc[i][j], __dmul_rn(a[i], b[j]));
+        for (int j = 0; j < 8; ++j) acc[i][j] = __fma_rn(a[i], b[j], acc[i][j]);
     }
   }
   double* sh = scores + static_cast<size_t>(bh) * C * C;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const int r = r0 + ty + 16 * i;
     if (r >= C) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const int c = c0 + tx + 16 * j;
       if (c < C) sh[static_cast<size_t>(r) * C + c] = acc[i][j];
     }
   }
 }
 
+constexpr int kTopkWarps = 4;
+constexpr int kTopkCap = 512;  // candidates per row kept for the exact selection
+
+// Order-preserving integer key of a finite double (larger value <-> larger key); -0 and +0,
+// equal as doubles, get the same key.
+__device__ __forceinline__ uint64_t score_key(double s) {
+  uint64_t b = static_cast<uint64_t>(__double_as_longlong(s));
+  if (b == 0x8000000000000000ull) b = 0ull;
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// Warp-wide maximum of (key desc, index asc) pairs; every lane gets the winning index.
+__device__ __forceinline__ int warp_argmax_key(uint64_t k, int c) {
+  const uint32_t hi = static_cast<uint32_t>(k >> 32), lo = static_cast<uint32_t>(k);
+  const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+  const bool top = hi == mhi && lo == mlo;
+  return static_cast<int>(__reduce_min_sync(0xffffffffu, top ? static_cast<uint32_t>(c) : 0x7fffffffu));
+}
+
 // Top-k of one score row per warp (score descending, ties to the smaller index) plus the own
 // cube; emits the bitset, the ascending list and the count.
-constexpr int kTopkWarps = 4;
-
+//
+// Fast path (topk <= 32): the smallest of the 32 lane maxima is a lower bound L on the k-th
+// largest score, since those 32 maxima are distinct entries that are all >= L.  Only entries
+// >= L (typically a few per cent of the row) are gathered, and the exact selection runs on
+// them.  With more than kTopkCap candidates, or topk > 32, every round scans the whole row.
 __global__ void __launch_bounds__(kTopkWarps * 32) cube_topk_kernel(const double* __restrict__ scores,
                                                                     const uint8_t* __restrict__ kinds, Geom g,
                                                                     int topk, uint32_t* __restrict__ bits,
                                                                     int32_t* __restrict__ kv_idx,
                                                                     int32_t* __restrict__ kv_cnt, int max_kv,
                                                                     int* err) {
-  extern __shared__ __align__(16) uint8_t topk_smem[];  // [kTopkWarps][C] doubles, then [kTopkWarps][nwords]
+  // per warp: kTopkCap keys, kTopkCap indices, nwords selection words
+  extern __shared__ __align__(16) uint8_t topk_smem[];
   const int bh = blockIdx.y;
   if (kinds[bh] != kCube) return;
   const int C = g.ncubes;
   const int nwords = (g.nblk + 31) >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kTopkWarps + warp;
-  double* srow = reinterpret_cast<double*>(topk_smem) + static_cast<size_t>(warp) * C;
-  uint32_t* sel = reinterpret_cast<uint32_t*>(reinterpret_cast<double*>(topk_smem) + static_cast<size_t>(kTopkWarps) * C) +
+  uint64_t* ck = reinterpret_cast<uint64_t*>(topk_smem) + static_cast<size_t>(warp) * kTopkCap;
+  int* ci = reinterpret_cast<int*>(reinterpret_cast<uint64_t*>(topk_smem) + kTopkWarps * kTopkCap) + warp * kTopkCap;
+  uint32_t* sel = reinterpret_cast<uint32_t*>(reinterpret_cast<int*>(reinterpret_cast<uint64_t*>(topk_smem) +
+                                                                     kTopkWarps * kTopkCap) +
+                                              kTopkWarps * kTopkCap) +
                   warp * nwords;
   for (int x = lane; x < nwords; x += 32) sel[x] = 0u;
   if (row >= C) return;
   const double* grow = scores + (static_cast<size_t>(bh) * C + row) * C;
-  for (int c = lane; c < C; c += 32) srow[c] = __ldg(grow + c);
-  __syncwarp();
   const int picks = topk < C ? topk : C;
-  for (int p = 0; p < picks; ++p) {
-    double best = -DBL_MAX;
-    int best_c = 0x7fffffff;
-    for (int c = lane; c < C; c += 32) {
-      if ((sel[c >> 5] >> (c & 31)) & 1u) continue;
-      const double s = srow[c];
-      if (s > best || (s == best && c < best_c)) {
-        best = s;
-        best_c = c;
+  bool exact_scan = picks > 32;
+  if (!exact_scan && picks > 0) {
+    uint64_t lmax = 0ull;  // 0: below every finite key
+    for (int c = lane; c < C; c += 32) lmax = max(lmax, score_key(__ldg(grow + c)));
+    const uint32_t lhi = static_cast<uint32_t>(lmax >> 32), llo = static_cast<uint32_t>(lmax);
+    const uint32_t bhi = __reduce_min_sync(0xffffffffu, lhi);
+    const uint32_t blo = __reduce_min_sync(0xffffffffu, lhi == bhi ? llo : 0xffffffffu);
+    const uint64_t bound = (static_cast<uint64_t>(bhi) << 32) | blo;
+    int n = 0;
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      const int c = c0 + lane;
+      const uint64_t k = c < C ? score_key(__ldg(grow + c)) : 0ull;
+      const bool cand = c < C && k >= bound;
+      const uint32_t m = __ballot_sync(0xffffffffu, cand);
+      const int pos = n + __popc(m & ((1u << lane) - 1u));
+      if (cand && pos < kTopkCap) {
+        ck[pos] = k;
+        ci[pos] = c;
       }
+      n += __popc(m);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oc = __shfl_xor_sync(0xffffffffu, best_c, off);
-      if (ob > best || (ob == best && oc < best_c)) {
-        best = ob;
-        best_c = oc;
-      }
-    }
-    if (lane == 0 && best_c < C) sel[best_c >> 5] |= 1u << (best_c & 31);
     __syncwarp();
+    if (n > kTopkCap) {
+      exact_scan = true;
+    } else {
+      // exact selection among the n candidates; lane owns slots lane + 32 m
+      const int M = (n + 31) >> 5;  // <= kTopkCap / 32 = 16
+      uint32_t taken = 0u;
+      for (int p = 0; p < picks; ++p) {
+        uint64_t bk = 0ull;
+        int bc = 0x7fffffff, bm = -1;
+        for (int m = 0; m < M; ++m) {
+          const int x = lane + 32 * m;
+          if (x >= n || ((taken >> m) & 1u)) continue;
+          const uint64_t k = ck[x];
+          const int c = ci[x];
+          if (bm < 0 || k > bk || (k == bk && c < bc)) {
+            bk = k;
+            bc = c;
+            bm = m;
+          }
+        }
+        const int win = warp_argmax_key(bm < 0 ? 0ull : bk, bm < 0 ? 0x7fffffff : bc);
+        if (bm >= 0 && bc == win) {
+          taken |= 1u << bm;
+          sel[win >> 5] |= 1u << (win & 31);
+        }
+        __syncwarp();
+      }
+    }
+  }
+  if (exact_scan) {  // every round scans the whole row (topk > 32 or too many candidates)
+    for (int p = 0; p < picks; ++p) {
+      double best = -DBL_MAX;
+      int best_c = 0x7fffffff;
+      for (int c = lane; c < C; c += 32) {
+        if ((sel[c >> 5] >> (c & 31)) & 1u) continue;
+        const double s = __ldg(grow + c);
+        if (s > best || (s == best && c < best_c)) {
+          best = s;
+          best_c = c;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oc = __shfl_xor_sync(0xffffffffu, best_c, off);
+        if (ob > best || (ob == best && oc < best_c)) {
+          best = ob;
+          best_c = oc;
+        }
+      }
+      if (lane == 0 && best_c < C) sel[best_c >> 5] |= 1u << (best_c & 31);
+      __syncwarp();
+    }
   }
   if (lane == 0) sel[row >> 5] |= 1u << (row & 31);
   __syncwarp();
@@ -339,17 +454,16 @@ cudaError_t launch_cube_mask(const uint8_t* kinds, const void* q_cube, const voi
   double* qbar = static_cast<double*>(ws);
   double* kbar = qbar + static_cast<size_t>(BH) * C * d;
   double* scores = kbar + static_cast<size_t>(BH) * C * d;
-  cube_pool_kernel<<<dim3(C, BH), kPoolThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q_cube),
-                                                              static_cast<const __nv_bfloat16*>(k_cube), kinds, g, d,
-                                                              qbar, kbar);
+  cube_pool_kernel<<<dim3((C + kPoolWarps - 1) / kPoolWarps, BH), kPoolWarps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q_cube), static_cast<const __nv_bfloat16*>(k_cube), kinds, g, d, qbar, kbar);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nt = (C + kScoreTile - 1) / kScoreTile;
-  cube_score_kernel<<<dim3(nt, nt, BH), 256, 0, stream>>>(qbar, kbar, kinds, C, d, scores);
+  cube_score_kernel<<<dim3(nt, nt, BH), kScoreThreads, 0, stream>>>(qbar, kbar, kinds, C, d, scores);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nwords = (g.nblk + 31) >> 5;
-  const size_t smem = sizeof(double) * kTopkWarps * C + sizeof(uint32_t) * kTopkWarps * nwords;
+  const size_t smem = (sizeof(uint64_t) + sizeof(int)) * kTopkWarps * kTopkCap + sizeof(uint32_t) * kTopkWarps * nwords;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(cube_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -8,6 +8,8 @@
 // Both kernels are HBM-bound row copies: each thread moves one 16-byte vector (8 bf16) of
 // a row and every thread keeps four rows in flight.  Rows are 128 or 256 bytes, so each
 // warp touches whole 128-byte lines.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -62,6 +64,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const void* __res
     return;
   }
   if (!kSrcF32 && kind == kSpatial) return;
+  if (kind == kCube && g.ncubes > 0) return;  // cube_permute_kernel
   const int vpr = d / 8;  // 16-byte vectors per row
   const int rows_per_pass = kPermThreads / vpr;
   const int v = threadIdx.x % vpr;
@@ -99,6 +102,7 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __nv_bflo
     return;
   }
   if (!kDstF32 && kind == kSpatial) return;
+  if (kind == kCube && g.ncubes > 0) return;  // cube_unpermute_kernel
   const int vpr = d / 8;
   const int rows_per_pass = kPermThreads / vpr;
   const int v = threadIdx.x % vpr;
@@ -127,30 +131,162 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __nv_bflo
   }
 }
 
-static int perm_grid_x(int rows, int d) {
+// Cube heads: one warp per cube.  A lane keeps one 16-byte column v of the row and walks the
+// cube's slots r = r_lane, r_lane + 32/vpr, ...; the slot's (df, dh, dw) offsets are advanced
+// incrementally, so no division runs per row.  Consecutive slots of a cube line (fixed df, dh)
+// are consecutive tokens, so every warp access is contiguous on both sides.
+constexpr int kCubeWarps = 8;
+constexpr int kCubeUnroll = 8;
+
+struct CubeWalk {
+  int dw, dh, df;
+  __device__ __forceinline__ void init(const Geom& g, int r) {
+    dw = r % g.cw;
+    const int t = r / g.cw;
+    dh = t % g.ch;
+    df = t / g.ch;
+  }
+  __device__ __forceinline__ void advance(const Geom& g, int step) {
+    dw += step;
+    while (dw >= g.cw) {
+      dw -= g.cw;
+      if (++dh == g.ch) {
+        dh = 0;
+        ++df;
+      }
+    }
+  }
+};
+
+// dst[bh, cube*vol + r] = bf16(src[bh, token of slot r of the cube]), zero for padding slots.
+template <bool kSrcF32>
+__global__ void __launch_bounds__(kCubeWarps * 32) cube_permute_kernel(const void* __restrict__ src,
+                                                                      __nv_bfloat16* __restrict__ dst,
+                                                                      const uint8_t* __restrict__ kinds, Geom g,
+                                                                      int d) {
+  const int bh = blockIdx.y;
+  if (kinds[bh] != kCube) return;
+  const int cube = blockIdx.x * kCubeWarps + (threadIdx.x >> 5);
+  if (cube >= g.ncubes) return;
+  const int lane = threadIdx.x & 31;
+  const int vpr = d / 8, rstep = 32 / vpr;
+  const int v = lane % vpr;
+  const int cw_i = cube % g.ncw, ch_i = (cube / g.ncw) % g.nch, cf_i = cube / (g.ncw * g.nch);
+  const int f0 = cf_i * g.cf, h0 = ch_i * g.ch, w0 = cw_i * g.cw;
+  const size_t src_head = static_cast<size_t>(bh) * g.N * d + v * 8;
+  const size_t dst_cube = (static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol) * d + v * 8;
+  const int r_lane = lane / vpr;
+  CubeWalk c;
+  c.init(g, r_lane);
+  const int steps = g.vol / rstep;
+  for (int k0 = 0; k0 < steps; k0 += kCubeUnroll) {
+    uint4 val[kCubeUnroll];
+#pragma unroll
+    for (int u = 0; u < kCubeUnroll; ++u) {
+      const int f = f0 + c.df, h = h0 + c.dh, w = w0 + c.dw;
+      const bool ok = k0 + u < steps && f < g.F && h < g.Hl && w < g.Wl;
+      val[u] = ok ? load8_as_bf16(src, src_head + static_cast<size_t>((f * g.Hl + h) * g.Wl + w) * d, kSrcF32)
+                  : make_uint4(0, 0, 0, 0);
+      c.advance(g, rstep);
+    }
+#pragma unroll
+    for (int u = 0; u < kCubeUnroll; ++u)
+      if (k0 + u < steps)
+        *reinterpret_cast<uint4*>(dst + dst_cube + static_cast<size_t>(r_lane + (k0 + u) * rstep) * d) = val[u];
+  }
+}
+
+// dst[bh, token] = src[bh, cube*vol + r] for every real token of the cube; same for LSE.
+template <bool kDstF32>
+__global__ void __launch_bounds__(kCubeWarps * 32) cube_unpermute_kernel(const __nv_bfloat16* __restrict__ src,
+                                                                        const float* __restrict__ src_lse,
+                                                                        void* __restrict__ dst,
+                                                                        float* __restrict__ dst_lse,
+                                                                        const uint8_t* __restrict__ kinds, Geom g,
+                                                                        int d) {
+  const int bh = blockIdx.y;
+  if (kinds[bh] != kCube) return;
+  const int cube = blockIdx.x * kCubeWarps + (threadIdx.x >> 5);
+  if (cube >= g.ncubes) return;
+  const int lane = threadIdx.x & 31;
+  const int vpr = d / 8, rstep = 32 / vpr;
+  const int v = lane % vpr;
+  const int cw_i = cube % g.ncw, ch_i = (cube / g.ncw) % g.nch, cf_i = cube / (g.ncw * g.nch);
+  const int f0 = cf_i * g.cf, h0 = ch_i * g.ch, w0 = cw_i * g.cw;
+  const size_t src_cube = (static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol) * d + v * 8;
+  const size_t dst_head = static_cast<size_t>(bh) * g.N * d + v * 8;
+  const bool lse = src_lse != nullptr && dst_lse != nullptr && v == 0;
+  const int r_lane = lane / vpr;
+  CubeWalk c;
+  c.init(g, r_lane);
+  const int steps = g.vol / rstep;
+  for (int k0 = 0; k0 < steps; k0 += kCubeUnroll) {
+    uint4 val[kCubeUnroll];
+    int tok[kCubeUnroll];
+#pragma unroll
+    for (int u = 0; u < kCubeUnroll; ++u) {
+      const int f = f0 + c.df, h = h0 + c.dh, w = w0 + c.dw;
+      const bool ok = k0 + u < steps && f < g.F && h < g.Hl && w < g.Wl;
+      tok[u] = ok ? (f * g.Hl + h) * g.Wl + w : -1;
+      val[u] = ok ? __ldg(reinterpret_cast<const uint4*>(src + src_cube +
+                                                         static_cast<size_t>(r_lane + (k0 + u) * rstep) * d))
+                  : make_uint4(0, 0, 0, 0);
+      c.advance(g, rstep);
+    }
+#pragma unroll
+    for (int u = 0; u < kCubeUnroll; ++u) {
+      if (tok[u] < 0) continue;
+      store8_from_bf16(dst, dst_head + static_cast<size_t>(tok[u]) * d, val[u], kDstF32);
+      if (lse)
+        dst_lse[static_cast<size_t>(bh) * g.N + tok[u]] =
+            src_lse[static_cast<size_t>(bh) * g.R + static_cast<size_t>(cube) * g.vol + r_lane + (k0 + u) * rstep];
+    }
+  }
+}
+
+// Row-copy grid: enough CTAs for every row, except with cube dims set, where the cube kernels
+// do the cube heads and the row kernel (grid-stride) only needs enough CTAs to fill the GPU
+// for the other heads; its CTAs of cube heads exit at once.
+static int perm_grid_x(const Geom& g, int rows, int d, int BH) {
   const int rows_per_cta = (kPermThreads / (d / 8)) * kPermUnroll;
   int x = (rows + rows_per_cta - 1) / rows_per_cta;
+  if (g.ncubes > 0) x = std::min(x, (148 * 16 + BH - 1) / BH);
   return x < 1 ? 1 : x;
 }
 
 cudaError_t launch_permute(const void* src, bool src_f32, void* dst, const uint8_t* kinds, const Geom& g, int BH,
                            int d, int* err, cudaStream_t stream) {
-  dim3 grid(perm_grid_x(g.R, d), BH);
+  dim3 grid(perm_grid_x(g, g.R, d, BH), BH);
   if (src_f32)
     permute_kernel<true><<<grid, kPermThreads, 0, stream>>>(src, static_cast<__nv_bfloat16*>(dst), kinds, g, d, err);
   else
     permute_kernel<false><<<grid, kPermThreads, 0, stream>>>(src, static_cast<__nv_bfloat16*>(dst), kinds, g, d, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || g.ncubes == 0) return e;
+  const dim3 cgrid((g.ncubes + kCubeWarps - 1) / kCubeWarps, BH);
+  auto* out = static_cast<__nv_bfloat16*>(dst);
+  if (src_f32)
+    cube_permute_kernel<true><<<cgrid, kCubeWarps * 32, 0, stream>>>(src, out, kinds, g, d);
+  else
+    cube_permute_kernel<false><<<cgrid, kCubeWarps * 32, 0, stream>>>(src, out, kinds, g, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const void* src, const float* src_lse, void* dst, bool dst_f32, float* dst_lse,
                              const uint8_t* kinds, const Geom& g, int BH, int d, int* err, cudaStream_t stream) {
-  dim3 grid(perm_grid_x(g.N, d), BH);
+  dim3 grid(perm_grid_x(g, g.N, d, BH), BH);
   const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
   if (dst_f32)
     unpermute_kernel<true><<<grid, kPermThreads, 0, stream>>>(s, src_lse, dst, dst_lse, kinds, g, d, err);
   else
     unpermute_kernel<false><<<grid, kPermThreads, 0, stream>>>(s, src_lse, dst, dst_lse, kinds, g, d, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || g.ncubes == 0) return e;
+  const dim3 cgrid((g.ncubes + kCubeWarps - 1) / kCubeWarps, BH);
+  if (dst_f32)
+    cube_unpermute_kernel<true><<<cgrid, kCubeWarps * 32, 0, stream>>>(s, src_lse, dst, dst_lse, kinds, g, d);
+  else
+    cube_unpermute_kernel<false><<<cgrid, kCubeWarps * 32, 0, stream>>>(s, src_lse, dst, dst_lse, kinds, g, d);
   return cudaGetLastError();
 }
 

@@ -34,15 +34,17 @@
  *     those intervals are at most w apart (the block-level cover of |f_q - f_k| <= w_s,
  *     respectively |s_q - s_k| <= w_t);
  *   - the window is the smallest w whose kept-block fraction reaches the target;
- *   - cube selection: fp64 mean of Q and K over each cube's real tokens, score
- *     qbar_c . kbar_c', keep the top k per row (score descending, ties to the smaller
- *     index) together with the cube itself;
+ *   - cube selection: fp64 mean of Q and K over each cube's real tokens (summed in token
+ *     order), score qbar_c . kbar_c' (summed in dimension order, one fused multiply-add
+ *     per term), keep the top k per row (score descending, ties to the smaller index)
+ *     together with the cube itself;
  *   - profiling rows rho_i = floor((2i+1) N / (2r)), r = ceil(frac * N); error = mean
  *     squared difference to dense attention on those rows under the block masks that
  *     would be executed; ties go to the spatial pattern;
  *   - a row with no allowed key has output 0 and log-sum-exp -inf.
  *
- * Build: gcc -O2 -fopenmp -shared -fPIC (no -ffast-math, no FMA contraction flags).
+ * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no -ffast-math; the only fused
+ * multiply-adds are the explicit fma() calls of the coarse scores).
  */
 #include <math.h>
 #include <stdint.h>
@@ -171,12 +173,12 @@ int or_cube_topk_keep(const double *q, const double *k, int64_t F, int64_t Hl, i
             qbar[c * d + x] /= (double)count[c];
             kbar[c * d + x] /= (double)count[c];
         }
-    /* coarse scores */
+    /* coarse scores: fp64 dot products in dimension order, one fused multiply-add per term */
 #pragma omp parallel for schedule(static)
     for (int64_t c = 0; c < C; ++c)
         for (int64_t c2 = 0; c2 < C; ++c2) {
             double acc = 0.0;
-            for (int64_t x = 0; x < d; ++x) acc += qbar[c * d + x] * kbar[c2 * d + x];
+            for (int64_t x = 0; x < d; ++x) acc = fma(qbar[c * d + x], kbar[c2 * d + x], acc);
             score[c * C + c2] = acc;
         }
     /* per row: pick the best remaining column topk times (selection by repeated max) */

@@ -142,6 +142,29 @@ def test_cube_masks_bit_exact(F, Hl, Wl, topk):
         assert np.array_equal(bits[0, h].numpy().view(np.uint32), oracle.keep_to_bits(keep))
 
 
+@pytest.mark.parametrize("F,Hl,Wl,topk,ties", [
+    (8, 16, 32, 8, True),      # 32 cubes, every score of a row equal: candidates = whole row
+    (64, 32, 64, 32, True),    # 1024 cubes, all equal: more candidates than the gather holds
+    (16, 16, 32, 40, False),   # topk above 32: full scan every round
+])
+def test_cube_topk_paths_bit_exact(F, Hl, Wl, topk, ties):
+    """The candidate filter, its overflow fallback and the full-scan path pick the same
+    cubes as the oracle, including the smaller-index rule on ties."""
+    wl = _wl(F, Hl, Wl, 128, 128, H=2, topk=topk)
+    q, k, _ = synthetic.make_qkv(wl)
+    if ties:  # K constant: within a row every coarse score is the same number
+        k = torch.ones_like(k)
+    bits, idx, cnt, max_kv, nblk = _run_masks(wl, [C_, C_], 0, 0, cubes=True, q=q, k=k)
+    for h in range(2):
+        keep = oracle.cube_topk_keep(q[0, h], k[0, h], F, Hl, Wl, topk, wl.cube)
+        want_idx, want_cnt = oracle.keep_to_lists(keep, max_kv)
+        assert np.array_equal(cnt[0, h].numpy(), want_cnt)
+        assert np.array_equal(idx[0, h].numpy(), want_idx)
+        if ties:
+            C = keep.shape[0]
+            assert keep[C - 1, :topk].all()      # the smallest indices win the ties
+
+
 def test_mask_overflow_flag():
     wl = _wl(21, 30, 52, 128, 128, H=1)
     shape = _shape(wl, False)
