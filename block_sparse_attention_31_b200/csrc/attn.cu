@@ -70,8 +70,11 @@ enum {
   B_DRAIN = 16
 };
 constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kPartial = 1u << 29, kKbMask = (1u << 29) - 1u;
-// Probability pairs (2 columns) whose exponentials run on the FMA pipe: 1 pair in 8.
-constexpr int kPolyPairMask = 7;
+// Probability pairs (2 columns) whose exponentials run on the FMA pipe: kPolyPairs8 in 8.
+#ifndef VSA_POLY_PAIRS8
+#define VSA_POLY_PAIRS8 1
+#endif
+constexpr int kPolyPairs8 = VSA_POLY_PAIRS8;
 
 // One CTA per pair of consecutive query blocks (tiles 0 and 1) of one head.  The K/V blocks
 // of the union of the two lists stream through a 2-stage ring once and serve both tiles; the
@@ -197,15 +200,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (lane == 0) misc[2] = base;
     __syncwarp();
-    // valid-key bits of the blocks that are not full (ragged tail, cube padding)
+    // valid-key bits of the blocks that are not full (ragged tail, cube padding).  A cube
+    // block is one cube (V == BN); its slot r = (df*ch + dh)*cw + dw holds a token when the
+    // offsets fall inside the cube's real extent, and the offsets of r = 32w + lane are the
+    // same for every cube, so they are computed once.
+    int cdw[BN / 32], cdh[BN / 32], cdf[BN / 32];
+    if (kind == kCube) {
+#pragma unroll
+      for (int w = 0; w < BN / 32; ++w) {
+        const int r = w * 32 + lane;
+        cdw[w] = r % g.cw;
+        cdh[w] = (r / g.cw) % g.ch;
+        cdf[w] = r / (g.cw * g.ch);
+      }
+    }
     for (int n = 0; n < base; ++n) {
       const uint32_t e = uni[n];
       if (!(e & kPartial)) continue;
       const int kb = static_cast<int>(e & kKbMask);
+      int nf = 0, nh = 0, nw = 0;
+      if (kind == kCube) {
+        const int cw_i = kb % g.ncw, ch_i = (kb / g.ncw) % g.nch, cf_i = kb / (g.ncw * g.nch);
+        nf = min(g.cf, g.F - cf_i * g.cf);
+        nh = min(g.ch, g.Hl - ch_i * g.ch);
+        nw = min(g.cw, g.Wl - cw_i * g.cw);
+      }
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) {
-        const int slot = kb * BN + w * 32 + lane;
-        const bool ok = kind == kCube ? token_of_slot(g, kCube, slot) >= 0 : slot < g.N;
+        const bool ok = kind == kCube ? (cdf[w] < nf && cdh[w] < nh && cdw[w] < nw) : kb * BN + w * 32 + lane < g.N;
         const uint32_t m = __ballot_sync(0xffffffffu, ok);
         if (lane == 0) uvalid[n * (BN / 32) + w] = m;
       }
@@ -408,7 +430,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_ld();
           reg_fence<64>(r);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
+          for (int c = 0; c < 32; ++c)
+            mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
         }
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -434,9 +457,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float m_use = m == -INFINITY ? 0.f : m;
         // pass 2: 64 scores at a time -> 32 packed bf16 pairs written over the consumed S columns;
         // the row sum is kept in eight partial sums
-        float rs8[8];
+        // (scale and max subtraction, row sums and the polynomial exponentials on packed pairs)
+        uint64_t rs4[4];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) rs8[x] = 0.f;
+        for (int x = 0; x < 4; ++x) rs4[x] = 0ull;
+        const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
 #pragma unroll
         for (int h = 0; h < BN / 64; ++h) {
           uint32_t r[64];
@@ -447,18 +472,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float x0 = fmaf(__uint_as_float(r[2 * c]), sl2, -m_use);
-            const float x1 = fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m_use);
-            const bool poly = (c & kPolyPairMask) == kPolyPairMask;
-            const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
-            const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
-            rs8[(2 * c) & 7] += p0;
-            rs8[(2 * c + 1) & 7] += p1;
+            const uint64_t x = f2_fma(f2_make(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2x2, negm2);
+            uint64_t p;
+            if ((c & 7) >= 8 - kPolyPairs8) {
+              p = exp2_poly2(x);
+            } else {
+              float x0, x1;
+              f2_split(x, x0, x1);
+              p = f2_make(fast_exp2(x0), fast_exp2(x1));
+            }
+            rs4[c & 3] = f2_add(rs4[c & 3], p);
+            float p0, p1;
+            f2_split(p, p0, p1);
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st32_u(t_s + h * 32, pk);
         }
-        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        {
+          const uint64_t s2 = f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3]));
+          float s0, s1;
+          f2_split(s2, s0, s1);
+          l += s0 + s1;
+        }
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL + t));
       }

@@ -11,7 +11,14 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
                                      float* __restrict__ y_mufu, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
-    y_poly[i] = exp2_poly(x[i]);
+    // the packed form the attention kernel runs, on the pair (x[i], x[i ^ 1]); it must agree
+    // with the scalar form bit for bit, else the result is NaN
+    const float other = (i ^ 1) < n ? x[i ^ 1] : 0.0f;
+    float lo, hi;
+    f2_split(exp2_poly2((i & 1) ? f2_make(other, x[i]) : f2_make(x[i], other)), lo, hi);
+    const float packed = (i & 1) ? hi : lo;
+    const float scalar = exp2_poly(x[i]);
+    y_poly[i] = __float_as_uint(packed) == __float_as_uint(scalar) ? scalar : __int_as_float(0x7fc00000);
     y_mufu[i] = fast_exp2(x[i]);
   }
 }

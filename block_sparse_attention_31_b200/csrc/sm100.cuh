@@ -300,6 +300,58 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x < -125.0f ? 0.0f : r;
 }
 
+// ---- packed fp32 pairs (two lanes of one 64-bit register pair per instruction) ----
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_split(uint64_t d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max of three floats in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly on a packed pair: the rounding split and the cubic run as f32x2 operations.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_split(x, x0, x1);
+  const uint64_t xc = f2_make(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t magic = f2_make(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(xc, magic);
+  const uint64_t n = f2_add(t, f2_make(-12582912.0f, -12582912.0f));       // round(xc)
+  const uint64_t f = f2_fma(n, f2_make(-1.0f, -1.0f), xc);                  // xc - round(xc), exact
+  uint64_t p = f2_fma(f2_make(0.05517149344086647f, 0.05517149344086647f), f,
+                      f2_make(0.24261093139648438f, 0.24261093139648438f));
+  p = f2_fma(p, f, f2_make(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_make(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2_make(x0 < -125.0f ? 0.0f : r0, x1 < -125.0f ? 0.0f : r1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
