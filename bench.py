@@ -90,53 +90,94 @@ def attention_work(wl, kinds, kv_idx, kv_cnt):
 # clocks
 # ---------------------------------------------------------------------------------------
 
+def gpu_smi_id(device_index: int) -> str:
+    """nvidia-smi's name for a torch device: its PCI address (indices differ when
+    CUDA_VISIBLE_DEVICES reorders or hides GPUs)."""
+    try:
+        p = torch.cuda.get_device_properties(device_index)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except (AttributeError, RuntimeError):
+        return str(device_index)
+
+
 class ClockSampler:
+    """nvidia-smi clock samples, each stamped with the host time it arrived; only samples
+    inside mark_start()..mark_stop() are summarised (the neighbours of the window when none
+    fall inside it, flagged "window": "nearest")."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
-        self.proc = None
+    def __init__(self, smi_id: str, period_ms: int = 20):
+        self.idx, self.period = smi_id, period_ms
+        self.proc, self.samples, self.t0, self.t1 = None, [], None, None
+
+    def _reader(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.monotonic(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        deadline = time.monotonic() + 5.0
+        while not self.samples and time.monotonic() < deadline:  # sampler running before timing starts
+            time.sleep(0.01)
         return self
 
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_stop(self):
+        self.t1 = time.monotonic()
+        time.sleep(2.0 * self.period / 1000.0)  # let the sample after the window arrive
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        rows = []
+        for t, ln in self.samples:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                rows.append((t, float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        window = "inside"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if self.t0 <= r[0] <= self.t1]
+            if not inside and rows:  # region shorter than the sampling period
+                before = [r for r in rows if r[0] < self.t0][-1:]
+                after = [r for r in rows if r[0] > self.t1][:1]
+                inside, window = before + after, "nearest"
+            rows = inside
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median([r[1] for r in rows]), "sm_max_mhz": rows[-1][2],
+                "reasons": sorted(reasons), "samples": len(rows), "window": window,
+                "period_ms": self.period}
 
 
 # ---------------------------------------------------------------------------------------
@@ -257,12 +298,14 @@ def gpu_arm(args, wl, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(gpu_smi_id(torch.cuda.current_device())) as clk:
+        clk.mark_start()
         start.record()
         for i in range(args.steps):
             pipe.step(qd, kd, vd, o, evs[i])
         stop.record()
         torch.cuda.synchronize()
+        clk.mark_stop()
     if world > 1:
         torch.distributed.barrier()
     total_ms = start.elapsed_time(stop)
