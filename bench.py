@@ -34,6 +34,10 @@ if ROOT not in sys.path:
 import synthetic  # noqa: E402
 
 METRIC = "ms/attention call and effective TFLOP/s (sparse & dense-equiv) vs bf16 peak"
+# DRAM bytes (read + write) per launch of the attention kernel from one ncu capture of the current
+# kernel on that workload (profiles/ has the command and the figures); absent -> null.
+TRAFFIC = {}
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -84,6 +88,51 @@ def attention_work(wl, kinds, kv_idx, kv_cnt):
                 exe += 4.0 * wl.d * 128 * wl.block * cnt[i]
                 pairs += int(cnt[i])
     return alg, exe, pairs
+
+
+def stage_work(wl, kinds, pipe, pairs):
+    """Algorithmic bytes (HBM stages) or executed flops (profiling) per call of each stage,
+    and the number of exponentials the attention evaluates."""
+    from block_sparse_attention_31_b200 import _lib
+    N, d, row = wl.N, wl.d, wl.d * 2
+    R = _lib.vsa_layout_rows(pipe.shape)
+    n_t = sum(1 for k in kinds if k == _lib.VSA_TEMPORAL)
+    n_c = sum(1 for k in kinds if k == _lib.VSA_CUBE)
+    BH = wl.B * wl.H
+    # permute: temporal heads read and write N rows; cube heads read N real rows and write every
+    # one of the R slots (padding zeroed); spatial bf16 heads are read in place (no copy)
+    perm = 3.0 * (n_t * 2 * N + n_c * (N + R)) * row
+    unperm = (n_t + n_c) * 2.0 * N * row
+    nwords = -(-pipe.nblk // 32)
+    mask = BH * pipe.nblk * (nwords + pipe.max_kv + 1) * 4.0
+    if wl.mode == "cube":
+        C = R // (wl.cube[0] * wl.cube[1] * wl.cube[2])
+        mask += n_c * (2.0 * R * row + 2.0 * 2 * C * d * 8 + 2.0 * C * C * 8)  # pool reads, means, scores w+r
+    out = {"permute": {"bytes": perm, "bound": "hbm"}, "unpermute": {"bytes": unperm, "bound": "hbm"},
+           "mask": {"bytes": mask, "bound": "hbm"}}
+    if wl.mode == "profiled":
+        r = _lib.vsa_profile_rows(pipe.shape, pipe.params)
+        # tensor work of the profiling kernel: Q.K^T once and three P.V over all N keys
+        out["profile"] = {"flops": BH * 8.0 * d * r * N, "bound": "tensor", "rows": r}
+    exp2 = float(pairs) * 128 * wl.block
+    return out, exp2
+
+
+def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
+    out = {}
+    for name, w in work.items():
+        t = stage_ms[name] / 1e3
+        if t <= 0:
+            continue
+        if w["bound"] == "hbm":
+            gbs = w["bytes"] / t / 1e9
+            out[name] = {"bound": "hbm", "bytes": w["bytes"], "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": gbs / hbm_gbs}
+        else:
+            tf = w["flops"] / t / 1e12
+            out[name] = {"bound": "tensor", "flops": w["flops"], "achieved": tf, "peak": tensor_tflops,
+                         "unit": "TFLOP/s", "frac": tf / tensor_tflops}
+    return out
 
 
 # ---------------------------------------------------------------------------------------
@@ -290,6 +339,7 @@ def gpu_arm(args, wl, rank, world, device):
     alg, exe, pairs = attention_work(wl, pipe.kinds.cpu().numpy(), pipe.kv_idx.cpu().numpy(),
                                      pipe.kv_cnt.cpu().numpy())
     dense = synthetic.dense_flops(wl)
+    swork, exp2 = stage_work(wl, pipe.kinds.cpu().tolist(), pipe, pairs)
     nb = -(-wl.N // wl.block)
     kept_frac = pairs / (wl.B * wl.H * float(pipe.nblk if wl.mode == "cube" else nb) ** 2)
     # timed region
@@ -318,6 +368,7 @@ def gpu_arm(args, wl, rank, world, device):
     e2e = e2e_arm(args, wl, q, k, v, device)
     e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], device)
     return dict(ms=ms, stage_ms=stage_ms, alg=alg, exe=exe, dense=dense, pairs=pairs, kept=kept_frac,
+                swork=swork, exp2=exp2,
                 clocks=clk.summary(), launches=pipe.launches, e2e=e2e, w_s=pipe.params.w_s, w_t=pipe.params.w_t,
                 kinds=pipe.kinds.cpu().tolist())
 
@@ -488,11 +539,15 @@ def main():
         "dense_equiv_tflops": aggregate_tflops(res["dense"], res["ms"], world),
         "stage_ms": res["stage_ms"],
         "roofline": {"kernel": "vsa_sparse_attn_fwd", "bound": "tensor", "achieved": achieved,
-                     "peak": peak_sust, "unit": "TFLOP/s", "frac": achieved / peak_sust,
-                     "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
-                     "frac_of_burst_peak": achieved / peak_burst,
+                     "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                     "peak_source": f"{src} bf16_tflops (burst; the kernel runs at the maximum SM clock, "
+                                    "see clocks)",
+                     "frac_of_sustained_peak": achieved / peak_sust,
                      "executed_tflops": res["exe"] / attn_s / 1e12,
-                     "traffic": None},
+                     "executed_frac": res["exe"] / attn_s / 1e12 / peak_burst,
+                     "traffic": TRAFFIC.get(wl.name)},
+        "stage_roofline": stage_roofline(res["swork"], res["stage_ms"], float(peaks["hbm_gbs"]), peak_burst),
+        "softmax_exp2_per_call": res["exp2"],
         "gpu_launches": res["launches"] * args.steps,
         "clocks": res["clocks"],
         "e2e": {"value": aggregate_tflops(res["alg"], res["e2e"]["ms_per_step"], world), "unit": "TFLOP/s",
