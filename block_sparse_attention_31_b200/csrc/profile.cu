@@ -34,6 +34,7 @@ namespace vsa {
 constexpr int kProfThreads = 192;
 constexpr int kPM = 128;  // rows per tile
 constexpr int kNumSMs = 148;
+constexpr int kMaxSplits = 16;  // key-range splits per row tile, at most
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -54,14 +55,14 @@ ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
     return w / std::ceil(w);
   };
   int splits = 0;
-  for (int s = 1; s <= 16 && s <= nb; ++s)
+  for (int s = 1; s <= kMaxSplits && s <= nb; ++s)
     if (tiles * s >= kNumSMs && wave_eff(s) >= 0.9) {
       splits = s;
       break;
     }
   if (splits == 0) {
     splits = 1;
-    for (int s = 2; s <= 16 && s <= nb; ++s)
+    for (int s = 2; s <= kMaxSplits && s <= nb; ++s)
       if (wave_eff(s) > wave_eff(splits) + 1e-9) splits = s;
   }
   p.splits = splits;
@@ -84,6 +85,7 @@ ProfilePlan profile_plan_splits(const Geom& g, int BH, int d, double frac, int s
   ProfilePlan p = profile_plan(g, BH, d, frac);
   const int nb = (g.N + g.block - 1) / g.block;
   p.splits = splits < 1 ? 1 : (splits > nb ? nb : splits);
+  if (p.splits > kMaxSplits) p.splits = kMaxSplits;
   size_t off = p.off_opart;
   off = align256(off + static_cast<size_t>(BH) * p.splits * 3 * p.r_pad * d * sizeof(float));
   p.off_ml = off;
@@ -95,18 +97,27 @@ ProfilePlan profile_plan_splits(const Geom& g, int BH, int d, double frac, int s
 }
 
 // Contiguous range [lo, hi] of key blocks kept for query block i, groups of G slots.
+// Block j spans groups [a_j, b_j]; both ends are non-decreasing in j, so the blocks kept for
+// block i (max(0, a_j - b_i, a_i - b_j) <= w) are the contiguous run from the first j with
+// b_j >= a_i - w to the last j with a_j <= b_i + w.  Two binary searches find it.
 __device__ __forceinline__ void kept_block_range(int i, int N, int B, int G, int w, int& lo, int& hi) {
   const int nb = (N + B - 1) / B;
   const int ai = (i * B) / G, bi = (min(N, (i + 1) * B) - 1) / G;
-  lo = nb;
-  hi = -1;
-  for (int j = 0; j < nb; ++j) {
-    const int aj = (j * B) / G, bj = (min(N, (j + 1) * B) - 1) / G;
-    if (max(0, max(aj - bi, ai - bj)) <= w) {
-      lo = min(lo, j);
-      hi = j;
-    }
+  int l = 0, h = nb;  // first j in [0, nb) with b_j >= ai - w
+  while (l < h) {
+    const int m = (l + h) >> 1;
+    if ((min(N, (m + 1) * B) - 1) / G >= ai - w) h = m;
+    else l = m + 1;
   }
+  lo = l;
+  l = 0;
+  h = nb;  // first j with a_j > bi + w
+  while (l < h) {
+    const int m = (l + h) >> 1;
+    if ((m * B) / G > bi + w) h = m;
+    else l = m + 1;
+  }
+  hi = l - 1;
 }
 
 __global__ void __launch_bounds__(256) profile_prep_kernel(const __nv_bfloat16* __restrict__ q, Geom g, int d, int r,
@@ -421,6 +432,28 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
       const bool tp_on = tany != 0u;
+      // Exponentials first, into registers (packed bf16 pairs): this overlaps the previous
+      // block's P.V products, which still read the P tiles.
+      const float m_next = grow ? m_new : m;
+      const float m_use = m_next == -INFINITY ? 0.f : m_next;
+      const bool warp_tp = __any_sync(0xffffffffu, tp_on);
+      const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
+      uint64_t rs2[2] = {0ull, 0ull};
+      float rt4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN / 2; ++c) {
+        const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
+        float x0, x1;
+        f2_split(x, x0, x1);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
+        pk[c] = pack_bf16x2(p0, p1);
+        if (warp_tp) {
+          const uint32_t b = (mt[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
+          rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+        }
+      }
       // the previous block's P.V products must be done: O stable, P tiles free
       if (j > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (j - 1) & 1, abort_flag, a.err));
@@ -445,41 +478,26 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         l[2] *= alpha;
         m = m_new;
       }
-      const float m_use = m == -INFINITY ? 0.f : m;
-      const bool warp_tp = __any_sync(0xffffffffu, tp_on);
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f}, rt4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ch = 0; ch < BN / 8; ++ch) {  // 8 probabilities -> one 16-byte chunk of each P tile
-        uint4 v4;
-        uint32_t* w4 = reinterpret_cast<uint32_t*>(&v4);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int col = ch * 8 + 2 * x;
-          const float p0 = fast_exp2(fmaf(s[col], sl2, -m_use));
-          const float p1 = fast_exp2(fmaf(s[col + 1], sl2, -m_use));
-          rs4[x] += p0 + p1;
-          w4[x] = pack_bf16x2(p0, p1);
-          if (warp_tp) {
-            const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-            rt4[x] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
-          }
-        }
+        const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         const int kc = ch >> 3, cc = ch & 7;
         const int off = kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(pPD + off) = v4;
         if (tp_on) {
-          uint4 t4;
-          uint32_t* m4 = reinterpret_cast<uint32_t*>(&t4);
+          uint32_t m4[4];
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             const int col = ch * 8 + 2 * x;
             const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-            m4[x] = w4[x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
+            m4[x] = pk[4 * ch + x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
           }
-          *reinterpret_cast<uint4*>(pPT + off) = t4;
+          *reinterpret_cast<uint4*>(pPT + off) = make_uint4(m4[0], m4[1], m4[2], m4[3]);
         }
       }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      float rs0, rs1;
+      f2_split(f2_add(rs2[0], rs2[1]), rs0, rs1);
+      const float rs = rs0 + rs1;
       const float rt = (rt4[0] + rt4[1]) + (rt4[2] + rt4[3]);
       l[0] += rs;
       if (sp_on) l[1] += rs;
@@ -536,19 +554,29 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
   float o[3];
 #pragma unroll
   for (int vv = 0; vv < 3; ++vv) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) {
-      const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-      M = fmaxf(M, ml[prow * 2]);
+    // all splits' partials are loaded before they are combined (at most kMaxSplits)
+    float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      ms[sp] = -INFINITY;
+      ls[sp] = os[sp] = 0.f;
+      if (sp < splits) {
+        const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
+        ms[sp] = __ldg(ml + prow * 2);
+        ls[sp] = __ldg(ml + prow * 2 + 1);
+        os[sp] = __ldg(opart + prow * d + x);
+      }
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) M = fmaxf(M, ms[sp]);
     float L = 0.f, acc = 0.f;
-    for (int sp = 0; sp < splits; ++sp) {
-      const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-      const float ms = ml[prow * 2];
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      L += ml[prow * 2 + 1] * w;
-      acc += opart[prow * d + x] * w;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      if (ms[sp] == -INFINITY) continue;
+      const float w = exp2f(ms[sp] - M);
+      L += ls[sp] * w;
+      acc += os[sp] * w;
     }
     o[vv] = L > 0.f ? acc / L : 0.f;
   }
@@ -627,6 +655,7 @@ cudaError_t launch_profile(const void* q, const void* k, const void* v, const Ge
   int4* ranges = reinterpret_cast<int4*>(w + plan.off_ranges);
   float* opart = reinterpret_cast<float*>(w + plan.off_opart);
   float* ml = reinterpret_cast<float*>(w + plan.off_ml);
+  if (plan.splits < 1 || plan.splits > kMaxSplits) return cudaErrorInvalidValue;
   {
     const int vpr = d / 8;
     dim3 grid((plan.r_pad * vpr + 255) / 256, BH);
