@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) cube_score_kernel(const doub
 
 constexpr int kTopkWarps = 4;
 constexpr int kTopkCap = 512;  // candidates per row kept for the exact selection
+constexpr int kLaneTop = 8;    // largest keys each lane keeps for the candidate bound
 
 // Order-preserving integer key of a finite double (larger value <-> larger key); -0 and +0,
 // equal as doubles, get the same key.
@@ -240,11 +241,12 @@ __device__ __forceinline__ int warp_argmax_key(uint64_t k, int c) {
 // Top-k of one score row per warp (score descending, ties to the smaller index) plus the own
 // cube; emits the bitset, the ascending list and the count.
 //
-// Fast path (topk <= 32): the smallest of the 32 lane maxima is a lower bound L on the k-th
-// largest score, since those 32 maxima are distinct entries that are all >= L.  Only entries
-// >= L (typically a few per cent of the row) are gathered, and the exact selection runs on
-// them.  With more than kTopkCap candidates, or topk > 32, every round scans the whole row.
-__global__ void __launch_bounds__(kTopkWarps * 32) cube_topk_kernel(const double* __restrict__ scores,
+// Fast path (topk <= 32): every lane keeps its kLaneTop largest keys; the k-th largest of those
+// 32*kLaneTop keys is a lower bound L on the row's k-th largest score, since k distinct entries
+// are >= L.  Only entries >= L (about k, unless a lane held more than kLaneTop of the winners)
+// are gathered, and the exact selection runs on them.  With more than kTopkCap candidates, or
+// topk > 32, every round scans the whole row.
+__global__ void __launch_bounds__(kTopkWarps * 32, 1) cube_topk_kernel(const double* __restrict__ scores,
                                                                     const uint8_t* __restrict__ kinds, Geom g,
                                                                     int topk, uint32_t* __restrict__ bits,
                                                                     int32_t* __restrict__ kv_idx,
@@ -270,12 +272,33 @@ __global__ void __launch_bounds__(kTopkWarps * 32) cube_topk_kernel(const double
   const int picks = topk < C ? topk : C;
   bool exact_scan = picks > 32;
   if (!exact_scan && picks > 0) {
-    uint64_t lmax = 0ull;  // 0: below every finite key
-    for (int c = lane; c < C; c += 32) lmax = max(lmax, score_key(__ldg(grow + c)));
-    const uint32_t lhi = static_cast<uint32_t>(lmax >> 32), llo = static_cast<uint32_t>(lmax);
-    const uint32_t bhi = __reduce_min_sync(0xffffffffu, lhi);
-    const uint32_t blo = __reduce_min_sync(0xffffffffu, lhi == bhi ? llo : 0xffffffffu);
-    const uint64_t bound = (static_cast<uint64_t>(bhi) << 32) | blo;
+    // each lane's kLaneTop largest keys, descending (0: empty, below every finite key)
+    uint64_t tk[kLaneTop];
+#pragma unroll
+    for (int j = 0; j < kLaneTop; ++j) tk[j] = 0ull;
+    for (int c = lane; c < C; c += 32) {
+      const uint64_t k = score_key(__ldg(grow + c));
+      if (k > tk[kLaneTop - 1]) {
+#pragma unroll
+        for (int j = kLaneTop - 1; j > 0; --j) tk[j] = max(tk[j], min(k, tk[j - 1]));
+        tk[0] = max(tk[0], k);
+      }
+    }
+    // the picks-th largest key of all lanes' lists: picks real entries are >= it, so it bounds
+    // the picks-th largest score of the row from below
+    uint64_t bound = 0ull;
+    for (int p = 0; p < picks; ++p) {
+      const uint32_t hi = static_cast<uint32_t>(tk[0] >> 32), lo = static_cast<uint32_t>(tk[0]);
+      const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+      bound = (static_cast<uint64_t>(mhi) << 32) | mlo;
+      const uint32_t holders = __ballot_sync(0xffffffffu, tk[0] == bound);
+      if (lane == __ffs(holders) - 1) {  // that lane's head is taken
+#pragma unroll
+        for (int j = 0; j < kLaneTop - 1; ++j) tk[j] = tk[j + 1];
+        tk[kLaneTop - 1] = 0ull;
+      }
+    }
     int n = 0;
     for (int c0 = 0; c0 < C; c0 += 32) {
       const int c = c0 + lane;
