@@ -310,6 +310,35 @@ def test_attention_block_order(F, Hl, Wl):
     _attention_case(wl, [C_, S_, T_], keeps, q, k, v, perm=True, ordered=True)
 
 
+@pytest.mark.parametrize("q_scale", [0.0, 1.0, 8.0])
+def test_attention_weights_within_bf16_rounding(q_scale):
+    """With V rows = 64 * unit vectors, O[i, j] = 64 * P[i, j] / l: the kernel's softmax weights
+    seen directly.  Their error is bf16 rounding of P (half an ulp, 2^-8 relative) plus the
+    bf16 rounding of the output (another 2^-8); Q = 0 gives equal weights, exactly."""
+    d = N = 128
+    shape = _lib.make_shape(1, 1, 1, 1, N, d, 128)
+    g = torch.Generator().manual_seed(1)
+    q = (torch.randn(1, 1, N, d, generator=g) * q_scale).to(torch.bfloat16)
+    k = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    v = (torch.eye(N, d) * 64).reshape(1, 1, N, d).to(torch.bfloat16)
+    o = torch.empty(1, 1, N, d, dtype=torch.bfloat16, device="cuda")
+    kinds = torch.zeros(1, dtype=torch.uint8, device="cuda")
+    idx = torch.zeros(1, 1, 1, 1, dtype=torch.int32, device="cuda")
+    cnt = torch.ones(1, 1, 1, dtype=torch.int32, device="cuda")
+    err = cuda_err()
+    _lib.vsa_sparse_attn_fwd(_lib.qkvo(q.cuda(), k.cuda(), v.cuda(), o), None, kinds, idx, cnt, 1, shape, 0.0, err)
+    assert _lib.vsa_get_device_error(err) == 0
+    s = (q[0, 0].double() @ k[0, 0].double().T) / math.sqrt(d)
+    want = torch.softmax(s, dim=1) * 64
+    got = o[0, 0].cpu().double()
+    if q_scale == 0.0:
+        assert torch.equal(got, torch.full_like(got, 0.5))
+        return
+    big = want > 1e-3
+    rel = ((got - want).abs() / want)[big]
+    assert rel.max() <= 2.0 ** -7 * 1.01, rel.max()
+
+
 def test_attention_large_scores_stable():
     """Inputs scaled x8: logits up to a few hundred must not overflow the online softmax."""
     wl = _wl(3, 8, 16, 128, 128, H=1)

@@ -41,25 +41,26 @@ def _run(wl, rows_per_head=None, seed_rows=0, heads=None):
     o, lse = plan(q.cuda(), k.cuda(), v.cuda(), kinds=kinds)
     assert plan.device_error() == 0
     o, lse = o.cpu(), lse.cpu()
-    got_kinds = plan.kinds.cpu().numpy()
+    got_kinds = plan.kinds.cpu().numpy()  # [B*H]
     heads = range(wl.H) if heads is None else heads
-    for h in heads:
-        kind = int(got_kinds[h])
-        if wl.mode == "profiled":
-            want_kind, _, _ = oracle.profile_head(q[0, h], k[0, h], v[0, h], wl.F, wl.Hl, wl.Wl, wl.block, plan.w_s,
-                                                  plan.w_t, wl.profile_frac)
-            assert kind == want_kind, h
-        keep = keep_for_head(kind, wl, plan.w_s, plan.w_t, q[0, h], k[0, h])
-        # the masks the kernels executed
-        nb = keep.shape[0]
-        want_idx, want_cnt = oracle.keep_to_lists(keep, plan.max_kv)
-        assert np.array_equal(plan.kv_cnt[0, h, :nb].cpu().numpy(), want_cnt)
-        assert np.array_equal(plan.kv_idx[0, h, :nb].cpu().numpy(), want_idx)
-        rows = (np.arange(wl.N) if rows_per_head is None else
-                synthetic.sample_indices(wl.N, rows_per_head, seed_rows + h).numpy())
-        want, want_lse = oracle_rows(q[0, h], k[0, h], v[0, h], kind, wl, keep, rows)
-        assert_close_attention(to_f64(o[0, h])[rows], want, f"{wl.name} head {h}")
-        assert np.abs(to_f64(lse[0, h])[rows] - want_lse).max() < 2e-2
+    for b in range(wl.B):
+        for h in heads:
+            kind = int(got_kinds[b * wl.H + h])
+            if wl.mode == "profiled":
+                want_kind, _, _ = oracle.profile_head(q[b, h], k[b, h], v[b, h], wl.F, wl.Hl, wl.Wl, wl.block,
+                                                      plan.w_s, plan.w_t, wl.profile_frac)
+                assert kind == want_kind, (b, h)
+            keep = keep_for_head(kind, wl, plan.w_s, plan.w_t, q[b, h], k[b, h])
+            # the masks the kernels executed
+            nb = keep.shape[0]
+            want_idx, want_cnt = oracle.keep_to_lists(keep, plan.max_kv)
+            assert np.array_equal(plan.kv_cnt[b, h, :nb].cpu().numpy(), want_cnt)
+            assert np.array_equal(plan.kv_idx[b, h, :nb].cpu().numpy(), want_idx)
+            rows = (np.arange(wl.N) if rows_per_head is None else
+                    synthetic.sample_indices(wl.N, rows_per_head, seed_rows + b * wl.H + h).numpy())
+            want, want_lse = oracle_rows(q[b, h], k[b, h], v[b, h], kind, wl, keep, rows)
+            assert_close_attention(to_f64(o[b, h])[rows], want, f"{wl.name} batch {b} head {h}")
+            assert np.abs(to_f64(lse[b, h])[rows] - want_lse).max() < 2e-2
     return plan
 
 
@@ -73,6 +74,18 @@ def test_tiny_fixed_masks_full():
 def test_small_profiled_full():
     wl = synthetic.Workload("small profiled", 1, 4, 8, 12, 20, 128, 128, "bf16", "profiled", target=0.3,
                             profile_frac=0.05)
+    _run(wl)
+
+
+def test_batched_profiled_full():
+    """B = 2: every (batch, head) is profiled, masked and attended on its own."""
+    wl = synthetic.Workload("batched profiled", 2, 3, 7, 10, 18, 128, 128, "bf16", "profiled", target=0.3,
+                            profile_frac=0.05)
+    _run(wl)
+
+
+def test_batched_cube_full():
+    wl = synthetic.Workload("batched cubes", 2, 2, 16, 16, 32, 128, 128, "bf16", "cube", cube=(4, 4, 8), topk=32)
     _run(wl)
 
 
