@@ -90,6 +90,62 @@ class SparseAttention:
                       self.mse, self.ws, self.ws_bytes, self.err, stream)
         return (out, lse) if self.with_lse else out
 
+    def run_host(self, batches, outs=None, kinds: Optional[torch.Tensor] = None, timing=None):
+        """Run the call on a sequence of host batches with the transfers overlapped: while call i
+        computes, the inputs of call i+1 upload and the output of call i-1 downloads (three
+        streams, two device buffer sets).  ``batches`` is a list of (q, k, v) CPU tensors, which
+        must be pinned for the copies to overlap; ``outs`` is a list of CPU output tensors
+        (pinned ones are allocated when None).  Returns ``outs`` once every output has arrived.
+        The log-sum-exp, when configured, stays on the device and is not returned.  ``timing``, a
+        pair of timing-enabled CUDA events, is recorded before the first upload and after the
+        last download."""
+        n = len(batches)
+        shape = (self.B, self.H, self.N, self.d)
+        if outs is None:
+            outs = [torch.empty(shape, dtype=self.dtype).pin_memory() for _ in range(n)]
+        if len(outs) != n:
+            raise ValueError("need one output tensor per batch")
+        for (q, k, v), o in zip(batches, outs):
+            for t in (q, k, v, o):
+                if t.device.type != "cpu" or t.dtype != self.dtype or tuple(t.shape) != shape:
+                    raise ValueError(f"host tensors of shape {shape} and dtype {self.dtype} expected")
+        if not hasattr(self, "_host_bufs"):
+            self._host_bufs = [[torch.empty(shape, dtype=self.dtype, device=self.device) for _ in range(4)]
+                               for _ in range(2)]  # q, k, v, o per buffer set
+            self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]  # upload, compute, download
+        up, comp, down = self._streams
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        up_done, comp_done, down_done = [], [], []
+        up.wait_stream(torch.cuda.current_stream(self.device))
+        if timing is not None:
+            timing[0].record(up)
+        for i, ((q, k, v), o) in enumerate(zip(batches, outs)):
+            dq, dk, dv, do = self._host_bufs[i % 2]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[i - 2])  # call i-2 has read this buffer set
+                dq.copy_(q, non_blocking=True)
+                dk.copy_(k, non_blocking=True)
+                dv.copy_(v, non_blocking=True)
+                up_done.append(ev())
+                up_done[i].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(up_done[i])
+                if i >= 2:
+                    comp.wait_event(down_done[i - 2])  # call i-2's output has left this buffer
+                self(dq, dk, dv, out=do, kinds=kinds, stream=comp)
+                comp_done.append(ev())
+                comp_done[i].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[i])
+                o.copy_(do, non_blocking=True)
+                down_done.append(ev())
+                down_done[i].record(down)
+        if timing is not None:
+            timing[1].record(down)
+        down.synchronize()
+        return outs
+
     def device_error(self) -> int:
         return vsa_get_device_error(self.err)
 

@@ -115,3 +115,17 @@ def test_repeated_calls_identical():
     o2, l2 = plan(q, k, v)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert plan.device_error() == 0
+
+
+def test_run_host_overlapped_matches_single_calls():
+    """run_host (uploads, compute and downloads of consecutive calls overlapped on three
+    streams) returns exactly what one call per batch returns."""
+    wl = synthetic.Workload("host", 1, 4, 6, 8, 16, 128, 128, "bf16", "profiled", target=0.3, profile_frac=0.05)
+    plan = _plan(wl)
+    batches = [tuple(t.pin_memory() for t in synthetic.make_qkv(wl, seed=s)) for s in range(5)]
+    outs = plan.run_host(batches)
+    assert plan.device_error() == 0
+    for (q, k, v), got in zip(batches, outs):
+        want = plan(q.cuda(), k.cuda(), v.cuda())
+        want = want[0] if isinstance(want, tuple) else want
+        assert torch.equal(got, want.cpu())
