@@ -101,8 +101,9 @@ def stage_work(wl, kinds, pipe, pairs):
     BH = wl.B * wl.H
     # permute: temporal heads read and write N rows; cube heads read N real rows and write every
     # one of the R slots (padding zeroed); spatial bf16 heads are read in place (no copy)
-    perm = 3.0 * (n_t * 2 * N + n_c * (N + R)) * row
-    unperm = (n_t + n_c) * 2.0 * N * row
+    n_tc = 0 if pipe.in_kernel else n_t  # temporal heads copied (not gathered in the kernel)
+    perm = 3.0 * (n_tc * 2 * N + n_c * (N + R)) * row
+    unperm = (n_tc + n_c) * 2.0 * N * row
     nwords = -(-pipe.nblk // 32)
     mask = BH * pipe.nblk * (nwords + pipe.max_kv + 1) * 4.0
     if wl.mode == "cube":
@@ -122,7 +123,7 @@ def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
     out = {}
     for name, w in work.items():
         t = stage_ms[name] / 1e3
-        if t <= 0:
+        if t <= 0 or w.get("bytes", 1) == 0:
             continue
         if w["bound"] == "hbm":
             gbs = w["bytes"] / t / 1e9
@@ -236,10 +237,11 @@ class ClockSampler:
 class Pipeline:
     """Buffers for the stage-by-stage path through the public entry points."""
 
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, in_kernel=False):
         import block_sparse_attention_31_b200 as vsa
         from block_sparse_attention_31_b200 import _lib
         self.vsa, self.lib, self.wl, self.dev = vsa, _lib, wl, device
+        self.in_kernel = bool(in_kernel) and wl.mode != "cube"  # cube heads always use their copies
         cube = wl.cube if wl.mode == "cube" else None
         self.shape = _lib.make_shape(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, cube)
         if wl.mode == "profiled":
@@ -272,7 +274,12 @@ class Pipeline:
         # work order for cube heads, as the whole call builds it
         self.order = (torch.empty(wl.B * wl.H * self.nblk, dtype=torch.int32, device=device)
                       if wl.mode == "cube" else None)
-        self.launches = ((3 if wl.mode == "profiled" else 0) + 3 + (4 if wl.mode == "cube" else 1) + 1 + 1)
+        cube = wl.mode == "cube"
+        self.launches = ((4 if wl.mode == "profiled" else 0)                 # prep, attn3, row error, reduce
+                         + (0 if self.in_kernel else 6 if cube else 3)        # permutes
+                         + (5 if cube else 1)                                 # masks (+ pool, score, top-k, order)
+                         + 1                                                  # attention
+                         + (0 if self.in_kernel else 2 if cube else 1))       # unpermute
 
     def step(self, q, k, v, o, ev=None):
         L, s = self.lib, None
@@ -283,8 +290,9 @@ class Pipeline:
                                 self.err, s)
         if ev is not None:
             ev[1].record()
-        for src, dst in ((q, self.qp), (k, self.kp), (v, self.vp)):
-            L.vsa_permute(src, L.VSA_BF16, dst, self.kinds, self.shape, self.err, s)
+        if not self.in_kernel:
+            for src, dst in ((q, self.qp), (k, self.kp), (v, self.vp)):
+                L.vsa_permute(src, L.VSA_BF16, dst, self.kinds, self.shape, self.err, s)
         if ev is not None:
             ev[2].record()
         L.vsa_build_mask(self.kinds, self.qp, self.kp, self.shape, self.params, self.bits, self.kv_idx, self.kv_cnt,
@@ -293,11 +301,16 @@ class Pipeline:
             L.vsa_block_order(self.kinds, self.kv_idx, self.kv_cnt, self.max_kv, self.shape, self.order, s)
         if ev is not None:
             ev[3].record()
-        L.vsa_sparse_attn_fwd(L.qkvo(q, k, v, o), L.qkvo(self.qp, self.kp, self.vp, self.op), self.kinds,
-                              self.kv_idx, self.kv_cnt, self.max_kv, self.shape, 0.0, self.err, s, order=self.order)
+        if self.in_kernel:  # temporal heads gathered through the frame-major map inside the kernel
+            L.vsa_sparse_attn_fwd_natural(L.qkvo(q, k, v, o), self.kinds, self.kv_idx, self.kv_cnt, self.max_kv,
+                                          self.shape, 0.0, self.err, s)
+        else:
+            L.vsa_sparse_attn_fwd(L.qkvo(q, k, v, o), L.qkvo(self.qp, self.kp, self.vp, self.op), self.kinds,
+                                  self.kv_idx, self.kv_cnt, self.max_kv, self.shape, 0.0, self.err, s, order=self.order)
         if ev is not None:
             ev[4].record()
-        L.vsa_unpermute(self.op, None, o, L.VSA_BF16, None, self.kinds, self.shape, self.err, s)
+        if not self.in_kernel:
+            L.vsa_unpermute(self.op, None, o, L.VSA_BF16, None, self.kinds, self.shape, self.err, s)
         if ev is not None:
             ev[5].record()
 
@@ -329,7 +342,7 @@ def gpu_arm(args, wl, rank, world, device):
     q, k, v = synthetic.make_qkv(wl, seed=rank_seed(wl.seed, rank))
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     o = torch.empty_like(qd)
-    pipe = Pipeline(wl, device)
+    pipe = Pipeline(wl, device, in_kernel=args.layout == "kernel")
     for _ in range(args.warmup):
         pipe.step(qd, kd, vd, o)
     torch.cuda.synchronize()
@@ -376,7 +389,7 @@ def gpu_arm(args, wl, rank, world, device):
 def e2e_arm(args, wl, q, k, v, device):
     import block_sparse_attention_31_b200 as vsa
     select = {"profiled": "profile", "fixed": "given", "cube": "cube"}[wl.mode]
-    kw = dict(select=select, dtype=q.dtype, device=device)
+    kw = dict(select=select, dtype=q.dtype, device=device, layout_in_kernel=args.layout == "kernel")
     if wl.mode == "profiled":
         kw.update(target=wl.target, profile_frac=wl.profile_frac)
     elif wl.mode == "cube":
@@ -487,6 +500,9 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", default="copies", choices=["copies", "kernel"],
+                    help="temporal heads: permuted into copies (faster at these sizes), or gathered inside "
+                         "the attention kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = synthetic.WORKLOADS[args.config]
@@ -523,6 +539,8 @@ def main():
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.F, wl.Hl, wl.Wl], "d": wl.d,
                    "block": wl.block, "mode": wl.mode, "w_s": res["w_s"], "w_t": res["w_t"],
                    "kept_block_fraction": res["kept"], "head_kinds": res["kinds"],
+                   "layout": ("temporal heads gathered in the attention kernel"
+                              if args.layout == "kernel" and wl.mode != "cube" else "permuted copies"),
                    "l2": "inputs larger than L2 (Q,K,V = %.0f MB > 126 MB); no flush" %
                          (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6)},
         "value_definition": "sparse-actual TFLOP/s of the whole call: algorithmic flops of the kept blocks "

@@ -38,7 +38,7 @@ class Shape(ctypes.Structure):
 
 class Params(ctypes.Structure):
     _fields_ = [("w_s", ctypes.c_int), ("w_t", ctypes.c_int), ("profile_frac", ctypes.c_double),
-                ("topk", ctypes.c_int), ("scale", ctypes.c_float)]
+                ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("layout_in_kernel", ctypes.c_int)]
 
 
 class QKVO(ctypes.Structure):
@@ -71,6 +71,7 @@ def _load():
         "vsa_build_mask": (st, [vp, vp, vp, P(Shape), P(Params), vp, vp, vp, i32, vp, sz, vp, vp]),
         "vsa_block_order": (st, [vp, vp, vp, i32, P(Shape), vp, vp]),
         "vsa_sparse_attn_fwd": (st, [P(QKVO), P(QKVO), vp, vp, vp, i32, vp, P(Shape), ctypes.c_float, vp, vp]),
+        "vsa_sparse_attn_fwd_natural": (st, [P(QKVO), vp, vp, vp, i32, vp, P(Shape), ctypes.c_float, vp, vp]),
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
@@ -123,8 +124,8 @@ def make_shape(B, H, F, Hl, Wl, d, block, cube=None) -> Shape:
     return Shape(B, H, F, Hl, Wl, d, block, cf, ch, cw)
 
 
-def make_params(w_s=0, w_t=0, profile_frac=0.01, topk=0, scale=0.0) -> Params:
-    return Params(int(w_s), int(w_t), float(profile_frac), int(topk), float(scale))
+def make_params(w_s=0, w_t=0, profile_frac=0.01, topk=0, scale=0.0, layout_in_kernel=False) -> Params:
+    return Params(int(w_s), int(w_t), float(profile_frac), int(topk), float(scale), int(bool(layout_in_kernel)))
 
 
 # ---------------------------------------------------------------------------------------
@@ -234,6 +235,13 @@ def vsa_sparse_attn_fwd(natural: QKVO, permuted, kinds, kv_idx, kv_cnt, max_kv, 
                                    _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt), int(max_kv), _ptr(order),
                                    ctypes.byref(shape), float(scale), _ptr(err), _stream(stream)),
            "vsa_sparse_attn_fwd")
+
+
+def vsa_sparse_attn_fwd_natural(natural: QKVO, kinds, kv_idx, kv_cnt, max_kv, shape: Shape, scale, err, stream=None,
+                                order=None):
+    _check(lib.vsa_sparse_attn_fwd_natural(ctypes.byref(natural), _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt),
+                                           int(max_kv), _ptr(order), ctypes.byref(shape), float(scale), _ptr(err),
+                                           _stream(stream)), "vsa_sparse_attn_fwd_natural")
 
 
 def vsa_attention(io: QKVO, dtype: int, shape: Shape, params: Params, select: int, kinds, mse, ws, ws_bytes, err,

@@ -410,7 +410,49 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   a.g = g;
   a.nat_rows = nat_rows;
   a.ucap = std::min(g.nblk, 2 * max_kv);
+  a.gather = 0;
+  a.nat_q = a.nat_k = a.nat_v = nullptr;
+  a.nat_o = nullptr;
   const cudaError_t e = launch_sparse_attn(nat, perm, a, shape->d, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+vsa_status vsa_sparse_attn_fwd_natural(const vsa_qkvo* natural, const uint8_t* d_kind, const int32_t* d_kv_idx,
+                                       const int32_t* d_kv_cnt, int max_kv, const int32_t* d_order,
+                                       const vsa_shape* shape, float scale, int* d_err, cudaStream_t stream) {
+  Geom g;
+  vsa_status st = make_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (g.ncubes > 0) return VSA_ERR_UNSUPPORTED;  // cube heads read cube-major copies
+  if ((st = check_qkvo(natural)) != VSA_OK) return st;
+  if (!d_kind || !d_kv_idx || !d_kv_cnt || !d_err || max_kv <= 0 || !(scale >= 0.f)) return VSA_ERR_INVALID_ARG;
+  const int BH = shape->B * shape->H;
+  if (!on_device({natural->q, natural->k, natural->v, natural->o, natural->lse, d_kind, d_kv_idx, d_kv_cnt, d_order,
+                  d_err}))
+    return VSA_ERR_INVALID_ARG;
+  AttnMaps nat;
+  if ((st = encode_set(&nat, natural, g, g.N, BH, shape->d)) != VSA_OK) return st;
+  AttnArgs a;
+  a.kinds = d_kind;
+  a.kv_idx = d_kv_idx;
+  a.kv_cnt = d_kv_cnt;
+  a.order = d_order;
+  a.lse_nat = natural->lse;
+  a.lse_perm = natural->lse;
+  a.err = d_err;
+  a.BH = BH;
+  a.max_kv = max_kv;
+  a.has_perm = 0;
+  a.scale_log2 = scale_log2_of(scale, shape->d);
+  a.g = g;
+  a.nat_rows = g.N;
+  a.ucap = std::min(g.nblk, 2 * max_kv);
+  a.gather = 1;
+  a.nat_q = natural->q;
+  a.nat_k = natural->k;
+  a.nat_v = natural->v;
+  a.nat_o = natural->o;
+  const cudaError_t e = launch_sparse_attn(nat, nat, a, shape->d, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -446,7 +488,8 @@ static vsa_status attention_layout(const vsa_shape* shape, const vsa_params* par
   off = align256(off + BH * g.nblk * 4);
   L->off_order = off;
   if (g.ncubes > 0) off = align256(off + BH * g.nblk * 4);
-  const size_t tbytes = BH * g.R * d * 2;
+  const bool fused = params->layout_in_kernel != 0 && dtype == VSA_BF16 && g.ncubes == 0;
+  const size_t tbytes = fused ? 0 : BH * g.R * d * 2;  // permuted copies (none when fused)
   L->off_q = off;
   off = align256(off + tbytes);
   L->off_k = off;
@@ -456,7 +499,7 @@ static vsa_status attention_layout(const vsa_shape* shape, const vsa_params* par
   L->off_o = off;
   off = align256(off + tbytes);
   L->off_lse = off;
-  off = align256(off + BH * g.R * 4);
+  off = align256(off + (fused ? BH * 2 * 4 : BH * g.R * 4));  // fused: only the profiling MSE scratch
   L->off_prof = off;
   if (select == VSA_SELECT_PROFILE) off = align256(off + vsa_profile_workspace_size(shape, params));
   L->off_mask = off;
@@ -515,6 +558,15 @@ vsa_status vsa_attention(const vsa_qkvo* io, vsa_dtype dtype, const vsa_shape* s
       return st;
   } else if (select == VSA_SELECT_CUBE) {
     if (cudaMemsetAsync(d_kind, kCube, BH, stream) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  // In-kernel layout: no permuted copies for pattern heads; the attention gathers them.
+  const bool fused = params->layout_in_kernel != 0 && dtype == VSA_BF16 && g.ncubes == 0;
+  if (fused) {
+    if ((st = vsa_build_mask(d_kind, nullptr, nullptr, shape, params, bits, kv_idx, kv_cnt, L.max_kv, nullptr, 0,
+                             d_err, stream)) != VSA_OK)
+      return st;
+    return vsa_sparse_attn_fwd_natural(io, d_kind, kv_idx, kv_cnt, L.max_kv, nullptr, shape, params->scale, d_err,
+                                       stream);
   }
   // 2. layouts
   const vsa_dtype src_t = dtype;

@@ -34,7 +34,8 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1
+// warp 0 TMA (or Q and K gather), warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1, warp 10 V gather
+constexpr int kAttnThreads = 352;
 constexpr int kBM = 128;           // MMA M: query rows per tile
 
 template <int D, int BN>
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int bh = blockIdx.x / npairs;
   const int pair = blockIdx.x - bh * npairs;
   const int kind = a.kinds[bh];
-  if (kind > kCube) {
+  if (kind > kCube || (a.gather && kind == kCube)) {  // in-kernel layout: cube heads need their copies
     if (tid == 0 && pair == 0) atomicOr(a.err, kDevErrKind);
     return;
   }
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
   const bool use_perm = a.has_perm && kind != kSpatial;
+  const bool gather = a.gather && kind == kTemporal;  // rows through the frame-major map, in-kernel
   const CUtensorMap* tq = use_perm ? &tq_p : &tq_n;
   const CUtensorMap* tk = use_perm ? &tk_p : &tk_n;
   const CUtensorMap* tv = use_perm ? &tv_p : &tv_n;
@@ -236,15 +238,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ---- setup: barriers and TMEM ----
   if (tid == 0) {
+    const uint32_t nload = gather ? 32u : 1u;  // gather: one cp.async arrival per producer lane
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(B_Q + t), 1);
+      mbar_init(bar(B_Q + t), nload);
       mbar_init(bar(B_S_FULL + t), 1);
       mbar_init(bar(B_P_FULL + t), 128);
       mbar_init(bar(B_O_FINAL + t), 1);
     }
     for (int st = 0; st < C::NS; ++st) {
-      mbar_init(bar(B_FULL_K + st), 1);
-      mbar_init(bar(B_FULL_V + st), 1);
+      mbar_init(bar(B_FULL_K + st), nload);
+      mbar_init(bar(B_FULL_V + st), nload);
       mbar_init(bar(B_EMPTY_K + st), 1);
       mbar_init(bar(B_EMPTY_V + st), 1);
     }
@@ -266,7 +269,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int U = misc[2];
 
-  if (warp == 0) {
+  if ((warp == 0 || warp == 10) && gather) {
+    // ================= gather producers (temporal head, natural-order buffers) =================
+    // Warp 0 copies the Q and K tiles, warp 10 the V tiles, 16 bytes per copy: slot p of the
+    // frame-major layout is token (p % F) * S + p / F; copies land in the 128-byte-swizzled
+    // layout a TMA tile load would produce, slots past N are zero-filled.  Each lane's copies
+    // signal the stage's barrier when they land.  Lane l owns 16-byte column c = l % CPR of rows
+    // r = l / CPR + k * RSTEP, and walks them with incremental (frame, position) and source
+    // offsets, so no division runs per copy.
+    if (U > 0) {
+      constexpr int CPR = D / 8, RSTEP = 32 / CPR;
+      const int c = lane % CPR, r0 = lane / CPR;
+      const size_t head = static_cast<size_t>(bh) * g.N * D;
+      const size_t fstep = static_cast<size_t>(RSTEP) * g.S * D;  // RSTEP frames further
+      const size_t wrap = static_cast<size_t>(g.F) * g.S * D - D;  // frame F -> frame 0, next position
+      auto gather_tile = [&](uint32_t sdst, int rows_tile, int slot0, const __nv_bfloat16* src) {
+        const uint32_t panel = sdst + (c >> 3) * (rows_tile * 128);
+        int slot = slot0 + r0;
+        const int sp = slot / g.F;
+        int f = slot - sp * g.F;
+        const __nv_bfloat16* from = src + (static_cast<size_t>(f) * g.S + sp) * D + c * 8;
+#pragma unroll 4
+        for (int r = r0; r < rows_tile; r += RSTEP) {
+          const bool in = slot < g.N;
+          cp_async_16(panel + r * 128 + (((c & 7) ^ (r & 7)) << 4), in ? from : src, in ? 16u : 0u);
+          slot += RSTEP;
+          f += RSTEP;
+          from += fstep;
+          while (f >= g.F) {
+            f -= g.F;
+            from -= wrap;
+          }
+        }
+      };
+      const __nv_bfloat16* gq = static_cast<const __nv_bfloat16*>(a.nat_q) + head;
+      const __nv_bfloat16* gk = static_cast<const __nv_bfloat16*>(a.nat_k) + head;
+      const __nv_bfloat16* gv = static_cast<const __nv_bfloat16*>(a.nat_v) + head;
+      const int cnts[2] = {cnt0, cnt1};
+      if (warp == 0) {
+        for (int t = 0; t < 2; ++t) {
+          if (cnts[t] == 0) continue;
+          gather_tile(sbase + C::OFF_Q + t * C::Q_BYTES, kBM, (t ? qb1 : qb0) * BN, gq);
+          cp_async_mbar_arrive_noinc(bar(B_Q + t));
+        }
+      }
+      const int eb = warp == 0 ? B_EMPTY_K : B_EMPTY_V, fb = warp == 0 ? B_FULL_K : B_FULL_V;
+      const uint32_t sdst0 = warp == 0 ? sK : sV;
+      const __nv_bfloat16* gsrc = warp == 0 ? gk : gv;
+      for (int n = 0; n < U; ++n) {
+        const int st = n % C::NS;
+        const uint32_t u = n / C::NS;
+        const int kb = static_cast<int>(uni[n] & kKbMask);
+        if (n >= C::NS && !__all_sync(0xffffffffu, mbar_wait(bar(eb + st), (u - 1) & 1, abort_flag, a.err))) break;
+        gather_tile(sdst0 + st * C::KV_BYTES, BN, kb * BN, gsrc);
+        cp_async_mbar_arrive_noinc(bar(fb + st));
+      }
+      // every copy lands before the CTA can exit (they always complete; nothing to bound)
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0 && U > 0) {
       int nk = 0, nv = 0;  // copies issued
@@ -329,6 +391,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int np = pend[t];
         if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
         if (!mbar_wait(bar(B_FULL_V + np % C::NS), (np / C::NS) & 1, abort_flag, a.err)) return false;
+        if (gather) fence_proxy_async_smem();  // cp.async data, written by the generic proxy
         tc_fence_after();
         const uint64_t vd = (np & 1) ? dv1 : dv0;
         const uint32_t d_o = tmem + C::TMEM_O + t * D, a_p = tmem + C::TMEM_S + t * BN;
@@ -361,6 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             qready[t] = true;
           }
+          if (gather) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t d_s = tmem + C::TMEM_S + t * BN;
           const uint64_t qd = t ? dq1 : dq0, kd = st ? dk1 : dk0;
@@ -383,7 +447,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait_drain(bar(B_DRAIN), 0, a.err);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 10) {
     // ================= softmax: warps 2-5 tile 0, warps 6-9 tile 1; one row per thread =================
     const int t = (warp - 2) >> 2;
     const int quad = warp & 3;          // TMEM lane quadrant this warp may access
@@ -505,6 +569,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool have = ok && cnt > 0 && l > 0.f;
       const float inv = have ? 1.f / l : 0.f;
       uint8_t* stage = smem + C::OFF_Q + t * C::Q_BYTES;
+      // in-kernel layout: this row's natural token (slot p -> (p % F) * S + p / F)
+      const int slot = qb * BN + row;
+      const bool row_live = row < BN && slot < rows;
+      const int tok = gather ? (slot % g.F) * g.S + slot / g.F : slot;
+      __nv_bfloat16* orow = gather ? static_cast<__nv_bfloat16*>(a.nat_o) + (static_cast<size_t>(bh) * g.N + tok) * D
+                                   : nullptr;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
@@ -523,22 +593,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             v4.z = pack_bf16x2(o[q4 * 8 + 4] * inv, o[q4 * 8 + 5] * inv);
             v4.w = pack_bf16x2(o[q4 * 8 + 6] * inv, o[q4 * 8 + 7] * inv);
             const int col = c * 32 + q4 * 8;
-            const int dc = col >> 6, cc = (col & 63) >> 3;
-            *reinterpret_cast<uint4*>(stage + dc * (BN * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v4;
+            if (gather) {
+              if (row_live) *reinterpret_cast<uint4*>(orow + col) = v4;
+            } else {
+              const int dc = col >> 6, cc = (col & 63) >> 3;
+              *reinterpret_cast<uint4*>(stage + dc * (BN * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v4;
+            }
           }
         }
       }
-      fence_proxy_async_smem();
-      named_barrier_sync(1 + t, 128);
-      if (quad == 2 && lane == 0) {
-        const uint32_t sstage = sbase + C::OFF_Q + t * C::Q_BYTES;
+      if (!gather) {
+        fence_proxy_async_smem();
+        named_barrier_sync(1 + t, 128);
+        if (quad == 2 && lane == 0) {
+          const uint32_t sstage = sbase + C::OFF_Q + t * C::Q_BYTES;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_store_3d(to, sstage + c * BN * 128, c * 64, qb * BN, bh);
-        tma_store_commit();
-        tma_store_wait_all();
+          for (int c = 0; c < D / 64; ++c) tma_store_3d(to, sstage + c * BN * 128, c * 64, qb * BN, bh);
+          tma_store_commit();
+          tma_store_wait_all();
+        }
       }
-      if (lse != nullptr && row < BN && qb * BN + row < rows)
-        lse[static_cast<size_t>(bh) * lse_stride + qb * BN + row] =
+      if (lse != nullptr && row_live)
+        lse[static_cast<size_t>(bh) * lse_stride + tok] =
             have ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }

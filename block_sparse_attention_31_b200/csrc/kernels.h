@@ -46,6 +46,13 @@ struct AttnArgs {
   int ucap;      // capacity of the per-CTA union list: min(nblk, 2 * max_kv)
   float scale_log2;
   Geom g;
+  // In-kernel layout: temporal heads read Q, K, V and write O in natural order through the
+  // frame-major slot map (no permuted copies); only with has_perm == 0.
+  int gather;
+  const void* nat_q;
+  const void* nat_k;
+  const void* nat_v;
+  void* nat_o;
 };
 
 cudaError_t launch_sparse_attn(const AttnMaps& nat, const AttnMaps& perm, const AttnArgs& a, int d,

@@ -101,6 +101,10 @@ typedef struct {
     double profile_frac;          /* profiled share of query rows: r = ceil(frac*N) */
     int topk;                     /* long-range cubes per query cube (cube heads) */
     float scale;                  /* softmax scale; 0 selects 1/sqrt(d) */
+    int layout_in_kernel;         /* vsa_attention only: 1 = temporal heads are read and written
+                                     in natural order through the frame-major map inside the
+                                     attention kernel (no permute / unpermute copies); used
+                                     for bf16 inputs without cube dims, ignored otherwise */
 } vsa_params;
 
 /* Pointers of one attention problem; o and lse are written. lse may be NULL. */
@@ -256,6 +260,21 @@ VSA_API vsa_status vsa_sparse_attn_fwd(const vsa_qkvo *natural, const vsa_qkvo *
                                const int32_t *d_kv_idx, const int32_t *d_kv_cnt, int max_kv,
                                const int32_t *d_order, const vsa_shape *shape, float scale, int *d_err,
                                cudaStream_t stream);
+
+/*
+ * vsa_sparse_attn_fwd with every head in natural order ("Sparse Video-Gen" summary page,
+ * "Approach": the frame-major layout of temporal heads, applied inside the kernel): temporal
+ * heads gather their Q, K, V rows through the frame-major slot map (slot p = s*F + f is token
+ * f*S + s) while loading tiles, and write O and LSE rows back to their natural tokens, so no
+ * permuted copies exist.  Spatial heads are as in vsa_sparse_attn_fwd.
+ *   natural   q, k, v, o, lse ([B, H, N, d] bf16, natural order; lse may be NULL)
+ *   the rest  as vsa_sparse_attn_fwd; masks of temporal heads are over frame-major blocks
+ * Shapes with cube dims return VSA_ERR_UNSUPPORTED; a cube kind byte sets VSA_DEVERR_KIND.
+ */
+VSA_API vsa_status vsa_sparse_attn_fwd_natural(const vsa_qkvo *natural, const uint8_t *d_kind,
+                                               const int32_t *d_kv_idx, const int32_t *d_kv_cnt, int max_kv,
+                                               const int32_t *d_order, const vsa_shape *shape, float scale,
+                                               int *d_err, cudaStream_t stream);
 
 /*
  * The whole call: kinds (profiled, given or cube) -> permute -> masks -> sparse attention

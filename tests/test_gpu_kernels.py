@@ -412,3 +412,69 @@ def test_profile_matches_oracle(wl, w_s, w_t, frac):
         big = int(np.argmax(want))
         assert mse[h, big] == pytest.approx(want[big], rel=2e-2)
         assert mse[h, 1 - big] <= want[1 - big] + 1e-4
+
+
+# ------------------------------------------------------------------------------------
+# in-kernel layout: temporal heads gathered through the frame-major map
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("F,Hl,Wl,d,block,w_t", [(6, 8, 16, 128, 128, 9), (5, 6, 10, 128, 128, 7),
+                                                 (7, 5, 9, 64, 64, 11), (21, 30, 52, 128, 128, 140)])
+def test_attention_natural_layout_matches_permuted(F, Hl, Wl, d, block, w_t):
+    """vsa_sparse_attn_fwd_natural (rows gathered in-kernel, ragged tails zero-filled) gives the
+    permute -> attention -> unpermute result bit for bit, and matches the oracle."""
+    wl = synthetic.Workload("nat", 1, 2, F, Hl, Wl, d, block, "bf16", "given")
+    q, k, v = synthetic.make_qkv(wl)
+    kinds_list = [S_, T_]
+    keeps = [keep_for_head(S_, wl, 1, 0), keep_for_head(T_, wl, 0, w_t)]
+    shape = _lib.make_shape(1, 2, F, Hl, Wl, d, block)
+    nblk = _lib.vsa_num_blocks(shape)
+    max_kv = max(int(kp.sum(axis=1).max()) for kp in keeps)
+    idx = np.full((1, 2, nblk, max_kv), -1, dtype=np.int32)
+    cnt = np.zeros((1, 2, nblk), dtype=np.int32)
+    for h, kp in enumerate(keeps):
+        i_, c_ = oracle.keep_to_lists(kp, max_kv)
+        idx[0, h, :kp.shape[0]] = i_
+        cnt[0, h, :kp.shape[0]] = c_
+    idx_d, cnt_d = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    kinds = torch.tensor(kinds_list, dtype=torch.uint8, device="cuda")
+    err = cuda_err()
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    # permuted path
+    o_p = torch.full_like(qd, 9.0)
+    lse_p = torch.full((1, 2, wl.N), 9.0, dtype=torch.float32, device="cuda")
+    qp, kp_, vp, op = (torch.empty_like(qd) for _ in range(4))
+    lsep = torch.empty(1, 2, wl.N, dtype=torch.float32, device="cuda")
+    for src, dst in ((qd, qp), (kd, kp_), (vd, vp)):
+        _lib.vsa_permute(src, _lib.VSA_BF16, dst, kinds, shape, err)
+    _lib.vsa_sparse_attn_fwd(_lib.qkvo(qd, kd, vd, o_p, lse_p), _lib.qkvo(qp, kp_, vp, op, lsep), kinds, idx_d,
+                             cnt_d, max_kv, shape, 0.0, err)
+    _lib.vsa_unpermute(op, lsep, o_p, _lib.VSA_BF16, lse_p, kinds, shape, err)
+    # in-kernel layout
+    o_n = torch.full_like(qd, 9.0)
+    lse_n = torch.full((1, 2, wl.N), 9.0, dtype=torch.float32, device="cuda")
+    _lib.vsa_sparse_attn_fwd_natural(_lib.qkvo(qd, kd, vd, o_n, lse_n), kinds, idx_d, cnt_d, max_kv, shape, 0.0, err)
+    assert _lib.vsa_get_device_error(err) == 0
+    assert torch.equal(o_n, o_p) and torch.equal(lse_n, lse_p)
+    o_n = o_n.cpu()
+    for h, kind in enumerate(kinds_list):
+        want, _ = oracle.attention_rows(q[0, h], k[0, h], v[0, h], head_slots(kind, wl), wl.block, keeps[h],
+                                        rows=np.arange(wl.N), scale=1.0 / math.sqrt(wl.d))
+        assert_close_attention(to_f64(o_n[0, h]), want, f"head {h}")
+
+
+def test_attention_natural_layout_rejects_cubes():
+    shape = _lib.make_shape(1, 1, 8, 8, 8, 128, 128, (4, 4, 8))
+    q = torch.zeros(1, 1, 512, 128, dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros(1, 1, 4, 1, dtype=torch.int32, device="cuda")
+    cnt = torch.ones(1, 1, 4, dtype=torch.int32, device="cuda")
+    kinds = torch.full((1,), 2, dtype=torch.uint8, device="cuda")
+    with pytest.raises(_lib.VsaError) as ex:
+        _lib.vsa_sparse_attn_fwd_natural(_lib.qkvo(q, q, q, q), kinds, idx, cnt, 1, shape, 0.0, cuda_err())
+    assert ex.value.status == _lib.VSA_ERR_UNSUPPORTED
+    # a cube kind byte on a shape without cubes is flagged on the device
+    shape = _lib.make_shape(1, 1, 8, 8, 8, 128, 128)
+    err = cuda_err()
+    o = torch.empty_like(q)
+    _lib.vsa_sparse_attn_fwd_natural(_lib.qkvo(q, q, q, o), kinds, idx, cnt, 1, shape, 0.0, err)
+    assert _lib.vsa_get_device_error(err) & _lib.VSA_DEVERR_KIND

@@ -129,3 +129,22 @@ def test_run_host_overlapped_matches_single_calls():
         want = plan(q.cuda(), k.cuda(), v.cuda())
         want = want[0] if isinstance(want, tuple) else want
         assert torch.equal(got, want.cpu())
+
+
+@pytest.mark.parametrize("wl", [
+    synthetic.Workload("small profiled", 1, 4, 8, 12, 20, 128, 128, "bf16", "profiled", target=0.3, profile_frac=0.05),
+    synthetic.WAN])
+def test_layout_in_kernel_same_result(wl):
+    """The whole call with temporal heads gathered in-kernel equals the call with permuted
+    copies bit for bit (same kinds, masks, outputs and LSE)."""
+    q, k, v = (t.cuda() for t in synthetic.make_qkv(wl))
+    outs = []
+    for fused in (False, True):
+        plan = vsa.SparseAttention(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, select="profile", target=wl.target,
+                                   profile_frac=wl.profile_frac, with_lse=True, layout_in_kernel=fused)
+        o, lse = plan(q, k, v)
+        assert plan.device_error() == 0
+        outs.append((o, lse, plan.kinds.clone(), plan.kv_idx.clone()))
+    (o0, l0, k0, i0), (o1, l1, k1, i1) = outs
+    assert torch.equal(k0, k1) and torch.equal(i0, i1)
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
