@@ -34,8 +34,9 @@
 
 namespace vsa {
 
-// warp 0 TMA (or Q and K gather), warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1, warp 10 V gather
-constexpr int kAttnThreads = 352;
+// warp 0 TMA (or Q and K gather), warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1, and for the
+// in-kernel layout warp 10 (V gather)
+constexpr int kAttnThreads = 320, kAttnThreadsGather = 352;
 constexpr int kBM = 128;           // MMA M: query rows per tile
 
 template <int D, int BN>
@@ -83,7 +84,7 @@ constexpr int kPolyPairs8 = VSA_POLY_PAIRS8;
 // tile) so the tensor core works on one tile while the other tile's softmax runs.  P is
 // written as packed bf16 over the tile's S columns in TMEM and read from there by the P.V MMA.
 template <int D, int BN>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreadsGather, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tq_n, const __grid_constant__ CUtensorMap tk_n,
                            const __grid_constant__ CUtensorMap tv_n, const __grid_constant__ CUtensorMap to_n,
                            const __grid_constant__ CUtensorMap tq_p, const __grid_constant__ CUtensorMap tk_p,
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* bits1 = bits0 + nwords;
   uint32_t* uvalid = bits1 + nwords;  // [ucap][BN/32] valid-key bits of partial union entries
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
   const Geom& g = a.g;
   const int npairs = (g.nblk + 1) >> 1;
   const int bh = blockIdx.x / npairs;
@@ -146,19 +147,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   int cnt0 = a.kv_cnt[mrow0];
   int cnt1 = has1 ? a.kv_cnt[mrow1] : 0;
   bool bad0 = cnt0 < 0 || cnt0 > a.max_kv, bad1 = cnt1 < 0 || cnt1 > a.max_kv;
-  for (int x = tid; x < 2 * nwords; x += kAttnThreads) bits0[x] = 0u;  // bits1 follows bits0
+  for (int x = tid; x < 2 * nwords; x += nthr) bits0[x] = 0u;  // bits1 follows bits0
   bool stop = false;
   if (tid == 0) stop = (*reinterpret_cast<volatile int*>(a.err) & kDevErrTimeout) != 0;
   if (__syncthreads_or(stop)) return;
   // Lists must be strictly ascending block indices in [0, nb_head).
   if (!bad0)
-    for (int j = tid; j < cnt0; j += kAttnThreads) {
+    for (int j = tid; j < cnt0; j += nthr) {
       const int kb = kvl0[j];
       if (kb < 0 || kb >= nb_head || (j > 0 && kvl0[j - 1] >= kb)) bad0 = true;
       else atomicOr(&bits0[kb >> 5], 1u << (kb & 31));
     }
   if (!bad1)
-    for (int j = tid; j < cnt1; j += kAttnThreads) {
+    for (int j = tid; j < cnt1; j += nthr) {
       const int kb = kvl1[j];
       if (kb < 0 || kb >= nb_head || (j > 0 && kvl1[j - 1] >= kb)) bad1 = true;
       else atomicOr(&bits1[kb >> 5], 1u << (kb & 31));
@@ -169,11 +170,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (tid == 0) atomicOr(a.err, kDevErrKvRange);
     if (bad0) {
       cnt0 = 0;
-      for (int x = tid; x < nwords; x += kAttnThreads) bits0[x] = 0u;
+      for (int x = tid; x < nwords; x += nthr) bits0[x] = 0u;
     }
     if (bad1) {
       cnt1 = 0;
-      for (int x = tid; x < nwords; x += kAttnThreads) bits1[x] = 0u;
+      for (int x = tid; x < nwords; x += nthr) bits1[x] = 0u;
     }
     __syncthreads();
   }
@@ -636,7 +637,7 @@ static cudaError_t launch_attn_t(const AttnMaps& nat, const AttnMaps& perm, cons
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(a.BH) * ((a.g.nblk + 1) / 2);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
+  kern<<<static_cast<unsigned>(grid), a.gather ? kAttnThreadsGather : kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
                                                                      perm.v, perm.o, a);
   return cudaGetLastError();
 }
