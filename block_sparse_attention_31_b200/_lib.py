@@ -76,6 +76,7 @@ def _load():
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
         "vsa_selftest_exp2": (st, [vp, vp, vp, i32, vp]),
+        "vsa_selftest_wait_timeout": (st, [vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -262,3 +263,7 @@ def vsa_get_device_error(err, stream=None) -> int:
 def vsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
     _check(lib.vsa_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), int(x.numel()), _stream(stream)),
            "vsa_selftest_exp2")
+
+
+def vsa_selftest_wait_timeout(err, waited, stream=None):
+    _check(lib.vsa_selftest_wait_timeout(_ptr(err), _ptr(waited), _stream(stream)), "vsa_selftest_wait_timeout")

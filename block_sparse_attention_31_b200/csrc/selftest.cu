@@ -23,7 +23,28 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
   }
 }
 
+// One thread waits, with the bounded wait every kernel uses, on an mbarrier that expects one
+// arrival which never comes: after the wait limit it must give up, raise the timeout bit of
+// the error word and return.
+__global__ void wait_timeout_selftest_kernel(int* __restrict__ err, int* __restrict__ waited) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    mbar_init_fence();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *waited = mbar_wait(smem_u32(&bar), 0, &abort_flag, err) ? 1 : 0;
+}
+
 }  // namespace vsa
+
+extern "C" vsa_status vsa_selftest_wait_timeout(int* d_err, int* d_waited, cudaStream_t stream) {
+  if (d_err == nullptr || d_waited == nullptr) return VSA_ERR_INVALID_ARG;
+  vsa::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(d_err, d_waited);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
 
 extern "C" vsa_status vsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int n, cudaStream_t stream) {
   if (x == nullptr || y_poly == nullptr || y_mufu == nullptr || n < 0) return VSA_ERR_INVALID_ARG;

@@ -298,6 +298,13 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
  * on n device floats, so that tests can bound the polynomial's error. */
 VSA_API vsa_status vsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n, cudaStream_t stream);
 
+/* Self-test hook for failure handling (no counterpart in the pages): one thread runs the
+ * bounded mbarrier wait all kernels use on a barrier that nothing completes.  After the wait
+ * limit (1 s of %globaltimer) it sets VSA_DEVERR_TIMEOUT in *d_err, writes 0 to *d_waited and
+ * returns; vsa_get_device_error then reports VSA_ERR_TIMEOUT and the context stays usable.
+ *   d_err, d_waited  device ints (d_waited: 1 if the wait succeeded, 0 if it gave up) */
+VSA_API vsa_status vsa_selftest_wait_timeout(int *d_err, int *d_waited, cudaStream_t stream);
+
 /* Synchronise `stream`, copy the device error word to *host_err and map it to a status
  * (VSA_OK when zero, VSA_ERR_TIMEOUT when the timeout bit is set, else VSA_ERR_DEVICE). */
 VSA_API vsa_status vsa_get_device_error(const int *d_err, cudaStream_t stream, int *host_err);

@@ -126,6 +126,26 @@ def test_kernel_entry_points_validate_before_launch():
     assert lib.vsa_attention(ctypes.byref(io), 1, ctypes.byref(shape), ctypes.byref(params), 2, FAKE, None, FAKE,
                              1 << 40, FAKE, s) == _lib.VSA_ERR_INVALID_ARG
     assert lib.vsa_get_device_error(None, s, None) == _lib.VSA_ERR_INVALID_ARG
+    # in-kernel layout: cube shapes are refused on the host, missing buffers too
+    cube_shape = _lib.make_shape(1, 2, 8, 8, 8, 64, 128, (4, 4, 8))
+    io = _lib.QKVO(FAKE, FAKE, FAKE, FAKE, None)
+    assert lib.vsa_sparse_attn_fwd_natural(ctypes.byref(io), FAKE, FAKE, FAKE, 4, None, ctypes.byref(cube_shape), 0.0,
+                                           FAKE, s) == _lib.VSA_ERR_UNSUPPORTED
+    io = _lib.QKVO(FAKE, None, FAKE, FAKE, None)
+    assert lib.vsa_sparse_attn_fwd_natural(ctypes.byref(io), FAKE, FAKE, FAKE, 4, None, ctypes.byref(shape), 0.0,
+                                           FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+    assert lib.vsa_selftest_wait_timeout(None, FAKE, s) == _lib.VSA_ERR_INVALID_ARG
+
+
+def test_in_kernel_layout_drops_the_permuted_copies():
+    shape = _lib.make_shape(1, 12, 21, 30, 52, 128, 128)
+    copies = _lib.vsa_attention_workspace_size(shape, _lib.make_params(2, 140), 1, 0)
+    fused = _lib.vsa_attention_workspace_size(shape, _lib.make_params(2, 140, layout_in_kernel=True), 1, 0)
+    per_tensor = 12 * 32760 * 128 * 2
+    assert copies - fused >= 4 * per_tensor          # Q, K, V, O copies
+    # fp32 inputs and cube shapes keep the copies
+    f32_fused = _lib.vsa_attention_workspace_size(shape, _lib.make_params(2, 140, layout_in_kernel=True), 0, 1)
+    assert f32_fused > 0 and f32_fused == _lib.vsa_attention_workspace_size(shape, _lib.make_params(2, 140), 0, 1)
 
 
 def test_workspace_sizes_monotone():
