@@ -58,6 +58,16 @@ def _load():
         lib.or_cube_topk_keep.argtypes = [vp, vp] + [i64] * 8 + [vp, vp]
         lib.or_attention_rows.restype = None
         lib.or_attention_rows.argtypes = [vp, vp, vp, i64, i64, dbl, vp, i64, vp, i64, vp, i64, vp, vp]
+        lib.or_attention_rows_qk.restype = None
+        lib.or_attention_rows_qk.argtypes = [vp, vp, vp, i64, i64, dbl, vp, vp, i64, vp, i64, vp, i64, vp, vp]
+        lib.or_exp_neg.restype = dbl
+        lib.or_exp_neg.argtypes = [dbl]
+        lib.or_kmeans.restype = ctypes.c_int
+        lib.or_kmeans.argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
+        lib.or_cluster_perm.restype = None
+        lib.or_cluster_perm.argtypes = [vp, i64, i64, vp, vp]
+        lib.or_semantic_keep.restype = None
+        lib.or_semantic_keep.argtypes = [vp, vp, i64, vp, vp, i64, i64, dbl, dbl, vp]
         lib.or_profile_rows.restype = i64
         lib.or_profile_rows.argtypes = [i64, dbl]
         lib.or_profile_head.restype = ctypes.c_int
@@ -121,22 +131,25 @@ def cube_topk_keep(q, k, F, Hl, Wl, topk, cube=(4, 4, 8), return_scores=False):
     return (keep.astype(bool), score) if return_scores else keep.astype(bool)
 
 
-def attention_rows(q, k, v, slots, block, keep, rows=None, scale=None):
+def attention_rows(q, k, v, slots, block, keep, rows=None, scale=None, kslots=None):
     """Masked softmax attention on natural-order rows of one head.
 
-    Returns (out [len(rows), d] fp64, lse [len(rows)] fp64, natural log).
+    ``slots`` maps tokens to slots of the queries' layout; ``kslots`` (default: the same)
+    those of the keys' layout.  Returns (out [len(rows), d] fp64, lse [len(rows)] fp64,
+    natural log).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     N, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     slots = np.ascontiguousarray(slots, dtype=np.int64)
+    kslots = slots if kslots is None else np.ascontiguousarray(kslots, dtype=np.int64)
     keep8 = np.ascontiguousarray(keep, dtype=np.uint8)
     nb = keep8.shape[0]
     rows = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     out = np.empty((len(rows), d), dtype=np.float64)
     lse = np.empty(len(rows), dtype=np.float64)
-    _load().or_attention_rows(_p(q), _p(k), _p(v), N, d, scale, _p(slots), block, _p(keep8), nb,
-                              _p(rows), len(rows), _p(out), _p(lse))
+    _load().or_attention_rows_qk(_p(q), _p(k), _p(v), N, d, scale, _p(slots), _p(kslots), block, _p(keep8), nb,
+                                 _p(rows), len(rows), _p(out), _p(lse))
     return out, lse
 
 
@@ -157,6 +170,107 @@ def profile_head(q, k, v, F, Hl, Wl, block, w_s, w_t, frac=0.01, scale=None):
     if kind < 0:
         raise MemoryError("oracle profiling allocation failed")
     return int(kind), mse, rows
+
+
+# ---------------------------------------------------------------------------------------
+# Semantic-aware permutation (Sparse VideoGen2 page, abstract); the readings are stated in
+# vsa_oracle.c next to the C functions.
+# ---------------------------------------------------------------------------------------
+
+def exp_neg(x: float) -> float:
+    """The oracle's own exp for x <= 0 (0 below -700)."""
+    return float(_load().or_exp_neg(float(x)))
+
+
+def _f32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def kmeans(x, C: int, iters: int):
+    """k-means of one head's rows x [N, d]: (centroids [C, d] fp32, labels [N], counts [C])."""
+    x = _f32(x)
+    N, d = x.shape
+    cent = np.empty((C, d), dtype=np.float32)
+    label = np.empty(N, dtype=np.int32)
+    count = np.empty(C, dtype=np.int32)
+    if _load().or_kmeans(_p(x), N, d, C, iters, _p(cent), _p(label), _p(count)) != 0:
+        raise ValueError("oracle k-means: bad arguments or allocation failure")
+    return cent, label, count
+
+
+def cluster_perm(label, C: int):
+    """Cluster-major order: (perm [N] slot -> token, offset [C + 1])."""
+    label = np.ascontiguousarray(label, dtype=np.int32)
+    perm = np.empty(label.size, dtype=np.int32)
+    offset = np.empty(C + 1, dtype=np.int32)
+    _load().or_cluster_perm(_p(label), label.size, C, _p(perm), _p(offset))
+    return perm, offset
+
+
+def semantic_keep(cq, nq, ck, nk, scale: float, top_p: float) -> np.ndarray:
+    """Kept key clusters per query cluster: bool [Cq, Ck]."""
+    cq, ck = _f32(cq), _f32(ck)
+    nq = np.ascontiguousarray(nq, dtype=np.int32)
+    nk = np.ascontiguousarray(nk, dtype=np.int32)
+    Cq, d = cq.shape
+    Ck = ck.shape[0]
+    keep = np.empty((Cq, Ck), dtype=np.uint8)
+    _load().or_semantic_keep(_p(cq), _p(nq), Cq, _p(ck), _p(nk), Ck, d, float(scale), float(top_p), _p(keep))
+    return keep.astype(bool)
+
+
+def semantic_block_keep(label_q, perm_q, label_k, perm_k, keep, block: int) -> np.ndarray:
+    """Block mask [nb, nb] over the two cluster-major layouts: block a of the queries and
+    block b of the keys are kept when a kept cluster pair joins one of a's slots to one of
+    b's slots."""
+    lq = np.asarray(label_q)[np.asarray(perm_q)]        # cluster of each query slot
+    lk = np.asarray(label_k)[np.asarray(perm_k)]
+    N = lq.size
+    nb = -(-N // block)
+    keep = np.asarray(keep, dtype=bool)
+    out = np.zeros((nb, nb), dtype=bool)
+    for a in range(nb):
+        qs = np.unique(lq[a * block:(a + 1) * block])
+        row = keep[qs].any(axis=0)                      # key clusters reached from block a
+        for b in range(nb):
+            out[a, b] = row[np.unique(lk[b * block:(b + 1) * block])].any()
+    return out
+
+
+def semantic_scale(d: int, scale: float = 0.0) -> float:
+    """Softmax scale of the criticality scores: the given one, else 1/sqrt(d) in fp64."""
+    return float(scale) if scale > 0 else 1.0 / math.sqrt(d)
+
+
+def semantic_head(q, k, v, cq: int, ck: int, iters: int, top_p: float, block: int, rows=None, scale: float = 0.0,
+                  attention: bool = True):
+    """The whole semantic path for one head (natural-order q, k, v [N, d]).
+
+    Returns a dict with the k-means results of Q and K, both permutations, the cluster and
+    block masks and, when ``attention``, the output rows (fp64) and their LSE.
+    """
+    d = q.shape[-1]
+    cent_q, lab_q, cnt_q = kmeans(q, cq, iters)
+    cent_k, lab_k, cnt_k = kmeans(k, ck, iters)
+    perm_q, _ = cluster_perm(lab_q, cq)
+    perm_k, _ = cluster_perm(lab_k, ck)
+    sc = semantic_scale(d, scale)
+    keep_c = semantic_keep(cent_q, cnt_q, cent_k, cnt_k, sc, top_p)
+    keep_b = semantic_block_keep(lab_q, perm_q, lab_k, perm_k, keep_c, block)
+    res = dict(cent_q=cent_q, label_q=lab_q, count_q=cnt_q, perm_q=perm_q, cent_k=cent_k, label_k=lab_k,
+               count_k=cnt_k, perm_k=perm_k, keep_clusters=keep_c, keep_blocks=keep_b)
+    if attention:
+        N = lab_q.size
+        qslot = np.empty(N, dtype=np.int64)
+        qslot[perm_q] = np.arange(N)
+        kslot = np.empty(N, dtype=np.int64)
+        kslot[perm_k] = np.arange(N)
+        out, lse = attention_rows(q, k, v, qslot, block, keep_b, rows=rows, kslots=kslot,
+                                  scale=None if scale <= 0 else scale)
+        res.update(out=out, lse=lse)
+    return res
 
 
 # ---------------------------------------------------------------------------------------

@@ -205,18 +205,20 @@ int or_cube_topk_keep(const double *q, const double *k, int64_t F, int64_t Hl, i
 /*
  * Masked softmax attention on selected query rows ([OSP] Method: FlashAttention-compatible
  * sparse attention; [SVG] Approach: block-wise masks).  Everything in natural token order:
- * key u is allowed for query t when keep[block(t) * nblk + block(u)] is set, with
- * block(x) = slot[x] / block.  q, k, v: [N, d] fp64.  out: [nrows, d]; lse: [nrows]
- * (natural log), or NULL.
+ * key u is allowed for query t when keep[qblock(t) * nblk + block(u)] is set, with
+ * qblock(t) = qslot[t] / block under the queries' layout and block(u) = slot[u] / block
+ * under the keys' layout (the same map except for the semantic permutation, which orders
+ * queries and keys by their own clusters).  q, k, v: [N, d] fp64.  out: [nrows, d];
+ * lse: [nrows] (natural log), or NULL.
  */
-void or_attention_rows(const double *q, const double *k, const double *v, int64_t N, int64_t d, double scale,
-                       const int64_t *slot, int64_t block, const uint8_t *keep, int64_t nblk,
-                       const int64_t *rows, int64_t nrows, double *out, double *lse)
+void or_attention_rows_qk(const double *q, const double *k, const double *v, int64_t N, int64_t d, double scale,
+                          const int64_t *qslot, const int64_t *slot, int64_t block, const uint8_t *keep,
+                          int64_t nblk, const int64_t *rows, int64_t nrows, double *out, double *lse)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nrows; ++r) {
         int64_t t = rows[r];
-        int64_t bi = slot[t] / block;
+        int64_t bi = qslot[t] / block;
         const double *qt = q + t * d;
         double *o = out + r * d;
         double m = -INFINITY;
@@ -244,6 +246,14 @@ void or_attention_rows(const double *q, const double *k, const double *v, int64_
         for (int64_t x = 0; x < d; ++x) o[x] /= sum;
         if (lse) lse[r] = m + log(sum);
     }
+}
+
+/* The same with one layout for queries and keys (every head kind of [SVG] and [USV]). */
+void or_attention_rows(const double *q, const double *k, const double *v, int64_t N, int64_t d, double scale,
+                       const int64_t *slot, int64_t block, const uint8_t *keep, int64_t nblk,
+                       const int64_t *rows, int64_t nrows, double *out, double *lse)
+{
+    or_attention_rows_qk(q, k, v, N, d, scale, slot, slot, block, keep, nblk, rows, nrows, out, lse);
 }
 
 /* Number of profiling rows: ceil(frac * N), clamped to [1, N]. */
@@ -296,4 +306,176 @@ int or_profile_head(const double *q, const double *k, const double *v, int64_t F
     free(rows); free(slot_id); free(slot_tp); free(all); free(ks); free(kt);
     free(od); free(osp); free(otp);
     return mse[1] < mse[0] ? OR_TEMPORAL : OR_SPATIAL;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Semantic-aware permutation ([SVG2] "Sparse VideoGen2: ... Semantic-Aware Permutation",
+ * abstract): tokens are clustered by k-means on their Q (respectively K) vectors,
+ * reordered so that each cluster is contiguous, and a top-p budget over the clusters
+ * picks the critical key clusters of each query cluster.  The page gives no formulas;
+ * the readings used here:
+ *   - Lloyd's k-means per head, separately on Q and on K, `iters` rounds of assignment
+ *     then update; initial centroids are the rows rho_j = floor((2j+1) N / (2C));
+ *   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32 (both dot products summed in
+ *     dimension order, one fused multiply-add per term), ties to the smaller j;
+ *   - update: fp64 sum of the members in token order, divided by the member count and
+ *     rounded to fp32; an empty cluster keeps its centroid;
+ *   - cluster-major order: slots sorted by (cluster, token);
+ *   - criticality of key cluster j for query cluster i: n_j exp(s_ij - max_j s_ij) with
+ *     s_ij = scale * cq_i . ck_j (fp64, dimension order, fused multiply-adds); the kept
+ *     clusters are the shortest prefix of the list sorted by weight (descending, ties to
+ *     the smaller j) whose running sum reaches top_p times the sum of the whole list;
+ *   - block pair (a, b) of the two cluster-major layouts is kept when some query slot of
+ *     block a and some key slot of block b belong to a kept cluster pair.
+ * The floating-point steps that decide an integer (assignment, top-p) are taken in the
+ * precision and order stated above, which is also the CUDA path's.
+ * ------------------------------------------------------------------------------------- */
+
+/* 2^n for an integer n in the normal range, built from its bit pattern (exact). */
+static double pow2i(int64_t n)
+{
+    uint64_t bits = (uint64_t)(n + 1023) << 52;
+    double r;
+    memcpy(&r, &bits, sizeof r);
+    return r;
+}
+
+/*
+ * exp(x) for x <= 0 (Cody and Waite's argument reduction, x = n ln2 + r with ln2 split into
+ * a 32-bit head and a tail, then the Taylor series of e^r to degree 13, Horner form with
+ * fused multiply-adds).  Below -700 the result is 0: weights that small do not matter and
+ * the scaling stays exact.
+ */
+double or_exp_neg(double x)
+{
+    static const double ln2_hi = 0x1.62e42fee00000p-1, ln2_lo = 0x1.a39ef35793c76p-33;
+    static const double inv_ln2 = 0x1.71547652b82fep+0;
+    static const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1,
+                                 0x1.5555555555555p-3, 0x1.5555555555555p-5, 0x1.1111111111111p-7,
+                                 0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
+                                 0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+                                 0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+    if (!(x > -700.0)) return 0.0;
+    if (x > 0.0) x = 0.0;
+    double n = nearbyint(x * inv_ln2);
+    double r = fma(-n, ln2_hi, x);
+    r = fma(-n, ln2_lo, r);
+    double p = c[13];
+    for (int i = 12; i >= 0; --i) p = fma(p, r, c[i]);
+    return p * pow2i((int64_t)n);
+}
+
+/* Squared norm and dot product in fp32, dimension order, one fused multiply-add per term. */
+static float dot_f32(const float *a, const float *b, int64_t d)
+{
+    float acc = 0.0f;
+    for (int64_t x = 0; x < d; ++x) acc = fmaf(a[x], b[x], acc);
+    return acc;
+}
+
+/*
+ * k-means of one head's rows x [N, d] (fp32 values) into C clusters with `iters` >= 1
+ * rounds.  Outputs: cent [C, d] after the last update, label [N] from the last assignment,
+ * count [C] of that assignment.  Returns 0, or -1 on a bad argument or allocation failure.
+ */
+int or_kmeans(const float *x, int64_t N, int64_t d, int64_t C, int64_t iters, float *cent, int32_t *label,
+              int32_t *count)
+{
+    if (C < 1 || C > N || iters < 1) return -1;
+    float *nc = (float *)malloc(sizeof(float) * (size_t)C);
+    double *sum = (double *)malloc(sizeof(double) * (size_t)(C * d));
+    if (!nc || !sum) { free(nc); free(sum); return -1; }
+    for (int64_t j = 0; j < C; ++j) {
+        int64_t r = ((2 * j + 1) * N) / (2 * C);
+        memcpy(cent + j * d, x + r * d, sizeof(float) * (size_t)d);
+    }
+    for (int64_t it = 0; it < iters; ++it) {
+        for (int64_t j = 0; j < C; ++j) nc[j] = dot_f32(cent + j * d, cent + j * d, d);
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < N; ++t) {
+            int32_t best = 0;
+            float best_d = 0.0f;
+            for (int64_t j = 0; j < C; ++j) {
+                float dist = nc[j] - 2.0f * dot_f32(x + t * d, cent + j * d, d);
+                if (j == 0 || dist < best_d) { best = (int32_t)j; best_d = dist; }
+            }
+            label[t] = best;
+        }
+        memset(count, 0, sizeof(int32_t) * (size_t)C);
+        memset(sum, 0, sizeof(double) * (size_t)(C * d));
+        for (int64_t t = 0; t < N; ++t) {
+            int64_t j = label[t];
+            count[j] += 1;
+            for (int64_t q = 0; q < d; ++q) sum[j * d + q] += (double)x[t * d + q];
+        }
+        for (int64_t j = 0; j < C; ++j)
+            if (count[j] > 0)
+                for (int64_t q = 0; q < d; ++q) cent[j * d + q] = (float)(sum[j * d + q] / (double)count[j]);
+    }
+    free(nc); free(sum);
+    return 0;
+}
+
+/* Cluster-major order: perm[slot] = token, slots sorted by (label, token).  offset [C + 1]. */
+void or_cluster_perm(const int32_t *label, int64_t N, int64_t C, int32_t *perm, int32_t *offset)
+{
+    for (int64_t j = 0; j <= C; ++j) offset[j] = 0;
+    for (int64_t t = 0; t < N; ++t) offset[label[t] + 1] += 1;
+    for (int64_t j = 0; j < C; ++j) offset[j + 1] += offset[j];
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (size_t)(C > 0 ? C : 1));
+    if (!next) return;
+    for (int64_t j = 0; j < C; ++j) next[j] = offset[j];
+    for (int64_t t = 0; t < N; ++t) perm[next[label[t]]++] = (int32_t)t;
+    free(next);
+}
+
+/*
+ * Top-p key clusters of every query cluster.  keep[i * Ck + j]; a query cluster with no
+ * member keeps nothing, an empty key cluster is never kept.  scale and p as described
+ * above (0 < p <= 1).
+ */
+void or_semantic_keep(const float *cq, const int32_t *nq, int64_t Cq, const float *ck, const int32_t *nk,
+                      int64_t Ck, int64_t d, double scale, double p, uint8_t *keep)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < Cq; ++i) {
+        uint8_t *row = keep + i * Ck;
+        memset(row, 0, (size_t)Ck);
+        if (nq[i] == 0) continue;
+        double *w = (double *)malloc(sizeof(double) * (size_t)Ck);
+        uint8_t *used = (uint8_t *)calloc((size_t)Ck, 1);
+        if (!w || !used) { free(w); free(used); continue; }
+        double m = -INFINITY;
+        for (int64_t j = 0; j < Ck; ++j) {
+            if (nk[j] == 0) continue;
+            double acc = 0.0;
+            for (int64_t x = 0; x < d; ++x) acc = fma((double)cq[i * d + x], (double)ck[j * d + x], acc);
+            w[j] = scale * acc;
+            if (w[j] > m) m = w[j];
+        }
+        int64_t live = 0;
+        for (int64_t j = 0; j < Ck; ++j)
+            if (nk[j] > 0) { w[j] = (double)nk[j] * or_exp_neg(w[j] - m); ++live; }
+        /* the list sorted by weight, by repeated selection of the largest remaining entry */
+        int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)(live > 0 ? live : 1));
+        if (!order) { free(w); free(used); continue; }
+        for (int64_t pos = 0; pos < live; ++pos) {
+            int64_t best = -1;
+            for (int64_t j = 0; j < Ck; ++j) {
+                if (nk[j] == 0 || used[j]) continue;
+                if (best < 0 || w[j] > w[best]) best = j;
+            }
+            used[best] = 1;
+            order[pos] = best;
+        }
+        double total = 0.0;
+        for (int64_t pos = 0; pos < live; ++pos) total += w[order[pos]];
+        double target = p * total, cum = 0.0;
+        for (int64_t pos = 0; pos < live; ++pos) {
+            row[order[pos]] = 1;
+            cum += w[order[pos]];
+            if (cum >= target) break;
+        }
+        free(order); free(w); free(used);
+    }
 }
