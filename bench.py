@@ -95,6 +95,19 @@ def stage_work(wl, kinds, pipe, pairs):
     and the number of exponentials the attention evaluates."""
     from block_sparse_attention_31_b200 import _lib
     N, d, row = wl.N, wl.d, wl.d * 2
+    if wl.mode == "semantic":
+        BH = wl.B * wl.H
+        nwords = -(-pipe.nblk // 32)
+        cq, ck = wl.clusters
+        out = {
+            # k-means: per round one fp32 dot product per (row, centroid) pair (2*d flops) for
+            # Q and K; the update, order and the rest are lower-order
+            "profile": {"flops": BH * wl.kmeans_iters * 2.0 * d * N * (cq + ck), "bound": "fp32"},
+            "permute": {"bytes": BH * 3.0 * 2 * N * row, "bound": "hbm"},
+            "mask": {"bytes": BH * pipe.nblk * (nwords + pipe.max_kv + 1) * 4.0, "bound": "hbm"},
+            "unpermute": {"bytes": BH * 2.0 * N * row, "bound": "hbm"},
+        }
+        return out, float(pairs) * 128 * wl.block
     R = _lib.vsa_layout_rows(pipe.shape)
     n_t = sum(1 for k in kinds if k == _lib.VSA_TEMPORAL)
     n_c = sum(1 for k in kinds if k == _lib.VSA_CUBE)
@@ -119,13 +132,23 @@ def stage_work(wl, kinds, pipe, pairs):
     return out, exp2
 
 
+# fp32 FMA peak of the CUDA cores (not measured): 148 SMs x 128 lanes x 2 flops at the maximum
+# SM clock (1965 MHz); the k-means assignment runs there, not on the tensor cores
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
     out = {}
     for name, w in work.items():
         t = stage_ms[name] / 1e3
         if t <= 0 or w.get("bytes", 1) == 0:
             continue
-        if w["bound"] == "hbm":
+        if w["bound"] == "fp32":
+            tf = w["flops"] / t / 1e12
+            out[name] = {"bound": "alu", "flops": w["flops"], "achieved": tf, "peak": FP32_PEAK_TFLOPS,
+                         "unit": "TFLOP/s", "frac": tf / FP32_PEAK_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"}
+        elif w["bound"] == "hbm":
             gbs = w["bytes"] / t / 1e9
             out[name] = {"bound": "hbm", "bytes": w["bytes"], "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": gbs / hbm_gbs}
@@ -315,6 +338,75 @@ class Pipeline:
             ev[5].record()
 
 
+class SemanticPipeline:
+    """The semantic-permutation call (Sparse VideoGen2 page, abstract), stage by stage through
+    the C ABI.  Its stages fill the same five timing slots: k-means of Q and K ("profile"),
+    row gathers into the cluster-major orders ("permute"), the top-p cluster budget and block
+    mask ("mask"), the attention, and the scatter of O back to token order ("unpermute")."""
+
+    def __init__(self, wl, device):
+        from block_sparse_attention_31_b200 import _lib
+        self.lib, self.wl, self.in_kernel, self.order = _lib, wl, False, None
+        self.shape = _lib.make_shape(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block)
+        self.cq, self.ck = wl.clusters
+        self.params = _lib.make_sem_params(self.cq, self.ck, wl.kmeans_iters, wl.top_p)
+        BH, N, d = wl.B * wl.H, wl.N, wl.d
+        self.nblk = -(-N // wl.block)
+        self.max_kv = self.nblk
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        self.cent = [torch.empty(BH, c, d, dtype=f32, device=device) for c in (self.cq, self.ck)]
+        self.label = [torch.empty(BH, N, dtype=i32, device=device) for _ in range(2)]
+        self.count = [torch.empty(BH, c, dtype=i32, device=device) for c in (self.cq, self.ck)]
+        self.perm = [torch.empty(BH, N, dtype=i32, device=device) for _ in range(2)]
+        self.qp, self.kp, self.vp, self.op = (torch.empty(wl.B, wl.H, N, d, dtype=bf, device=device)
+                                              for _ in range(4))
+        self.keep = torch.empty(BH, self.cq, -(-self.ck // 32), dtype=i32, device=device)
+        self.bits = torch.zeros(wl.B, wl.H, self.nblk, -(-self.nblk // 32), dtype=i32, device=device)
+        self.kv_idx = torch.zeros(wl.B, wl.H, self.nblk, self.max_kv, dtype=i32, device=device)
+        self.kv_cnt = torch.zeros(wl.B, wl.H, self.nblk, dtype=i32, device=device)
+        # every head is read from the permuted rows (the kernel's VSA_TEMPORAL addressing)
+        self.kinds = torch.full((BH,), _lib.VSA_TEMPORAL, dtype=torch.uint8, device=device)
+        self.km_bytes = _lib.vsa_kmeans_workspace_size(self.shape, max(self.cq, self.ck))
+        self.km_ws = torch.empty(self.km_bytes, dtype=torch.uint8, device=device)
+        self.mask_bytes = _lib.vsa_semantic_mask_workspace_size(self.shape)
+        self.mask_ws = torch.empty(self.mask_bytes, dtype=torch.uint8, device=device)
+        self.err = torch.zeros(1, dtype=i32, device=device)
+        self.launches = (2 * (1 + 3 * wl.kmeans_iters)  # k-means: init, then assign, sort, update per round
+                         + 3 + 4 + 1 + 1)               # gathers, mask (keep, 2 ranges, blocks), attention, scatter
+
+    def step(self, q, k, v, o, ev=None):
+        L, s, wl = self.lib, None, self.wl
+        if ev is not None:
+            ev[0].record()
+        for j, (x, C) in enumerate(((q, self.cq), (k, self.ck))):
+            L.vsa_kmeans(x, self.shape, C, wl.kmeans_iters, self.cent[j], self.label[j], self.count[j], self.perm[j],
+                         self.km_ws, self.km_bytes, self.err, s)
+        if ev is not None:
+            ev[1].record()
+        L.vsa_gather_rows(q, self.perm[0], self.qp, self.shape, self.err, s)
+        L.vsa_gather_rows(k, self.perm[1], self.kp, self.shape, self.err, s)
+        L.vsa_gather_rows(v, self.perm[1], self.vp, self.shape, self.err, s)
+        if ev is not None:
+            ev[2].record()
+        L.vsa_semantic_mask(self.cent[0], self.count[0], self.label[0], self.perm[0], self.cq, self.cent[1],
+                            self.count[1], self.label[1], self.perm[1], self.ck, self.shape, wl.top_p, 0.0,
+                            self.keep, self.bits, self.kv_idx, self.kv_cnt, self.max_kv, self.mask_ws,
+                            self.mask_bytes, self.err, s)
+        if ev is not None:
+            ev[3].record()
+        L.vsa_sparse_attn_fwd(L.qkvo(q, k, v, o), L.qkvo(self.qp, self.kp, self.vp, self.op), self.kinds,
+                              self.kv_idx, self.kv_cnt, self.max_kv, self.shape, 0.0, self.err, s)
+        if ev is not None:
+            ev[4].record()
+        L.vsa_scatter_rows(self.op, None, self.perm[0], o, None, self.shape, self.err, s)
+        if ev is not None:
+            ev[5].record()
+
+
+def make_pipeline(wl, device, in_kernel=False):
+    return SemanticPipeline(wl, device) if wl.mode == "semantic" else Pipeline(wl, device, in_kernel=in_kernel)
+
+
 STAGES = ("profile", "permute", "mask", "attention", "unpermute")
 
 
@@ -342,7 +434,7 @@ def gpu_arm(args, wl, rank, world, device):
     q, k, v = synthetic.make_qkv(wl, seed=rank_seed(wl.seed, rank))
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     o = torch.empty_like(qd)
-    pipe = Pipeline(wl, device, in_kernel=args.layout == "kernel")
+    pipe = make_pipeline(wl, device, in_kernel=args.layout == "kernel")
     for _ in range(args.warmup):
         pipe.step(qd, kd, vd, o)
     torch.cuda.synchronize()
@@ -382,12 +474,17 @@ def gpu_arm(args, wl, rank, world, device):
     e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], device)
     return dict(ms=ms, stage_ms=stage_ms, alg=alg, exe=exe, dense=dense, pairs=pairs, kept=kept_frac,
                 swork=swork, exp2=exp2,
-                clocks=clk.summary(), launches=pipe.launches, e2e=e2e, w_s=pipe.params.w_s, w_t=pipe.params.w_t,
+                clocks=clk.summary(), launches=pipe.launches, e2e=e2e, w_s=getattr(pipe.params, "w_s", None),
+                w_t=getattr(pipe.params, "w_t", None),
                 kinds=pipe.kinds.cpu().tolist())
 
 
 def e2e_arm(args, wl, q, k, v, device):
     import block_sparse_attention_31_b200 as vsa
+    if wl.mode == "semantic":
+        plan = vsa.SemanticAttention(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, cq=wl.clusters[0],
+                                     ck=wl.clusters[1], iters=wl.kmeans_iters, top_p=wl.top_p, device=device)
+        return _e2e_run(args, plan, q, k, v, None, "SemanticAttention.run_host")
     select = {"profiled": "profile", "fixed": "given", "cube": "cube"}[wl.mode]
     kw = dict(select=select, dtype=q.dtype, device=device, layout_in_kernel=args.layout == "kernel")
     if wl.mode == "profiled":
@@ -397,8 +494,12 @@ def e2e_arm(args, wl, q, k, v, device):
     else:
         kw.update(w_s=wl.w_s, w_t=wl.w_t)
     plan = vsa.SparseAttention(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, **kw)
-    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     kinds = torch.tensor(list(wl.fixed_kinds), dtype=torch.uint8, device=device) if wl.mode == "fixed" else None
+    return _e2e_run(args, plan, q, k, v, kinds, "SparseAttention.run_host")
+
+
+def _e2e_run(args, plan, q, k, v, kinds, api):
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     steps = max(2, min(args.steps, 10))
     # every step uploads its Q, K, V from pinned host memory and downloads its O; the public
     # run_host overlaps the uploads of step i+1 and the download of step i-1 with step i
@@ -414,7 +515,7 @@ def e2e_arm(args, wl, q, k, v, device):
     bpe = hq.element_size()
     return {"ms_per_step": a.elapsed_time(b) / steps, "h2d_bytes_per_step": 3 * hq.numel() * bpe,
             "d2h_bytes_per_step": outs[0].numel() * bpe, "steps": steps,
-            "api": "SparseAttention.run_host (uploads, compute and downloads of consecutive steps overlap)"}
+            "api": f"{api} (uploads, compute and downloads of consecutive steps overlap)"}
 
 
 # ---------------------------------------------------------------------------------------
@@ -427,9 +528,20 @@ def oracle_sample(wl, seconds: float, seed: int = 0):
     t_begin = time.perf_counter()
     q, k, v = synthetic.make_qkv(wl, seed=seed, heads=[0, 1] if wl.H > 1 else [0])
     heads = q.shape[1]
-    kinds, keeps = [], []
+    kinds, keeps, kslots = [], [], []
     t0 = time.perf_counter()
     for h in range(heads):
+        if wl.mode == "semantic":
+            res = oracle.semantic_head(q[0, h], k[0, h], None, wl.clusters[0], wl.clusters[1], wl.kmeans_iters,
+                                       wl.top_p, wl.block, attention=False)
+            qs, ks = np.empty(wl.N, dtype=np.int64), np.empty(wl.N, dtype=np.int64)
+            qs[res["perm_q"]] = np.arange(wl.N)
+            ks[res["perm_k"]] = np.arange(wl.N)
+            kinds.append(qs)
+            kslots.append(ks)
+            keeps.append(res["keep_blocks"])
+            continue
+        kslots.append(None)
         if wl.mode == "cube":
             kinds.append(oracle.CUBE)
             keeps.append(oracle.cube_topk_keep(q[0, h], k[0, h], wl.F, wl.Hl, wl.Wl, wl.topk, wl.cube))
@@ -452,13 +564,15 @@ def oracle_sample(wl, seconds: float, seed: int = 0):
     rng = np.random.default_rng(seed)
     while spent < seconds:
         for h in range(heads):
-            slots = oracle.layout_slots(kinds[h], wl.F, wl.Hl, wl.Wl, wl.cube)
+            # semantic heads: kinds[h] holds the query slots, kslots[h] the key slots
+            slots = (kinds[h] if kslots[h] is not None
+                     else oracle.layout_slots(kinds[h], wl.F, wl.Hl, wl.Wl, wl.cube))
+            ks = slots if kslots[h] is None else kslots[h]
             rows = np.sort(rng.choice(wl.N, size=min(n, wl.N), replace=False))
             t1 = time.perf_counter()
-            oracle.attention_rows(q[0, h], k[0, h], v[0, h], slots, wl.block, keeps[h], rows=rows)
+            oracle.attention_rows(q[0, h], k[0, h], v[0, h], slots, wl.block, keeps[h], rows=rows, kslots=ks)
             spent += time.perf_counter() - t1
-            blk = slots // wl.block
-            allowed = keeps[h][blk[rows]][:, blk].sum()
+            allowed = keeps[h][(slots // wl.block)[rows]][:, ks // wl.block].sum()
             flops += 4.0 * wl.d * float(allowed)
             rows_done += len(rows)
         n = min(n * 2, 4096)
@@ -539,10 +653,16 @@ def main():
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.F, wl.Hl, wl.Wl], "d": wl.d,
                    "block": wl.block, "mode": wl.mode, "w_s": res["w_s"], "w_t": res["w_t"],
                    "kept_block_fraction": res["kept"], "head_kinds": res["kinds"],
-                   "layout": ("temporal heads gathered in the attention kernel"
+                   "layout": ("cluster-major copies (Q by its k-means clusters, K and V by theirs)"
+                              if wl.mode == "semantic" else "temporal heads gathered in the attention kernel"
                               if args.layout == "kernel" and wl.mode != "cube" else "permuted copies"),
                    "l2": "inputs larger than L2 (Q,K,V = %.0f MB > 126 MB); no flush" %
                          (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6)},
+        **({"semantic": {"clusters_q": wl.clusters[0], "clusters_k": wl.clusters[1],
+                         "kmeans_iters": wl.kmeans_iters, "top_p": wl.top_p,
+                         "stage_slots": "profile = k-means of Q and K, permute = row gathers, mask = top-p "
+                                        "budget and block mask, unpermute = scatter of O"}}
+           if wl.mode == "semantic" else {}),
         "value_definition": "sparse-actual TFLOP/s of the whole call: algorithmic flops of the kept blocks "
                             "(4*d*valid_q*valid_k per kept pair) / ms per call, summed over ranks",
         "dense_equiv_tflops": aggregate_tflops(res["dense"], res["ms"], world),

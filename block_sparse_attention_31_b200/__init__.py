@@ -17,13 +17,77 @@ from ._lib import (VSA_BF16, VSA_CUBE, VSA_F32, VSA_SELECT_CUBE, VSA_SELECT_GIVE
                    vsa_attention_workspace_layout, vsa_attention_workspace_size, vsa_block_order,
                    vsa_build_mask, vsa_get_device_error, vsa_layout_rows, vsa_mask_workspace_size, vsa_max_kv, vsa_num_blocks,
                    vsa_pattern_window, vsa_permute, vsa_profile_heads, vsa_profile_rows, vsa_profile_workspace_size,
-                   vsa_sparse_attn_fwd, vsa_sparse_attn_fwd_natural, vsa_unpermute)
+                   vsa_sparse_attn_fwd, vsa_sparse_attn_fwd_natural, vsa_unpermute, SemParams, make_sem_params,
+                   vsa_gather_rows, vsa_kmeans, vsa_kmeans_workspace_size, vsa_scatter_rows, vsa_semantic_attention,
+                   vsa_semantic_mask, vsa_semantic_mask_workspace_size, vsa_semantic_workspace_size)
 
 _SELECT = {"profile": VSA_SELECT_PROFILE, "given": VSA_SELECT_GIVEN, "cube": VSA_SELECT_CUBE}
 _DTYPE = {torch.float32: VSA_F32, torch.bfloat16: VSA_BF16}
 
 
-class SparseAttention:
+class _HostPipelined:
+    """run_host for a configured call: subclasses provide __call__(q, k, v, out=, kinds=, stream=)
+    and the attributes B, H, N, d, dtype and device."""
+
+    def run_host(self, batches, outs=None, kinds: Optional[torch.Tensor] = None, timing=None):
+        """Run the call on a sequence of host batches with the transfers overlapped: while call i
+        computes, the inputs of call i+1 upload and the output of call i-1 downloads (three
+        streams, two device buffer sets).  ``batches`` is a list of (q, k, v) CPU tensors, which
+        must be pinned for the copies to overlap; ``outs`` is a list of CPU output tensors
+        (pinned ones are allocated when None).  Returns ``outs`` once every output has arrived.
+        The log-sum-exp, when configured, stays on the device and is not returned.  ``timing``, a
+        pair of timing-enabled CUDA events, is recorded before the first upload and after the
+        last download."""
+        n = len(batches)
+        shape = (self.B, self.H, self.N, self.d)
+        if outs is None:
+            outs = [torch.empty(shape, dtype=self.dtype).pin_memory() for _ in range(n)]
+        if len(outs) != n:
+            raise ValueError("need one output tensor per batch")
+        for (q, k, v), o in zip(batches, outs):
+            for t in (q, k, v, o):
+                if t.device.type != "cpu" or t.dtype != self.dtype or tuple(t.shape) != shape:
+                    raise ValueError(f"host tensors of shape {shape} and dtype {self.dtype} expected")
+        if not hasattr(self, "_host_bufs"):
+            self._host_bufs = [[torch.empty(shape, dtype=self.dtype, device=self.device) for _ in range(4)]
+                               for _ in range(2)]  # q, k, v, o per buffer set
+            self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]  # upload, compute, download
+        up, comp, down = self._streams
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        up_done, comp_done, down_done = [], [], []
+        up.wait_stream(torch.cuda.current_stream(self.device))
+        if timing is not None:
+            timing[0].record(up)
+        for i, ((q, k, v), o) in enumerate(zip(batches, outs)):
+            dq, dk, dv, do = self._host_bufs[i % 2]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[i - 2])  # call i-2 has read this buffer set
+                dq.copy_(q, non_blocking=True)
+                dk.copy_(k, non_blocking=True)
+                dv.copy_(v, non_blocking=True)
+                up_done.append(ev())
+                up_done[i].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(up_done[i])
+                if i >= 2:
+                    comp.wait_event(down_done[i - 2])  # call i-2's output has left this buffer
+                self(dq, dk, dv, out=do, kinds=kinds, stream=comp)
+                comp_done.append(ev())
+                comp_done[i].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[i])
+                o.copy_(do, non_blocking=True)
+                down_done.append(ev())
+                down_done[i].record(down)
+        if timing is not None:
+            timing[1].record(down)
+        down.synchronize()
+        return outs
+
+
+
+class SparseAttention(_HostPipelined):
     """One configured attention call over a B x H x (F x Hl x Wl) x d problem.
 
     select:  "profile" (heads pick spatial/temporal by online profiling), "given" (kinds
@@ -92,67 +156,56 @@ class SparseAttention:
                       self.mse, self.ws, self.ws_bytes, self.err, stream)
         return (out, lse) if self.with_lse else out
 
-    def run_host(self, batches, outs=None, kinds: Optional[torch.Tensor] = None, timing=None):
-        """Run the call on a sequence of host batches with the transfers overlapped: while call i
-        computes, the inputs of call i+1 upload and the output of call i-1 downloads (three
-        streams, two device buffer sets).  ``batches`` is a list of (q, k, v) CPU tensors, which
-        must be pinned for the copies to overlap; ``outs`` is a list of CPU output tensors
-        (pinned ones are allocated when None).  Returns ``outs`` once every output has arrived.
-        The log-sum-exp, when configured, stays on the device and is not returned.  ``timing``, a
-        pair of timing-enabled CUDA events, is recorded before the first upload and after the
-        last download."""
-        n = len(batches)
-        shape = (self.B, self.H, self.N, self.d)
-        if outs is None:
-            outs = [torch.empty(shape, dtype=self.dtype).pin_memory() for _ in range(n)]
-        if len(outs) != n:
-            raise ValueError("need one output tensor per batch")
-        for (q, k, v), o in zip(batches, outs):
-            for t in (q, k, v, o):
-                if t.device.type != "cpu" or t.dtype != self.dtype or tuple(t.shape) != shape:
-                    raise ValueError(f"host tensors of shape {shape} and dtype {self.dtype} expected")
-        if not hasattr(self, "_host_bufs"):
-            self._host_bufs = [[torch.empty(shape, dtype=self.dtype, device=self.device) for _ in range(4)]
-                               for _ in range(2)]  # q, k, v, o per buffer set
-            self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]  # upload, compute, download
-        up, comp, down = self._streams
-        ev = lambda: torch.cuda.Event()  # noqa: E731
-        up_done, comp_done, down_done = [], [], []
-        up.wait_stream(torch.cuda.current_stream(self.device))
-        if timing is not None:
-            timing[0].record(up)
-        for i, ((q, k, v), o) in enumerate(zip(batches, outs)):
-            dq, dk, dv, do = self._host_bufs[i % 2]
-            with torch.cuda.stream(up):
-                if i >= 2:
-                    up.wait_event(comp_done[i - 2])  # call i-2 has read this buffer set
-                dq.copy_(q, non_blocking=True)
-                dk.copy_(k, non_blocking=True)
-                dv.copy_(v, non_blocking=True)
-                up_done.append(ev())
-                up_done[i].record(up)
-            with torch.cuda.stream(comp):
-                comp.wait_event(up_done[i])
-                if i >= 2:
-                    comp.wait_event(down_done[i - 2])  # call i-2's output has left this buffer
-                self(dq, dk, dv, out=do, kinds=kinds, stream=comp)
-                comp_done.append(ev())
-                comp_done[i].record(comp)
-            with torch.cuda.stream(down):
-                down.wait_event(comp_done[i])
-                o.copy_(do, non_blocking=True)
-                down_done.append(ev())
-                down_done[i].record(down)
-        if timing is not None:
-            timing[1].record(down)
-        down.synchronize()
-        return outs
-
     def device_error(self) -> int:
         return vsa_get_device_error(self.err)
 
     def clear_error(self):
         self.err.zero_()
+
+
+class SemanticAttention(_HostPipelined):
+    """Block-sparse attention with the semantic-aware permutation (Sparse VideoGen2 page,
+    abstract): per-head k-means of Q (``cq`` clusters) and K (``ck``), cluster-major orders,
+    a ``top_p`` budget over cluster pairs, then the same attention kernel.  bf16 only, no
+    cube dims."""
+
+    def __init__(self, B: int, H: int, F: int, Hl: int, Wl: int, d: int, block: int = 128, *, cq: int = 128,
+                 ck: int = 128, iters: int = 4, top_p: float = 0.6, scale: float = 0.0, with_lse: bool = False,
+                 device="cuda"):
+        self.B, self.H, self.F, self.Hl, self.Wl, self.d, self.block = B, H, F, Hl, Wl, d, block
+        self.N = F * Hl * Wl
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device, self.dtype = dev, torch.bfloat16
+        self.shape = make_shape(B, H, F, Hl, Wl, d, block)
+        self.params = make_sem_params(cq, ck, iters, top_p, scale)
+        self.ws_bytes = vsa_semantic_workspace_size(self.shape, self.params)
+        if self.ws_bytes == 0:
+            raise VsaError(_lib.VSA_ERR_INVALID_ARG, "vsa_semantic_workspace_size")
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.with_lse = with_lse
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, kinds=None, stream=None):
+        if kinds is not None:
+            raise ValueError("the semantic call chooses its blocks itself; kinds must be None")
+        for t in (q, k, v):
+            if t.dtype != torch.bfloat16 or t.device != self.device or not t.is_contiguous():
+                raise ValueError("q, k, v must be contiguous bf16 tensors on the configured device")
+            if tuple(t.shape) != (self.B, self.H, self.N, self.d):
+                raise ValueError(f"expected shape {(self.B, self.H, self.N, self.d)}, got {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty_like(q)
+        if self.with_lse and lse is None:
+            lse = torch.empty(self.B, self.H, self.N, dtype=torch.float32, device=self.device)
+        vsa_semantic_attention(qkvo(q, k, v, out, lse), self.shape, self.params, self.ws, self.ws_bytes, self.err,
+                               stream)
+        return (out, lse) if self.with_lse else out
+
+    def device_error(self) -> int:
+        return vsa_get_device_error(self.err)
 
 
 def attention(q, k, v, F: int, Hl: int, Wl: int, **kw):
@@ -162,7 +215,9 @@ def attention(q, k, v, F: int, Hl: int, Wl: int, **kw):
     return plan(q, k, v)
 
 
-__all__ = ["SparseAttention", "attention", "VsaError", "Shape", "Params", "QKVO", "make_shape", "make_params", "qkvo",
+__all__ = ["SparseAttention", "SemanticAttention", "attention", "SemParams", "make_sem_params", "vsa_gather_rows",
+           "vsa_kmeans", "vsa_kmeans_workspace_size", "vsa_scatter_rows", "vsa_semantic_attention",
+           "vsa_semantic_mask", "vsa_semantic_mask_workspace_size", "vsa_semantic_workspace_size", "VsaError", "Shape", "Params", "QKVO", "make_shape", "make_params", "qkvo",
            "vsa_attention", "vsa_attention_workspace_layout", "vsa_attention_workspace_size", "vsa_block_order", "vsa_build_mask",
            "vsa_get_device_error", "vsa_layout_rows", "vsa_mask_workspace_size", "vsa_max_kv", "vsa_num_blocks",
            "vsa_pattern_window", "vsa_permute", "vsa_profile_heads", "vsa_profile_rows",

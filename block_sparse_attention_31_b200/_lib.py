@@ -41,6 +41,11 @@ class Params(ctypes.Structure):
                 ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("layout_in_kernel", ctypes.c_int)]
 
 
+class SemParams(ctypes.Structure):
+    _fields_ = [("cq", ctypes.c_int), ("ck", ctypes.c_int), ("iters", ctypes.c_int), ("top_p", ctypes.c_float),
+                ("scale", ctypes.c_float)]
+
+
 class QKVO(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
                 ("lse", ctypes.c_void_p)]
@@ -75,6 +80,15 @@ def _load():
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
+        "vsa_kmeans_workspace_size": (sz, [P(Shape), i32]),
+        "vsa_kmeans": (st, [vp, P(Shape), i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]),
+        "vsa_semantic_mask_workspace_size": (sz, [P(Shape)]),
+        "vsa_semantic_mask": (st, [vp, vp, vp, vp, i32, vp, vp, vp, vp, i32, P(Shape), ctypes.c_float,
+                                   ctypes.c_float, vp, vp, vp, vp, i32, vp, sz, vp, vp]),
+        "vsa_gather_rows": (st, [vp, vp, vp, P(Shape), vp, vp]),
+        "vsa_scatter_rows": (st, [vp, vp, vp, vp, vp, P(Shape), vp, vp]),
+        "vsa_semantic_workspace_size": (sz, [P(Shape), P(SemParams)]),
+        "vsa_semantic_attention": (st, [P(QKVO), P(Shape), P(SemParams), vp, sz, vp, vp]),
         "vsa_selftest_exp2": (st, [vp, vp, vp, i32, vp]),
         "vsa_selftest_wait_timeout": (st, [vp, vp, vp]),
     }
@@ -267,3 +281,53 @@ def vsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
 
 def vsa_selftest_wait_timeout(err, waited, stream=None):
     _check(lib.vsa_selftest_wait_timeout(_ptr(err), _ptr(waited), _stream(stream)), "vsa_selftest_wait_timeout")
+
+
+# ---------------------------------------------------------------------------------------
+# semantic-aware permutation
+# ---------------------------------------------------------------------------------------
+
+def make_sem_params(cq, ck, iters, top_p, scale=0.0) -> SemParams:
+    return SemParams(int(cq), int(ck), int(iters), float(top_p), float(scale))
+
+
+def vsa_kmeans_workspace_size(shape: Shape, n_clusters: int) -> int:
+    return int(lib.vsa_kmeans_workspace_size(ctypes.byref(shape), int(n_clusters)))
+
+
+def vsa_kmeans(x, shape: Shape, n_clusters, iters, centroids, labels, counts, perm, ws, ws_bytes, err, stream=None):
+    _check(lib.vsa_kmeans(_ptr(x), ctypes.byref(shape), int(n_clusters), int(iters), _ptr(centroids), _ptr(labels),
+                          _ptr(counts), _ptr(perm), _ptr(ws), int(ws_bytes), _ptr(err), _stream(stream)),
+           "vsa_kmeans")
+
+
+def vsa_semantic_mask_workspace_size(shape: Shape) -> int:
+    return int(lib.vsa_semantic_mask_workspace_size(ctypes.byref(shape)))
+
+
+def vsa_semantic_mask(cent_q, counts_q, labels_q, perm_q, cq, cent_k, counts_k, labels_k, perm_k, ck, shape: Shape,
+                      top_p, scale, keep, bits, kv_idx, kv_cnt, max_kv, ws, ws_bytes, err, stream=None):
+    _check(lib.vsa_semantic_mask(_ptr(cent_q), _ptr(counts_q), _ptr(labels_q), _ptr(perm_q), int(cq), _ptr(cent_k),
+                                 _ptr(counts_k), _ptr(labels_k), _ptr(perm_k), int(ck), ctypes.byref(shape),
+                                 float(top_p), float(scale), _ptr(keep), _ptr(bits), _ptr(kv_idx), _ptr(kv_cnt),
+                                 int(max_kv), _ptr(ws), int(ws_bytes), _ptr(err), _stream(stream)),
+           "vsa_semantic_mask")
+
+
+def vsa_gather_rows(src, perm, dst, shape: Shape, err, stream=None):
+    _check(lib.vsa_gather_rows(_ptr(src), _ptr(perm), _ptr(dst), ctypes.byref(shape), _ptr(err), _stream(stream)),
+           "vsa_gather_rows")
+
+
+def vsa_scatter_rows(src, src_lse, perm, dst, dst_lse, shape: Shape, err, stream=None):
+    _check(lib.vsa_scatter_rows(_ptr(src), _ptr(src_lse), _ptr(perm), _ptr(dst), _ptr(dst_lse), ctypes.byref(shape),
+                                _ptr(err), _stream(stream)), "vsa_scatter_rows")
+
+
+def vsa_semantic_workspace_size(shape: Shape, params: SemParams) -> int:
+    return int(lib.vsa_semantic_workspace_size(ctypes.byref(shape), ctypes.byref(params)))
+
+
+def vsa_semantic_attention(io: QKVO, shape: Shape, params: SemParams, ws, ws_bytes, err, stream=None):
+    _check(lib.vsa_semantic_attention(ctypes.byref(io), ctypes.byref(shape), ctypes.byref(params), _ptr(ws),
+                                      int(ws_bytes), _ptr(err), _stream(stream)), "vsa_semantic_attention")

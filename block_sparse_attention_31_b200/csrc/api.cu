@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -454,6 +455,196 @@ vsa_status vsa_sparse_attn_fwd_natural(const vsa_qkvo* natural, const uint8_t* d
   a.nat_o = natural->o;
   const cudaError_t e = launch_sparse_attn(nat, nat, a, shape->d, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------
+// Semantic-aware permutation ("Sparse VideoGen2" page, abstract)
+// ---------------------------------------------------------------------------------------
+// Shapes of the semantic path: no cube dims (every head has N rows).
+static vsa_status semantic_geom(const vsa_shape* shape, Geom* g) {
+  vsa_status st = make_geom(shape, g);
+  if (st != VSA_OK) return st;
+  if (g->ncubes > 0) return VSA_ERR_UNSUPPORTED;
+  return VSA_OK;
+}
+
+static bool clusters_ok(const Geom& g, int C) { return C >= 1 && C <= kMaxClusters && C <= g.N; }
+
+size_t vsa_kmeans_workspace_size(const vsa_shape* shape, int n_clusters) {
+  Geom g;
+  if (semantic_geom(shape, &g) != VSA_OK || !clusters_ok(g, n_clusters)) return 0;
+  return kmeans_workspace_bytes(shape->B * shape->H, n_clusters);
+}
+
+vsa_status vsa_kmeans(const void* x, const vsa_shape* shape, int n_clusters, int iters, float* d_centroids,
+                      int32_t* d_labels, int32_t* d_counts, int32_t* d_perm, void* ws, size_t ws_bytes, int* d_err,
+                      cudaStream_t stream) {
+  Geom g;
+  vsa_status st = semantic_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!clusters_ok(g, n_clusters) || iters < 1 || iters > 1000) return VSA_ERR_INVALID_ARG;
+  if (!x || !d_centroids || !d_labels || !d_counts || !d_perm || !ws || !d_err || !aligned16(x) ||
+      !aligned16(d_centroids))
+    return VSA_ERR_INVALID_ARG;
+  if (ws_bytes < vsa_kmeans_workspace_size(shape, n_clusters)) return VSA_ERR_WORKSPACE;
+  if (!on_device({x, d_centroids, d_labels, d_counts, d_perm, ws, d_err})) return VSA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_kmeans(x, shape->B * shape->H, g.N, shape->d, n_clusters, iters, d_centroids,
+                                      d_labels, d_counts, d_perm, ws, d_err, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+size_t vsa_semantic_mask_workspace_size(const vsa_shape* shape) {
+  Geom g;
+  if (semantic_geom(shape, &g) != VSA_OK) return 0;
+  return align256(semantic_mask_workspace_bytes(shape->B * shape->H, g.N, g.block));
+}
+
+vsa_status vsa_semantic_mask(const float* d_cent_q, const int32_t* d_counts_q, const int32_t* d_labels_q,
+                             const int32_t* d_perm_q, int cq, const float* d_cent_k, const int32_t* d_counts_k,
+                             const int32_t* d_labels_k, const int32_t* d_perm_k, int ck, const vsa_shape* shape,
+                             float top_p, float scale, uint32_t* d_keep, uint32_t* d_bits, int32_t* d_kv_idx,
+                             int32_t* d_kv_cnt, int max_kv, void* ws, size_t ws_bytes, int* d_err,
+                             cudaStream_t stream) {
+  Geom g;
+  vsa_status st = semantic_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!clusters_ok(g, cq) || !clusters_ok(g, ck)) return VSA_ERR_INVALID_ARG;
+  if (!(top_p > 0.f && top_p <= 1.f) || !(scale >= 0.f) || max_kv <= 0) return VSA_ERR_INVALID_ARG;
+  if (!d_cent_q || !d_counts_q || !d_labels_q || !d_perm_q || !d_cent_k || !d_counts_k || !d_labels_k ||
+      !d_perm_k || !d_keep || !d_bits || !d_kv_idx || !d_kv_cnt || !ws || !d_err || !aligned16(ws))
+    return VSA_ERR_INVALID_ARG;
+  if (ws_bytes < vsa_semantic_mask_workspace_size(shape)) return VSA_ERR_WORKSPACE;
+  if (!on_device({d_cent_q, d_counts_q, d_labels_q, d_perm_q, d_cent_k, d_counts_k, d_labels_k, d_perm_k, d_keep,
+                  d_bits, d_kv_idx, d_kv_cnt, ws, d_err}))
+    return VSA_ERR_INVALID_ARG;
+  const double sc = scale > 0.f ? static_cast<double>(scale) : 1.0 / std::sqrt(static_cast<double>(shape->d));
+  const cudaError_t e = launch_semantic_mask(d_cent_q, d_counts_q, d_labels_q, d_perm_q, cq, d_cent_k, d_counts_k,
+                                             d_labels_k, d_perm_k, ck, shape->B * shape->H, g.N, shape->d, g.block,
+                                             sc, static_cast<double>(top_p), d_keep, d_bits, d_kv_idx, d_kv_cnt,
+                                             max_kv, ws, d_err, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+vsa_status vsa_gather_rows(const void* src, const int32_t* d_perm, void* dst, const vsa_shape* shape, int* d_err,
+                           cudaStream_t stream) {
+  Geom g;
+  vsa_status st = semantic_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!src || !d_perm || !dst || !d_err || !aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
+  if (!on_device({src, d_perm, dst, d_err})) return VSA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_gather_rows(src, d_perm, dst, shape->B * shape->H, g.N, shape->d, d_err, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+vsa_status vsa_scatter_rows(const void* src, const float* src_lse, const int32_t* d_perm, void* dst, float* dst_lse,
+                            const vsa_shape* shape, int* d_err, cudaStream_t stream) {
+  Geom g;
+  vsa_status st = semantic_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!src || !d_perm || !dst || !d_err || !aligned16(src) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
+  if ((src_lse == nullptr) != (dst_lse == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (!on_device({src, src_lse, d_perm, dst, dst_lse, d_err})) return VSA_ERR_INVALID_ARG;
+  const cudaError_t e =
+      launch_scatter_rows(src, src_lse, d_perm, dst, dst_lse, shape->B * shape->H, g.N, shape->d, d_err, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// Workspace of the whole semantic call.
+struct SemLayout {
+  size_t kinds, cent_q, lab_q, cnt_q, perm_q, cent_k, lab_k, cnt_k, perm_k, offs, keep, bits, idx, cnt, mws, pq, pk,
+      pv, po, plse, bytes;
+  int max_kv;
+};
+
+static vsa_status semantic_layout(const vsa_shape* shape, const vsa_semantic_params* sp, SemLayout* L) {
+  Geom g;
+  vsa_status st = semantic_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (sp == nullptr || L == nullptr) return VSA_ERR_INVALID_ARG;
+  if (!clusters_ok(g, sp->cq) || !clusters_ok(g, sp->ck) || sp->iters < 1 || sp->iters > 1000) return VSA_ERR_INVALID_ARG;
+  if (!(sp->top_p > 0.f && sp->top_p <= 1.f) || !(sp->scale >= 0.f)) return VSA_ERR_INVALID_ARG;
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H, N = g.N, d = shape->d, nb = g.nblk;
+  const size_t kwords = (sp->ck + 31) / 32, bwords = (nb + 31) / 32;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L->kinds = take(BH);
+  L->cent_q = take(BH * sp->cq * d * 4);
+  L->lab_q = take(BH * N * 4);
+  L->cnt_q = take(BH * sp->cq * 4);
+  L->perm_q = take(BH * N * 4);
+  L->cent_k = take(BH * sp->ck * d * 4);
+  L->lab_k = take(BH * N * 4);
+  L->cnt_k = take(BH * sp->ck * 4);
+  L->perm_k = take(BH * N * 4);
+  L->offs = take(kmeans_workspace_bytes(static_cast<int>(BH), std::max(sp->cq, sp->ck)));
+  L->keep = take(BH * sp->cq * kwords * 4);
+  L->bits = take(BH * nb * bwords * 4);
+  L->idx = take(BH * nb * nb * 4);
+  L->cnt = take(BH * nb * 4);
+  L->mws = take(semantic_mask_workspace_bytes(static_cast<int>(BH), g.N, g.block));
+  L->pq = take(BH * N * d * 2);
+  L->pk = take(BH * N * d * 2);
+  L->pv = take(BH * N * d * 2);
+  L->po = take(BH * N * d * 2);
+  L->plse = take(BH * N * 4);
+  L->bytes = off;
+  L->max_kv = static_cast<int>(nb);
+  return VSA_OK;
+}
+
+size_t vsa_semantic_workspace_size(const vsa_shape* shape, const vsa_semantic_params* params) {
+  SemLayout L;
+  return semantic_layout(shape, params, &L) == VSA_OK ? L.bytes : 0;
+}
+
+vsa_status vsa_semantic_attention(const vsa_qkvo* io, const vsa_shape* shape, const vsa_semantic_params* params,
+                                  void* ws, size_t ws_bytes, int* d_err, cudaStream_t stream) {
+  SemLayout L;
+  vsa_status st = semantic_layout(shape, params, &L);
+  if (st != VSA_OK) return st;
+  if ((st = check_qkvo(io)) != VSA_OK) return st;
+  if (!ws || !d_err || !aligned16(ws)) return VSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.bytes) return VSA_ERR_WORKSPACE;
+  if (!on_device({io->q, io->k, io->v, io->o, io->lse, ws, d_err})) return VSA_ERR_INVALID_ARG;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(w + off); };
+  auto i32 = [&](size_t off) { return reinterpret_cast<int32_t*>(w + off); };
+  const size_t kmws = L.keep - L.offs;  // bytes reserved for the k-means scratch
+  // 1. clusters and cluster-major orders of Q and of K
+  if ((st = vsa_kmeans(io->q, shape, params->cq, params->iters, f32(L.cent_q), i32(L.lab_q), i32(L.cnt_q),
+                       i32(L.perm_q), w + L.offs, kmws, d_err, stream)) != VSA_OK)
+    return st;
+  if ((st = vsa_kmeans(io->k, shape, params->ck, params->iters, f32(L.cent_k), i32(L.lab_k), i32(L.cnt_k),
+                       i32(L.perm_k), w + L.offs, kmws, d_err, stream)) != VSA_OK)
+    return st;
+  // 2. rows in cluster-major order: Q by its clusters, K and V by the key clusters
+  void *pq = w + L.pq, *pk = w + L.pk, *pv = w + L.pv, *po = w + L.po;
+  if ((st = vsa_gather_rows(io->q, i32(L.perm_q), pq, shape, d_err, stream)) != VSA_OK) return st;
+  if ((st = vsa_gather_rows(io->k, i32(L.perm_k), pk, shape, d_err, stream)) != VSA_OK) return st;
+  if ((st = vsa_gather_rows(io->v, i32(L.perm_k), pv, shape, d_err, stream)) != VSA_OK) return st;
+  // 3. top-p cluster budget and the block mask over the two layouts
+  if ((st = vsa_semantic_mask(f32(L.cent_q), i32(L.cnt_q), i32(L.lab_q), i32(L.perm_q), params->cq, f32(L.cent_k),
+                              i32(L.cnt_k), i32(L.lab_k), i32(L.perm_k), params->ck, shape, params->top_p,
+                              params->scale, reinterpret_cast<uint32_t*>(w + L.keep),
+                              reinterpret_cast<uint32_t*>(w + L.bits), i32(L.idx), i32(L.cnt), L.max_kv, w + L.mws,
+                              ws_bytes - L.mws, d_err, stream)) != VSA_OK)
+    return st;
+  // 4. attention on the permuted rows.  The kernel reads a VSA_TEMPORAL head's N rows from the
+  // permuted set; which permutation produced them does not matter to it.
+  uint8_t* kinds = w + L.kinds;
+  if (cudaMemsetAsync(kinds, kTemporal, static_cast<size_t>(shape->B) * shape->H, stream) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  float* plse = io->lse ? f32(L.plse) : nullptr;
+  const vsa_qkvo perm_set{pq, pk, pv, po, plse};
+  if ((st = vsa_sparse_attn_fwd(io, &perm_set, kinds, i32(L.idx), i32(L.cnt), L.max_kv, nullptr, shape,
+                                params->scale, d_err, stream)) != VSA_OK)
+    return st;
+  // 5. output rows back to token order through the query permutation
+  return vsa_scatter_rows(po, plse, i32(L.perm_q), io->o, io->lse, shape, d_err, stream);
 }
 
 // ---------------------------------------------------------------------------------------

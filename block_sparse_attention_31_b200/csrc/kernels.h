@@ -26,6 +26,27 @@ cudaError_t launch_cube_mask(const uint8_t* kinds, const void* q_cube, const voi
 cudaError_t launch_block_order(const uint8_t* kinds, const Geom& g, int BH, const int32_t* kv_idx,
                                const int32_t* kv_cnt, int max_kv, int32_t* order, cudaStream_t stream);
 
+// Semantic-aware permutation (see semantic.cu).  At most kMaxClusters clusters per tensor.
+constexpr int kMaxClusters = 1024;
+// k-means of x [BH, N, d] bf16: cent [BH, C, d] f32, label [BH, N], counts [BH, C], perm [BH, N]
+// (slot -> token, cluster-major).  ws (kmeans_workspace_bytes): the cluster offsets
+// [BH, C + 1] and the centroids' squared norms [BH, C].
+size_t kmeans_workspace_bytes(int BH, int C);
+cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
+                          int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream);
+// Workspace of launch_semantic_mask: the cluster range of every query and key block.
+size_t semantic_mask_workspace_bytes(int BH, int N, int block);
+cudaError_t launch_semantic_mask(const float* cent_q, const int32_t* counts_q, const int32_t* label_q,
+                                 const int32_t* perm_q, int Cq, const float* cent_k, const int32_t* counts_k,
+                                 const int32_t* label_k, const int32_t* perm_k, int Ck, int BH, int N, int d,
+                                 int block, double scale, double top_p, uint32_t* keep, uint32_t* bits,
+                                 int32_t* kv_idx, int32_t* kv_cnt, int max_kv, void* ws, int* err,
+                                 cudaStream_t stream);
+cudaError_t launch_gather_rows(const void* src, const int32_t* perm, void* dst, int BH, int N, int d, int* err,
+                               cudaStream_t stream);
+cudaError_t launch_scatter_rows(const void* src, const float* src_lse, const int32_t* perm, void* dst, float* dst_lse,
+                                int BH, int N, int d, int* err, cudaStream_t stream);
+
 // Tensor maps of one attention problem (3D: d, rows, B*H).
 struct AttnMaps {
   CUtensorMap q, k, v, o;

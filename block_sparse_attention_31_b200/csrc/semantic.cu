@@ -1,0 +1,690 @@
+// semantic.cu -- semantic-aware permutation ("Sparse VideoGen2" page, abstract): tokens are
+// clustered by k-means on their Q (respectively K) vectors, reordered so that every cluster
+// is contiguous, and a top-p budget over the clusters picks the key clusters each query
+// cluster attends to.  The page gives no formulas; the readings used here:
+//   - Lloyd's k-means per head on the bf16 rows (as fp32), `iters` rounds of assignment then
+//     update, initial centroids the rows rho_j = floor((2j+1) N / (2C));
+//   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32, both dot products summed in dimension
+//     order with one fused multiply-add per term, ties to the smaller j;
+//   - update: fp64 sum of the members in token order, divided by the count, rounded to fp32;
+//     an empty cluster keeps its centroid;
+//   - cluster-major order: slots sorted by (cluster, token);
+//   - weight of key cluster j for query cluster i: n_j exp(s_ij - max_j s_ij), s_ij = scale *
+//     cq_i . ck_j in fp64 (dimension order, fused multiply-adds); kept: the shortest prefix of
+//     the weights sorted in descending order (ties to the smaller j) whose running sum reaches
+//     top_p times the sum of all of them;
+//   - block pair (a, b) of the two cluster-major layouts is kept when some query slot of a
+//     and some key slot of b belong to a kept cluster pair.
+// Every floating-point step that decides an integer (assignment, order, top-p) is written
+// out with explicitly rounded operations, so the result does not depend on contraction.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace vsa {
+
+namespace {
+
+constexpr int kKmTile = 128;     // tokens and centroids per assignment tile
+constexpr int kKmThreads = 256;  // 16 x 16 threads; thread (ty, tx): tokens ty + 16i, centroids tx + 16j
+constexpr int kKeepThreads = 256;
+constexpr int kRowThreads = 256;
+
+constexpr int kKmLd = kKmTile + 4;   // centroid tile [D][kKmLd] fp32: 16-byte aligned rows
+constexpr int kKmLdB = kKmTile + 8;  // token tile [D][kKmLdB] bf16: 16-byte aligned rows
+
+template <int D>
+constexpr size_t assign_smem_bytes() {  // about 100 KB at D = 128: two CTAs per SM
+  return sizeof(float) * (D * kKmLd + kKmTile) + sizeof(__nv_bfloat16) * D * kKmLdB;
+}
+
+// |c|^2 of one centroid held in shared memory: fp32, dimension order, one fused multiply-add
+// per term (the first term of the assignment's distance).
+__device__ __forceinline__ float sq_norm(const float* c, int D) {
+  float acc = 0.f;
+  for (int k = 0; k < D; ++k) acc = __fmaf_rn(c[k], c[k], acc);
+  return acc;
+}
+
+// (dist, j) is a better assignment than (bd, bj): smaller distance, ties to the smaller index.
+__device__ __forceinline__ bool better(float dist, int j, float bd, int bj) {
+  return bj < 0 || dist < bd || (dist == bd && j < bj);
+}
+
+// ---------------------------------------------------------------------------------------
+// k-means
+// ---------------------------------------------------------------------------------------
+
+// cent[bh, j] = x[bh, rho_j] as fp32, and its squared norm.  128 threads, d <= 128.
+__global__ void __launch_bounds__(128) kmeans_init_kernel(const __nv_bfloat16* __restrict__ x, int N, int d, int C,
+                                                          float* __restrict__ cent, float* __restrict__ cnorm) {
+  __shared__ float row_s[128];
+  const int j = blockIdx.x, bh = blockIdx.y;
+  const long long r = ((2LL * j + 1) * N) / (2LL * C);
+  const __nv_bfloat16* src = x + (static_cast<size_t>(bh) * N + r) * d;
+  float* dst = cent + (static_cast<size_t>(bh) * C + j) * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    const float v = __bfloat162float(src[k]);
+    dst[k] = v;
+    row_s[k] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(row_s, d);
+}
+
+// label[bh, t] = nearest centroid of token t.  One CTA: 128 tokens of one head against all
+// centroids, 128 at a time.  Thread (ty, tx) holds tokens ty*8 + i and centroids tx*8 + j
+// (i, j < 8); the tiles are stored transposed ([dimension][token or centroid]) so that each
+// thread reads its 8 values of one dimension with two 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(kKmThreads, 2)
+    kmeans_assign_kernel(const __nv_bfloat16* __restrict__ x, int N, int C, const float* __restrict__ cent,
+                         const float* __restrict__ cnorm, int32_t* __restrict__ label) {
+  extern __shared__ __align__(16) float km_smem[];
+  float* cs = km_smem;            // [D][kKmLd]
+  float* nc = cs + D * kKmLd;     // [128]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(nc + kKmTile);  // [D][kKmLdB] bf16 bits
+  const int bh = blockIdx.y, t0 = blockIdx.x * kKmTile;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * N * D;
+  const float* chd = cent + static_cast<size_t>(bh) * C * D;
+  // token tile: thread e loads 8 dimensions of row e % 128
+  for (int e = tid; e < kKmTile * (D / 8); e += kKmThreads) {
+    const int r = e & (kKmTile - 1), c8 = e / kKmTile;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (t0 + r < N) w = *reinterpret_cast<const uint4*>(xh + static_cast<size_t>(t0 + r) * D + c8 * 8);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      xs[(c8 * 8 + 2 * q) * kKmLdB + r] = static_cast<uint16_t>(ww[q] & 0xffffu);
+      xs[(c8 * 8 + 2 * q + 1) * kKmLdB + r] = static_cast<uint16_t>(ww[q] >> 16);
+    }
+  }
+  float best_d[8];
+  int best_j[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    best_d[i] = 0.f;
+    best_j[i] = -1;
+  }
+  for (int c0 = 0; c0 < C; c0 += kKmTile) {
+    __syncthreads();  // the previous tile's reads of cs and nc are done
+    for (int e = tid; e < kKmTile * (D / 4); e += kKmThreads) {
+      const int r = e & (kKmTile - 1), c4 = e / kKmTile;
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + r < C) w = *reinterpret_cast<const float4*>(chd + static_cast<size_t>(c0 + r) * D + c4 * 4);
+      cs[(c4 * 4 + 0) * kKmLd + r] = w.x;
+      cs[(c4 * 4 + 1) * kKmLd + r] = w.y;
+      cs[(c4 * 4 + 2) * kKmLd + r] = w.z;
+      cs[(c4 * 4 + 3) * kKmLd + r] = w.w;
+    }
+    if (tid < kKmTile) nc[tid] = c0 + tid < C ? cnorm[static_cast<size_t>(bh) * C + c0 + tid] : 0.f;
+    __syncthreads();
+    // acc2[i][p] packs the sums of centroids tx*8 + 2p and tx*8 + 2p + 1; every lane of
+    // fma.rn.f32x2 is one correctly rounded fused multiply-add, as __fmaf_rn
+    uint64_t acc2[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) acc2[i][p] = 0ull;
+#pragma unroll 2
+    for (int k = 0; k < D; ++k) {
+      const uint4 aw = *reinterpret_cast<const uint4*>(xs + k * kKmLdB + ty * 8);  // 8 bf16 tokens
+      const ulonglong2 b_lo = *reinterpret_cast<const ulonglong2*>(cs + k * kKmLd + tx * 8);
+      const ulonglong2 b_hi = *reinterpret_cast<const ulonglong2*>(cs + k * kKmLd + tx * 8 + 4);
+      const uint64_t b2[4] = {b_lo.x, b_lo.y, b_hi.x, b_hi.y};
+      const uint32_t awv[4] = {aw.x, aw.y, aw.z, aw.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a = __uint_as_float((i & 1) ? (awv[i >> 1] & 0xffff0000u) : (awv[i >> 1] << 16));
+        const uint64_t a2 = f2_make(a, a);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) acc2[i][p] = f2_fma(a2, b2[p], acc2[i][p]);
+      }
+    }
+    __syncthreads();  // nc visible to every thread
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int jl = tx * 8 + 2 * p + h, cj = c0 + jl;
+        if (cj < C) {
+          const float n = nc[jl];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float lo, hi;
+            f2_split(acc2[i][p], lo, hi);
+            const float dist = __fmaf_rn(-2.f, h ? hi : lo, n);  // n - 2 dot, rounded once
+            if (better(dist, cj, best_d[i], best_j[i])) {
+              best_d[i] = dist;
+              best_j[i] = cj;
+            }
+          }
+        }
+      }
+    }
+  }
+  // the 16 threads of a half-warp share their tokens: reduce (distance, index) lexicographically
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) {
+      const float od = __shfl_xor_sync(0xffffffffu, best_d[i], off);
+      const int oj = __shfl_xor_sync(0xffffffffu, best_j[i], off);
+      if (oj >= 0 && better(od, oj, best_d[i], best_j[i])) {
+        best_d[i] = od;
+        best_j[i] = oj;
+      }
+    }
+    const int t = t0 + ty * 8 + i;
+    if (tx == 0 && t < N) label[static_cast<size_t>(bh) * N + t] = best_j[i];
+  }
+}
+
+// Counts, offsets and the stable cluster-major order of one head.  The head's tokens are cut
+// into kSortWarps contiguous segments, one per warp: per-segment histograms, offsets from their
+// column sums, each segment's first slot per cluster from the segments before it, then every
+// warp ranks its own segment in token order (32 tokens per step, ranks among equal labels from
+// __match_any_sync).  Shared memory: (kSortWarps + 1) * C ints.
+constexpr int kSortWarps = 16;
+constexpr int kSortPrefetch = 8;  // 32-token steps whose labels are loaded ahead
+
+__global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int32_t* __restrict__ label, int N, int C,
+                                                                      int32_t* __restrict__ counts,
+                                                                      int32_t* __restrict__ offsets,
+                                                                      int32_t* __restrict__ perm, int* err) {
+  extern __shared__ int sort_smem[];
+  int* hist = sort_smem;              // [kSortWarps][C]: counts, then first free slot, per segment
+  int* tot = sort_smem + kSortWarps * C;  // [C]
+  __shared__ int bad_s;
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t* lh = label + static_cast<size_t>(bh) * N;
+  const int seg = (N + kSortWarps - 1) / kSortWarps;
+  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
+  for (int e = tid; e < kSortWarps * C; e += kSortWarps * 32) hist[e] = 0;
+  if (tid == 0) bad_s = 0;
+  __syncthreads();
+  for (int t = s0 + lane; t < s1; t += 32) {
+    const int l = lh[t];
+    if (l >= 0 && l < C) atomicAdd(&hist[warp * C + l], 1);
+    else bad_s = 1;
+  }
+  __syncthreads();
+  if (bad_s) {  // empty clusters: the update and the mask read nothing
+    if (tid == 0) atomicOr(err, kDevErrKvRange);
+    for (int j = tid; j < C; j += kSortWarps * 32) {
+      counts[static_cast<size_t>(bh) * C + j] = 0;
+      offsets[static_cast<size_t>(bh) * (C + 1) + j] = 0;
+    }
+    return;
+  }
+  for (int j = tid; j < C; j += kSortWarps * 32) {
+    int sum = 0;
+    for (int w = 0; w < kSortWarps; ++w) sum += hist[w * C + j];
+    tot[j] = sum;
+    counts[static_cast<size_t>(bh) * C + j] = sum;
+  }
+  __syncthreads();
+  // exclusive scan of tot over the clusters (warp 0, 32 clusters per step)
+  if (warp == 0) {
+    int carry = 0;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+      const int j = j0 + lane;
+      const int v = j < C ? tot[j] : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (j < C) {
+        tot[j] = carry + incl - v;
+        offsets[static_cast<size_t>(bh) * (C + 1) + j] = carry + incl - v;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) offsets[static_cast<size_t>(bh) * (C + 1) + C] = carry;
+  }
+  __syncthreads();
+  for (int j = tid; j < C; j += kSortWarps * 32) {
+    int run = tot[j];
+    for (int w = 0; w < kSortWarps; ++w) {
+      const int c = hist[w * C + j];
+      hist[w * C + j] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  int* cur = hist + warp * C;
+  int32_t* ph = perm + static_cast<size_t>(bh) * N;
+  for (int base = s0; base < s1; base += 32 * kSortPrefetch) {
+    int lab[kSortPrefetch];
+#pragma unroll
+    for (int u = 0; u < kSortPrefetch; ++u) {
+      const int t = base + u * 32 + lane;
+      lab[u] = t < s1 ? lh[t] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kSortPrefetch; ++u) {
+      const int t = base + u * 32 + lane;
+      const int l = lab[u];
+      const unsigned peers = __match_any_sync(0xffffffffu, l);
+      const int rank = __popc(peers & lt);
+      const int slot = l >= 0 ? cur[l] + rank : 0;
+      __syncwarp();
+      if (l >= 0) {
+        ph[slot] = t;
+        if (rank == 0) cur[l] += __popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// New centroids: one CTA per (cluster, head).  The members' rows stream through shared memory
+// kUpdRows at a time (double-buffered; every thread loads 16-byte pieces of the next stage
+// while the current one is summed); thread x < D adds dimension x of the staged rows in token
+// order, in fp64.
+constexpr int kUpdThreads = 256;
+constexpr int kUpdRows = 128;
+
+template <int D>
+constexpr size_t update_smem_bytes() {
+  return 2 * static_cast<size_t>(kUpdRows) * D * sizeof(__nv_bfloat16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                                    const int32_t* __restrict__ counts,
+                                                                    const int32_t* __restrict__ offsets,
+                                                                    const int32_t* __restrict__ perm,
+                                                                    float* __restrict__ cent,
+                                                                    float* __restrict__ cnorm) {
+  extern __shared__ __align__(16) uint4 upd_smem[];
+  constexpr int VPR = D * 2 / 16;                        // 16-byte pieces per row
+  constexpr int PER_T = kUpdRows * VPR / kUpdThreads;    // pieces per thread per stage
+  const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int n = counts[static_cast<size_t>(bh) * C + j];
+  if (n <= 0) return;  // an empty cluster keeps its centroid
+  const int off = offsets[static_cast<size_t>(bh) * (C + 1) + j];
+  const int32_t* ph = perm + static_cast<size_t>(bh) * N + off;
+  const uint4* xh = reinterpret_cast<const uint4*>(x + static_cast<size_t>(bh) * N * D);
+  uint4 reg[PER_T];
+  auto load = [&](int m0) {
+#pragma unroll
+    for (int q = 0; q < PER_T; ++q) {
+      const int e = tid + q * kUpdThreads, r = e / VPR, v = e - r * VPR;
+      const int m = m0 + r;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (m < n) {
+        const int t = ph[m];
+        if (t >= 0 && t < N) val = xh[static_cast<size_t>(t) * VPR + v];
+      }
+      reg[q] = val;
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < PER_T; ++q) upd_smem[buf * kUpdRows * VPR + tid + q * kUpdThreads] = reg[q];
+  };
+  load(0);
+  store(0);
+  __syncthreads();
+  double s = 0.0;
+  int buf = 0;
+  for (int m0 = 0; m0 < n; m0 += kUpdRows) {
+    const bool more = m0 + kUpdRows < n;
+    if (more) load(m0 + kUpdRows);
+    if (tid < D) {
+      const __nv_bfloat16* rows = reinterpret_cast<const __nv_bfloat16*>(upd_smem + buf * kUpdRows * VPR);
+      const int cnt = min(kUpdRows, n - m0);
+      for (int r = 0; r < cnt; ++r) s = __dadd_rn(s, static_cast<double>(__bfloat162float(rows[r * D + tid])));
+    }
+    if (more) store(buf ^ 1);
+    __syncthreads();
+    buf ^= 1;
+  }
+  float* cnew = reinterpret_cast<float*>(upd_smem);  // the staged rows are no longer read
+  if (tid < D) {
+    const float c = __double2float_rn(__ddiv_rn(s, static_cast<double>(n)));
+    cent[(static_cast<size_t>(bh) * C + j) * D + tid] = c;
+    cnew[tid] = c;
+  }
+  __syncthreads();
+  if (tid == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(cnew, D);
+}
+
+// ---------------------------------------------------------------------------------------
+// top-p budget
+// ---------------------------------------------------------------------------------------
+
+// exp(x) for x <= 0: Cody and Waite's reduction x = n ln2 + r (ln2 split into a 32-bit head
+// and a tail), Taylor series of e^r to degree 13 in Horner form, scaling by 2^n built from its
+// bit pattern; 0 below -700.
+__device__ double exp_neg(double x) {
+  const double ln2_hi = 0x1.62e42fee00000p-1, ln2_lo = 0x1.a39ef35793c76p-33;
+  const double inv_ln2 = 0x1.71547652b82fep+0;
+  const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1, 0x1.5555555555555p-3,
+                        0x1.5555555555555p-5, 0x1.1111111111111p-7, 0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13,
+                        0x1.a01a01a01a01ap-16, 0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+                        0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+  if (!(x > -700.0)) return 0.0;
+  if (x > 0.0) x = 0.0;
+  const double n = rint(__dmul_rn(x, inv_ln2));
+  double r = __fma_rn(-n, ln2_hi, x);
+  r = __fma_rn(-n, ln2_lo, r);
+  double p = c[13];
+#pragma unroll
+  for (int i = 12; i >= 0; --i) p = __fma_rn(p, r, c[i]);
+  const double two_n = __longlong_as_double(static_cast<long long>(static_cast<int>(n) + 1023) << 52);
+  return __dmul_rn(p, two_n);
+}
+
+// Kept key clusters of query cluster blockIdx.x of head blockIdx.y: keep[bh, i, ceil(Ck/32)].
+__global__ void __launch_bounds__(kKeepThreads) semantic_keep_kernel(const float* __restrict__ cq,
+                                                                     const int32_t* __restrict__ nq, int Cq,
+                                                                     const float* __restrict__ ck,
+                                                                     const int32_t* __restrict__ nk, int Ck, int D,
+                                                                     double scale, double top_p, int n2,
+                                                                     uint32_t* __restrict__ keep) {
+  extern __shared__ double ks_w[];                 // [n2] weights, then [n2] cluster indices
+  int* ks_i = reinterpret_cast<int*>(ks_w + n2);
+  __shared__ double red[kKeepThreads / 32];
+  __shared__ uint32_t row_s[kMaxClusters / 32];
+  constexpr int kNone = 0x7fffffff;
+  const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int words = (Ck + 31) >> 5;
+  for (int w = tid; w < words; w += kKeepThreads) row_s[w] = 0u;
+  const bool live_row = nq[static_cast<size_t>(bh) * Cq + i] > 0;
+  const float* qi = cq + (static_cast<size_t>(bh) * Cq + i) * D;
+  const int32_t* nkh = nk + static_cast<size_t>(bh) * Ck;
+  double lmax = -INFINITY;
+  for (int j = tid; j < n2; j += kKeepThreads) {
+    double s = -1.0;
+    int id = kNone;
+    if (live_row && j < Ck && nkh[j] > 0) {
+      const float* kj = ck + (static_cast<size_t>(bh) * Ck + j) * D;
+      double acc = 0.0;
+      for (int x = 0; x < D; ++x) acc = __fma_rn(static_cast<double>(qi[x]), static_cast<double>(kj[x]), acc);
+      s = __dmul_rn(scale, acc);
+      id = j;
+      lmax = fmax(lmax, s);
+    }
+    ks_w[j] = s;
+    ks_i[j] = id;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
+  if ((tid & 31) == 0) red[tid >> 5] = lmax;
+  __syncthreads();
+  double m = red[0];
+#pragma unroll
+  for (int w = 1; w < kKeepThreads / 32; ++w) m = fmax(m, red[w]);
+  for (int j = tid; j < n2; j += kKeepThreads) {
+    if (ks_i[j] != kNone)
+      ks_w[j] = __dmul_rn(static_cast<double>(nkh[ks_i[j]]), exp_neg(__dsub_rn(ks_w[j], m)));
+    else
+      ks_w[j] = -1.0;  // below every weight (weights are >= 0)
+  }
+  __syncthreads();
+  // bitonic sort: weight descending, then cluster index ascending
+  for (int k = 2; k <= n2; k <<= 1)
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int e = tid; e < n2; e += kKeepThreads) {
+        const int p = e ^ jj;
+        if (p > e) {
+          const double wa = ks_w[e], wb = ks_w[p];
+          const int ia = ks_i[e], ib = ks_i[p];
+          const bool a_first = wa > wb || (wa == wb && ia < ib);
+          const bool up = (e & k) == 0;
+          if (up != a_first) {
+            ks_w[e] = wb;
+            ks_w[p] = wa;
+            ks_i[e] = ib;
+            ks_i[p] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  if (tid == 0 && live_row) {
+    double total = 0.0;
+    int live = 0;
+    while (live < n2 && ks_i[live] != kNone) total = __dadd_rn(total, ks_w[live++]);
+    const double target = __dmul_rn(top_p, total);
+    double cum = 0.0;
+    for (int e = 0; e < live; ++e) {
+      const int j = ks_i[e];
+      row_s[j >> 5] |= 1u << (j & 31);
+      cum = __dadd_rn(cum, ks_w[e]);
+      if (cum >= target) break;
+    }
+  }
+  __syncthreads();
+  uint32_t* krow = keep + (static_cast<size_t>(bh) * Cq + i) * words;
+  for (int w = tid; w < words; w += kKeepThreads) krow[w] = row_s[w];
+}
+
+// ---------------------------------------------------------------------------------------
+// block mask over the cluster-major layouts
+// ---------------------------------------------------------------------------------------
+
+// Cluster of the first and last slot of every block: in a cluster-major layout the clusters
+// present in a block are exactly the non-empty ones between these two.
+__global__ void block_cluster_range_kernel(const int32_t* __restrict__ label, const int32_t* __restrict__ perm,
+                                           int N, int block, int nblk, int C, int2* __restrict__ range, int* err) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x, bh = blockIdx.y;
+  if (b >= nblk) return;
+  const int s0 = b * block, s1 = min(N, (b + 1) * block) - 1;
+  const int32_t* ph = perm + static_cast<size_t>(bh) * N;
+  const int32_t* lh = label + static_cast<size_t>(bh) * N;
+  const int t0 = ph[s0], t1 = ph[s1];
+  int2 r = make_int2(0, -1);  // empty range
+  if (t0 >= 0 && t0 < N && t1 >= 0 && t1 < N) {
+    const int l0 = lh[t0], l1 = lh[t1];
+    if (l0 >= 0 && l0 <= l1 && l1 < C) r = make_int2(l0, l1);
+    else atomicOr(err, kDevErrKvRange);
+  } else {
+    atomicOr(err, kDevErrKvRange);
+  }
+  range[static_cast<size_t>(bh) * nblk + b] = r;
+}
+
+__device__ __forceinline__ bool any_bit_in_range(const uint32_t* bits, int lo, int hi) {
+  for (int w = lo >> 5; w <= (hi >> 5); ++w) {
+    uint32_t m = bits[w];
+    if (w == (lo >> 5)) m &= ~0u << (lo & 31);
+    if (w == (hi >> 5) && (hi & 31) != 31) m &= (1u << ((hi & 31) + 1)) - 1u;
+    if (m) return true;
+  }
+  return false;
+}
+
+// One warp per (head, query block): the key clusters reachable from the block's query
+// clusters, then every key block tested against its cluster range.
+__global__ void __launch_bounds__(32) semantic_block_mask_kernel(
+    const int2* __restrict__ qrange, const int2* __restrict__ krange, const int32_t* __restrict__ nq, int Cq,
+    const int32_t* __restrict__ nk, int Ck, const uint32_t* __restrict__ keep, int nblk, uint32_t* __restrict__ bits,
+    int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, int max_kv, int* err) {
+  __shared__ uint32_t reach[kMaxClusters / 32];
+  const int bq = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+  const int words = (Ck + 31) >> 5, nwb = (nblk + 31) >> 5;
+  const int2 qr = qrange[static_cast<size_t>(bh) * nblk + bq];
+  uint32_t acc = 0u;
+  for (int i = qr.x; i <= qr.y; ++i) {
+    if (nq[static_cast<size_t>(bh) * Cq + i] <= 0) continue;
+    if (lane < words) acc |= keep[(static_cast<size_t>(bh) * Cq + i) * words + lane];
+  }
+  if (lane < words) {
+    uint32_t ne = 0u;
+    for (int b = 0; b < 32; ++b) {
+      const int j = lane * 32 + b;
+      if (j < Ck && nk[static_cast<size_t>(bh) * Ck + j] > 0) ne |= 1u << b;
+    }
+    reach[lane] = acc & ne;
+  }
+  __syncwarp();
+  const size_t row = static_cast<size_t>(bh) * nblk + bq;
+  const unsigned lt = (1u << lane) - 1u;
+  int cnt = 0;
+  for (int b0 = 0; b0 < nblk; b0 += 32) {
+    const int bk = b0 + lane;
+    bool kept = false;
+    if (bk < nblk) {
+      const int2 kr = krange[static_cast<size_t>(bh) * nblk + bk];
+      kept = kr.x <= kr.y && any_bit_in_range(reach, kr.x, kr.y);
+    }
+    const unsigned ball = __ballot_sync(0xffffffffu, kept);
+    if (lane == 0) bits[row * nwb + (b0 >> 5)] = ball;
+    const int pos = cnt + __popc(ball & lt);
+    if (kept && pos < max_kv) kv_idx[row * max_kv + pos] = bk;
+    cnt += __popc(ball);
+  }
+  if (lane == 0) {
+    if (cnt > max_kv) atomicOr(err, kDevErrOverflow);
+    kv_cnt[row] = min(cnt, max_kv);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// row gather / scatter through a per-head permutation (16-byte vectors)
+// ---------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(const uint4* __restrict__ src,
+                                                                  const int32_t* __restrict__ perm,
+                                                                  uint4* __restrict__ dst, int N, int vpr, int* err) {
+  const int bh = blockIdx.y;
+  const size_t total = static_cast<size_t>(N) * vpr;
+  const size_t head = static_cast<size_t>(bh) * total;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * kRowThreads + threadIdx.x; e < total;
+       e += static_cast<size_t>(gridDim.x) * kRowThreads) {
+    const int s = static_cast<int>(e / vpr), v = static_cast<int>(e - static_cast<size_t>(s) * vpr);
+    const int t = perm[static_cast<size_t>(bh) * N + s];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0 && t < N) val = src[head + static_cast<size_t>(t) * vpr + v];
+    else if (v == 0) atomicOr(err, kDevErrKvRange);
+    dst[head + e] = val;
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(const uint4* __restrict__ src,
+                                                                   const float* __restrict__ src_lse,
+                                                                   const int32_t* __restrict__ perm,
+                                                                   uint4* __restrict__ dst, float* __restrict__ dst_lse,
+                                                                   int N, int vpr, int* err) {
+  const int bh = blockIdx.y;
+  const size_t total = static_cast<size_t>(N) * vpr;
+  const size_t head = static_cast<size_t>(bh) * total;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * kRowThreads + threadIdx.x; e < total;
+       e += static_cast<size_t>(gridDim.x) * kRowThreads) {
+    const int s = static_cast<int>(e / vpr), v = static_cast<int>(e - static_cast<size_t>(s) * vpr);
+    const int t = perm[static_cast<size_t>(bh) * N + s];
+    if (t < 0 || t >= N) {
+      if (v == 0) atomicOr(err, kDevErrKvRange);
+      continue;
+    }
+    dst[head + static_cast<size_t>(t) * vpr + v] = src[head + e];
+    if (v == 0 && dst_lse != nullptr)
+      dst_lse[static_cast<size_t>(bh) * N + t] = src_lse[static_cast<size_t>(bh) * N + s];
+  }
+}
+
+int rows_grid_x(int N, int vpr, int BH) {
+  const long long want = (static_cast<long long>(N) * vpr + kRowThreads - 1) / kRowThreads;
+  const long long cap = (148LL * 16 + BH - 1) / BH;
+  return static_cast<int>(want < cap ? want : cap);
+}
+
+template <int D>
+cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, float* cent, int32_t* label,
+                     int32_t* counts, int32_t* perm, int32_t* offsets, float* cnorm, int* err, cudaStream_t stream) {
+  constexpr size_t smem = assign_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const size_t ssmem = sizeof(int) * (kSortWarps + 1) * static_cast<size_t>(C);
+  if (ssmem > 48 * 1024) {
+    e = cudaFuncSetAttribute(kmeans_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem));
+    if (e != cudaSuccess) return e;
+  }
+  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, cnorm);
+  constexpr size_t usmem = update_smem_bytes<D>();
+  e = cudaFuncSetAttribute(kmeans_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(usmem));
+  if (e != cudaSuccess) return e;
+  const dim3 agrid((N + kKmTile - 1) / kKmTile, BH), ugrid(C, BH);
+  for (int it = 0; it < iters; ++it) {
+    kmeans_assign_kernel<D><<<agrid, kKmThreads, smem, stream>>>(x, N, C, cent, cnorm, label);
+    kmeans_sort_kernel<<<BH, kSortWarps * 32, ssmem, stream>>>(label, N, C, counts, offsets, perm, err);
+    kmeans_update_kernel<D><<<ugrid, kUpdThreads, usmem, stream>>>(x, N, C, counts, offsets, perm, cent, cnorm);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t kmeans_workspace_bytes(int BH, int C) {
+  const size_t offs = (static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  return offs + ((static_cast<size_t>(BH) * C * sizeof(float) + 255) & ~static_cast<size_t>(255));
+}
+
+cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
+                          int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream) {
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  int32_t* offsets = static_cast<int32_t*>(ws);
+  const size_t offs = (static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  float* cnorm = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + offs);
+  if (d == 128) return kmeans_d<128>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, err, stream);
+  if (d == 64) return kmeans_d<64>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, err, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_semantic_mask(const float* cent_q, const int32_t* counts_q, const int32_t* label_q,
+                                 const int32_t* perm_q, int Cq, const float* cent_k, const int32_t* counts_k,
+                                 const int32_t* label_k, const int32_t* perm_k, int Ck, int BH, int N, int d,
+                                 int block, double scale, double top_p, uint32_t* keep, uint32_t* bits,
+                                 int32_t* kv_idx, int32_t* kv_cnt, int max_kv, void* ws, int* err,
+                                 cudaStream_t stream) {
+  const int nblk = (N + block - 1) / block;
+  int n2 = 1;
+  while (n2 < Ck) n2 <<= 1;
+  const size_t ksmem = static_cast<size_t>(n2) * (sizeof(double) + sizeof(int));
+  semantic_keep_kernel<<<dim3(Cq, BH), kKeepThreads, ksmem, stream>>>(cent_q, counts_q, Cq, cent_k, counts_k, Ck,
+                                                                      d, scale, top_p, n2, keep);
+  int2* qr = static_cast<int2*>(ws);
+  int2* kr = qr + static_cast<size_t>(BH) * nblk;
+  const dim3 rgrid((nblk + 127) / 128, BH);
+  block_cluster_range_kernel<<<rgrid, 128, 0, stream>>>(label_q, perm_q, N, block, nblk, Cq, qr, err);
+  block_cluster_range_kernel<<<rgrid, 128, 0, stream>>>(label_k, perm_k, N, block, nblk, Ck, kr, err);
+  semantic_block_mask_kernel<<<dim3(nblk, BH), 32, 0, stream>>>(qr, kr, counts_q, Cq, counts_k, Ck, keep, nblk, bits,
+                                                                kv_idx, kv_cnt, max_kv, err);
+  return cudaGetLastError();
+}
+
+size_t semantic_mask_workspace_bytes(int BH, int N, int block) {
+  const size_t nblk = (static_cast<size_t>(N) + block - 1) / block;
+  return 2 * static_cast<size_t>(BH) * nblk * sizeof(int2);
+}
+
+cudaError_t launch_gather_rows(const void* src, const int32_t* perm, void* dst, int BH, int N, int d, int* err,
+                               cudaStream_t stream) {
+  const int vpr = d * 2 / 16;
+  gather_rows_kernel<<<dim3(rows_grid_x(N, vpr, BH), BH), kRowThreads, 0, stream>>>(
+      static_cast<const uint4*>(src), perm, static_cast<uint4*>(dst), N, vpr, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void* src, const float* src_lse, const int32_t* perm, void* dst, float* dst_lse,
+                                int BH, int N, int d, int* err, cudaStream_t stream) {
+  const int vpr = d * 2 / 16;
+  scatter_rows_kernel<<<dim3(rows_grid_x(N, vpr, BH), BH), kRowThreads, 0, stream>>>(
+      static_cast<const uint4*>(src), src_lse, perm, static_cast<uint4*>(dst), dst_lse, N, vpr, err);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

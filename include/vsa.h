@@ -23,6 +23,15 @@
  *   vsa_unpermute       scatter the output back to natural order
  *   vsa_attention       all of the above on one stream
  *
+ * A second way to choose the kept blocks, the semantic-aware permutation ("Sparse
+ * VideoGen2" page, abstract), runs on the same attention kernel:
+ *
+ *   vsa_kmeans          per-head k-means of Q (or K) and the cluster-major order
+ *   vsa_gather_rows     rows in a per-head order (Q by its clusters, K and V by theirs)
+ *   vsa_semantic_mask   top-p budget over cluster pairs -> block mask of the two layouts
+ *   vsa_scatter_rows    the output back to token order
+ *   vsa_semantic_attention  all of them with vsa_sparse_attn_fwd on one stream
+ *
  * Conventions
  *   - Tensors are [B, H, rows, d] row-major (d fastest), bf16 unless stated otherwise.
  *     A head's buffer holds N rows in natural or frame-major order, or C*V rows in
@@ -248,7 +257,9 @@ VSA_API vsa_status vsa_block_order(const uint8_t *d_kind, const int32_t *d_kv_id
  * key gets O = 0 and LSE = -inf.
  *   natural   q, k, v, o, lse of spatial heads ([B, H, N, d], natural order)
  *   permuted  q, k, v, o, lse of temporal and cube heads ([B, H, R, d]); may be NULL,
- *             in which case every head uses `natural`
+ *             in which case every head uses `natural`.  The kernel reads a VSA_TEMPORAL
+ *             head's N rows from here whatever order they are in (vsa_semantic_attention
+ *             passes its cluster-major rows this way)
  *   d_kind    [B*H] head kinds; d_kv_idx / d_kv_cnt from vsa_build_mask (each list strictly
  *             ascending; a malformed list sets VSA_DEVERR_KV_RANGE and its rows are zero)
  *   d_order   NULL (query blocks paired as 2i, 2i+1) or the [B, H, nblk] permutation from
@@ -292,6 +303,95 @@ VSA_API vsa_status vsa_attention(const vsa_qkvo *io, vsa_dtype dtype, const vsa_
 VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const vsa_params *params, vsa_dtype dtype,
                                           vsa_select select, size_t *off_bits, size_t *off_kv_idx,
                                           size_t *off_kv_cnt, int *max_kv);
+
+/* ---------------------------------------------------------------------------------------
+ * Semantic-aware permutation ("Sparse VideoGen2" page, abstract: tokens clustered by
+ * k-means and reordered by cluster, a top-p budget over clusters).  The page gives no
+ * formulas; the readings:
+ *   - Lloyd's k-means per head on the bf16 rows (as fp32), `iters` rounds of assignment then
+ *     update, starting from the rows floor((2j+1) N / (2C)), j < C;
+ *   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32, both dot products summed in dimension
+ *     order with one fused multiply-add per term, ties to the smaller j;
+ *   - update: fp64 sum of the members in token order / count, rounded to fp32; an empty
+ *     cluster keeps its centroid;
+ *   - cluster-major order: slots sorted by (cluster, token);
+ *   - weight of key cluster j for query cluster i: n_j exp(s_ij - max_j s_ij), s_ij =
+ *     scale * cq_i . ck_j in fp64; kept: the shortest prefix of the weights in descending
+ *     order (ties to the smaller j) whose running sum reaches top_p of their total;
+ *   - block pair (a, b) of the query and key layouts is kept when some query slot of a and
+ *     some key slot of b belong to a kept cluster pair.
+ * These entry points take shapes without cube dims (VSA_ERR_UNSUPPORTED otherwise), bf16
+ * rows, 1 <= C <= min(N, 1024) clusters and 1 <= iters <= 1000.
+ * ------------------------------------------------------------------------------------- */
+
+/* Scratch bytes of vsa_kmeans (cluster offsets and centroid norms); 0 for an invalid shape or
+ * count. */
+VSA_API size_t vsa_kmeans_workspace_size(const vsa_shape *shape, int n_clusters);
+
+/*
+ * k-means of x and its cluster-major order.
+ *   x            [B, H, N, d] bf16, natural order (device)
+ *   d_centroids  [B*H, C, d] fp32 out: centroids after the last update (16-byte aligned)
+ *   d_labels     [B*H, N] int32 out: cluster of every token (last assignment)
+ *   d_counts     [B*H, C] int32 out: members per cluster
+ *   d_perm       [B*H, N] int32 out: token at each slot of the cluster-major order
+ *   ws           vsa_kmeans_workspace_size bytes of scratch
+ */
+VSA_API vsa_status vsa_kmeans(const void *x, const vsa_shape *shape, int n_clusters, int iters, float *d_centroids,
+                              int32_t *d_labels, int32_t *d_counts, int32_t *d_perm, void *ws, size_t ws_bytes,
+                              int *d_err, cudaStream_t stream);
+
+/* Scratch bytes of vsa_semantic_mask (the cluster range of every block). */
+VSA_API size_t vsa_semantic_mask_workspace_size(const vsa_shape *shape);
+
+/*
+ * Top-p cluster budget and the block mask over the two cluster-major layouts.
+ *   d_cent_*, d_counts_*, d_labels_*, d_perm_*  vsa_kmeans outputs of Q (cq clusters) and K
+ *   top_p        in (0, 1];  scale  the score scale, 0 selects 1/sqrt(d) (fp64)
+ *   d_keep       [B*H, cq, ceil(ck/32)] uint32 out: bit j of row i set when key cluster j
+ *                is kept for query cluster i
+ *   d_bits, d_kv_idx, d_kv_cnt  as vsa_build_mask writes them, with nblk = ceil(N/block)
+ *                blocks of the query layout (rows) and of the key layout (columns); a row
+ *                keeping more than max_kv blocks sets VSA_DEVERR_OVERFLOW
+ *   ws           vsa_semantic_mask_workspace_size bytes of scratch
+ * Labels or orders out of range set VSA_DEVERR_KV_RANGE.
+ */
+VSA_API vsa_status vsa_semantic_mask(const float *d_cent_q, const int32_t *d_counts_q, const int32_t *d_labels_q,
+                                     const int32_t *d_perm_q, int cq, const float *d_cent_k, const int32_t *d_counts_k,
+                                     const int32_t *d_labels_k, const int32_t *d_perm_k, int ck,
+                                     const vsa_shape *shape, float top_p, float scale, uint32_t *d_keep,
+                                     uint32_t *d_bits, int32_t *d_kv_idx, int32_t *d_kv_cnt, int max_kv, void *ws,
+                                     size_t ws_bytes, int *d_err, cudaStream_t stream);
+
+/* dst[b, h, s] = src[b, h, d_perm[b*H + h, s]] for [B, H, N, d] bf16 rows.  An order entry
+ * outside [0, N) sets VSA_DEVERR_KV_RANGE and that row is written as zeros. */
+VSA_API vsa_status vsa_gather_rows(const void *src, const int32_t *d_perm, void *dst, const vsa_shape *shape,
+                                   int *d_err, cudaStream_t stream);
+
+/* dst[b, h, d_perm[b*H + h, s]] = src[b, h, s] (and the same for the fp32 LSE when both
+ * src_lse and dst_lse are given).  An order entry outside [0, N) sets VSA_DEVERR_KV_RANGE. */
+VSA_API vsa_status vsa_scatter_rows(const void *src, const float *src_lse, const int32_t *d_perm, void *dst,
+                                    float *dst_lse, const vsa_shape *shape, int *d_err, cudaStream_t stream);
+
+typedef struct {
+    int cq, ck;    /* clusters of Q and of K per head */
+    int iters;     /* k-means rounds */
+    float top_p;   /* budget, in (0, 1] */
+    float scale;   /* softmax and score scale, 0 selects 1/sqrt(d) */
+} vsa_semantic_params;
+
+VSA_API size_t vsa_semantic_workspace_size(const vsa_shape *shape, const vsa_semantic_params *params);
+
+/*
+ * The whole semantic call on `stream`: vsa_kmeans of Q and of K, vsa_gather_rows (Q by the
+ * query order, K and V by the key order), vsa_semantic_mask, vsa_sparse_attn_fwd with every
+ * head read from the permuted rows, vsa_scatter_rows of O (and LSE) through the query order.
+ *   io   natural q, k, v, o bf16 [B, H, N, d]; lse fp32 [B, H, N] or NULL
+ *   ws   vsa_semantic_workspace_size bytes (clusters, orders, masks and permuted rows)
+ */
+VSA_API vsa_status vsa_semantic_attention(const vsa_qkvo *io, const vsa_shape *shape,
+                                          const vsa_semantic_params *params, void *ws, size_t ws_bytes, int *d_err,
+                                          cudaStream_t stream);
 
 /* Self-test hook (the pages have no counterpart): evaluates the kernels' two base-2
  * exponentials, the FMA-pipe polynomial (y_poly) and the hardware approximation (y_mufu),

@@ -47,7 +47,7 @@ class Workload:
     d: int
     block: int
     dtype: str                       # "f32" or "bf16"
-    mode: str                        # "fixed", "profiled" or "cube"
+    mode: str                        # "fixed", "profiled", "cube" or "semantic"
     target: Optional[float] = None   # kept-block fraction the windows must reach
     w_s: Optional[int] = None        # fixed windows (mode "fixed")
     w_t: Optional[int] = None
@@ -57,6 +57,9 @@ class Workload:
     profile_frac: float = 0.01
     structure_scale: float = 2.0
     seed: int = 0
+    clusters: tuple = (128, 128)     # k-means clusters of Q and of K (mode "semantic")
+    kmeans_iters: int = 4
+    top_p: float = 0.6
 
     @property
     def S(self) -> int:
@@ -87,6 +90,8 @@ HUNYUAN = Workload("hunyuanvideo-720p: B1 H24 33x45x80 d128 block128 bf16", 1, 2
                    "bf16", "profiled", target=0.18)
 WAN_6X = Workload("wan2.1-1.3b 6x horizon: B1 H12 126x30x52 d128 cubes 4x4x8 top-32", 1, 12, 126, 30, 52,
                   128, 128, "bf16", "cube", topk=32)
+WAN_SEMANTIC = Workload("wan2.1-1.3b semantic: B1 H12 21x30x52 d128 block128 bf16, k-means 128/128 x4, top-p 0.6",
+                        1, 12, 21, 30, 52, 128, 128, "bf16", "semantic")
 SWEEP_TARGETS = (1.0, 0.35, 0.18, 0.13, 0.05)
 
 
@@ -94,7 +99,7 @@ def sweep(target: float) -> Workload:
     return WAN.with_(name=f"sparsity sweep kept={target}: B1 H12 21x30x52 d128 block128 bf16", target=target)
 
 
-WORKLOADS = {"tiny": TINY, "wan": WAN, "hunyuan": HUNYUAN, "wan6x": WAN_6X}
+WORKLOADS = {"tiny": TINY, "wan": WAN, "hunyuan": HUNYUAN, "wan6x": WAN_6X, "wan-semantic": WAN_SEMANTIC}
 for _t in SWEEP_TARGETS:
     WORKLOADS[f"sweep{_t}"] = sweep(_t)
 
@@ -152,5 +157,5 @@ def human(wl: Workload) -> str:
     return f"{wl.name} (N={wl.N})"
 
 
-__all__ = ["Workload", "WORKLOADS", "TINY", "WAN", "HUNYUAN", "WAN_6X", "SWEEP_TARGETS", "sweep",
+__all__ = ["Workload", "WORKLOADS", "TINY", "WAN", "HUNYUAN", "WAN_6X", "WAN_SEMANTIC", "SWEEP_TARGETS", "sweep",
            "make_qkv", "make_random", "sample_indices", "dense_flops", "SPATIAL", "TEMPORAL", "CUBE"]

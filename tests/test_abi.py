@@ -158,3 +158,50 @@ def test_workspace_sizes_monotone():
     ob, oi, oc, mk = _lib.vsa_attention_workspace_layout(shape, p, 1, 1)
     assert ob == 0 and oi > ob and oc > oi and mk == _lib.vsa_max_kv(shape, p)
     assert np.all(np.array([ob, oi, oc]) % 256 == 0)
+
+
+def test_semantic_entry_points_validate_before_launch():
+    """Semantic-permutation entry points: bad counts, budgets, shapes, workspaces and
+    pointer pairs are refused on the host, and the workspace sizes follow the documented
+    layout."""
+    lib = _lib.lib
+    s = ctypes.c_void_p(0)
+    shape = _lib.make_shape(1, 2, 4, 8, 8, 64, 64)          # N = 256
+    cube = _lib.make_shape(1, 2, 8, 8, 8, 64, 128, (4, 4, 8))
+    # offsets B*H*(C+1) int32 and norms B*H*C fp32, each 256-aligned
+    assert _lib.vsa_kmeans_workspace_size(shape, 16) == 256 + 256
+    assert _lib.vsa_kmeans_workspace_size(shape, 64) == 768 + 512
+    assert _lib.vsa_kmeans_workspace_size(shape, 0) == 0
+    assert _lib.vsa_kmeans_workspace_size(shape, 257) == 0   # more clusters than rows
+    assert _lib.vsa_kmeans_workspace_size(cube, 16) == 0
+    km = lambda sh, C, it, wsb: lib.vsa_kmeans(FAKE, ctypes.byref(sh), C, it, FAKE, FAKE, FAKE, FAKE, FAKE, wsb,  # noqa
+                                               FAKE, s)
+    assert km(shape, 0, 1, 1 << 20) == _lib.VSA_ERR_INVALID_ARG
+    assert km(shape, 1025, 1, 1 << 20) == _lib.VSA_ERR_INVALID_ARG
+    assert km(shape, 16, 0, 1 << 20) == _lib.VSA_ERR_INVALID_ARG
+    assert km(shape, 16, 3, 8) == _lib.VSA_ERR_WORKSPACE
+    assert km(cube, 16, 3, 1 << 20) == _lib.VSA_ERR_UNSUPPORTED
+    assert lib.vsa_kmeans(FAKE + 8, ctypes.byref(shape), 16, 3, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, FAKE,
+                          s) == _lib.VSA_ERR_INVALID_ARG       # misaligned rows
+
+    def mask(top_p, scale=0.0, cq=16, ck=16, wsb=1 << 20, max_kv=4):
+        return lib.vsa_semantic_mask(FAKE, FAKE, FAKE, FAKE, cq, FAKE, FAKE, FAKE, FAKE, ck, ctypes.byref(shape),
+                                     top_p, scale, FAKE, FAKE, FAKE, FAKE, max_kv, FAKE, wsb, FAKE, s)
+    assert mask(0.0) == _lib.VSA_ERR_INVALID_ARG
+    assert mask(1.5) == _lib.VSA_ERR_INVALID_ARG
+    assert mask(0.5, scale=-1.0) == _lib.VSA_ERR_INVALID_ARG
+    assert mask(0.5, ck=2000) == _lib.VSA_ERR_INVALID_ARG
+    assert mask(0.5, max_kv=0) == _lib.VSA_ERR_INVALID_ARG
+    assert mask(0.5, wsb=8) == _lib.VSA_ERR_WORKSPACE
+    assert _lib.vsa_semantic_mask_workspace_size(shape) == 256   # 2 * B*H * nblk int2, 256-aligned
+    assert lib.vsa_scatter_rows(FAKE, FAKE, FAKE, FAKE, None, ctypes.byref(shape), FAKE, s) == \
+        _lib.VSA_ERR_INVALID_ARG                                    # LSE needs both buffers
+    assert lib.vsa_gather_rows(FAKE, FAKE, FAKE, ctypes.byref(cube), FAKE, s) == _lib.VSA_ERR_UNSUPPORTED
+    good = _lib.make_sem_params(16, 16, 3, 0.5)
+    assert _lib.vsa_semantic_workspace_size(shape, good) > 0
+    for bad in (_lib.make_sem_params(0, 16, 3, 0.5), _lib.make_sem_params(16, 16, 0, 0.5),
+                _lib.make_sem_params(16, 16, 3, 0.0), _lib.make_sem_params(16, 16, 3, 0.5, -1.0)):
+        assert _lib.vsa_semantic_workspace_size(shape, bad) == 0
+    io = _lib.QKVO(FAKE, FAKE, FAKE, FAKE, None)
+    assert lib.vsa_semantic_attention(ctypes.byref(io), ctypes.byref(shape), ctypes.byref(good), FAKE, 8, FAKE,
+                                      s) == _lib.VSA_ERR_WORKSPACE
