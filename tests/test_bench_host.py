@@ -36,3 +36,55 @@ def test_clock_summary_reports_throttle_reasons():
 def test_clock_summary_without_samples():
     out = _sampler([], 1.0, 2.0).summary()
     assert out["samples"] == 0 and out["sm_mhz"] is None and out["reasons"] == ["unavailable"]
+
+
+# ---------------------------------------------------------------------------------------
+# work accounting: the figures the bench divides by time
+# ---------------------------------------------------------------------------------------
+
+import types  # noqa: E402
+
+import numpy as np  # noqa: E402
+
+import oracle  # noqa: E402
+import synthetic  # noqa: E402
+
+
+def test_attention_work_is_the_allowed_token_pairs():
+    """Algorithmic flops = 4·d per allowed (query, key) token pair, counted here from the
+    oracle's block mask at token level (ragged last block, spatial and temporal heads)."""
+    wl = synthetic.WAN.with_(H=2, F=3, Hl=5, Wl=20)          # N = 300: blocks of 128, 128, 44
+    nb = 3
+    keeps = [np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]], bool), np.ones((nb, nb), bool)]
+    kinds = [oracle.SPATIAL, oracle.TEMPORAL]
+    idx = np.full((1, 2, nb, nb), -1, np.int32)
+    cnt = np.zeros((1, 2, nb), np.int32)
+    for h in range(2):
+        i_, c_ = oracle.keep_to_lists(keeps[h], nb)
+        idx[0, h], cnt[0, h] = i_, c_
+    alg, exe, pairs = bench.attention_work(wl, np.array(kinds), idx, cnt)
+    want = 0
+    for h, kind in enumerate(kinds):
+        blk = oracle.layout_slots(kind, wl.F, wl.Hl, wl.Wl) // wl.block
+        want += int(keeps[h][blk[:, None], blk[None, :]].sum())
+    assert alg == 4.0 * wl.d * want
+    assert pairs == int(sum(k.sum() for k in keeps))
+    assert exe == 4.0 * wl.d * 128 * 128 * pairs
+
+
+def test_semantic_stage_work():
+    """k-means: 2·d flop per (row, centroid) pair per round for Q and K; gathers read and
+    write Q, K, V; the scatter reads and writes O."""
+    wl = synthetic.WAN_SEMANTIC
+    pipe = types.SimpleNamespace(nblk=256, max_kv=256)
+    work, exp2 = bench.stage_work(wl, [1] * wl.H, pipe, pairs=1000)
+    row = wl.d * 2
+    assert work["profile"]["flops"] == wl.H * wl.kmeans_iters * 2 * wl.d * wl.N * sum(wl.clusters)
+    assert work["permute"]["bytes"] == wl.H * 3 * 2 * wl.N * row
+    assert work["unpermute"]["bytes"] == wl.H * 2 * wl.N * row
+    assert work["mask"]["bytes"] == wl.H * 256 * (8 + 256 + 1) * 4
+    assert exp2 == 1000 * 128 * 128
+    roof = bench.stage_roofline(work, {"profile": 4.0, "permute": 0.1, "mask": 0.2, "unpermute": 0.05}, 6538.3,
+                                1631.1)
+    assert roof["profile"]["bound"] == "alu" and abs(roof["profile"]["peak"] - bench.FP32_PEAK_TFLOPS) < 1e-9
+    assert abs(roof["permute"]["achieved"] - work["permute"]["bytes"] / 1e-4 / 1e9) < 1e-6
