@@ -4,9 +4,10 @@ One step = the whole hot path on one batch of synthetic input resident in HBM:
 profiling -> frame-major permutation of Q/K/V -> block masks -> block-sparse attention
 -> un-permutation of O, each through its C-ABI entry point on one stream, with CUDA events
 between the stages for the per-kernel timing.  The default workload is the Wan2.1-1.3B
-latent grid (B1 H12 21x30x52, d 128, block 128, kept fraction 0.18, profiled heads).
+latent grid of HunyuanVideo-720p (B1 H24 33x45x80, d 128, block 128, kept fraction 0.18,
+profiled heads), the largest single-GPU workload by work and bytes.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan|hunyuan|wan6x|tiny|sweep0.35...]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config hunyuan|wan|wan6x|sweep0.35|...]
     python bench.py --impl reference ...   (the fp64 CPU oracle timed on host cores)
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent attention call
@@ -90,6 +91,34 @@ def attention_work(wl, kinds, kv_idx, kv_cnt):
     return alg, exe, pairs
 
 
+def kept_block_run(i, n, block, group, w):
+    """Kept key blocks [lo, hi] of query block i under the window rule: block j spans groups
+    [a_j, b_j] = [j*block // group, (min(n, (j+1)*block) - 1) // group] and is kept when the
+    two spans are at most w groups apart."""
+    nb = -(-n // block)
+    j = np.arange(nb)
+    a = (j * block) // group
+    b = (np.minimum(n, (j + 1) * block) - 1) // group
+    keep = np.maximum(0, np.maximum(a - b[i], a[i] - b)) <= w
+    idx = np.nonzero(keep)[0]
+    return int(idx[0]), int(idx[-1])
+
+
+def profile_allowed_keys(wl, r, w_s, w_t):
+    """Sum over the r sampled rows rho_i = floor((2i+1)N/(2r)) of the keys each pattern allows
+    (spatial: natural blocks, group = frame; temporal: frame-major blocks, group = position)."""
+    N, B, F, S = wl.N, wl.block, wl.F, wl.S
+    total = 0
+    for i in range(r):
+        t = ((2 * i + 1) * N) // (2 * r)
+        lo, hi = kept_block_run(t // B, N, B, S, w_s)
+        total += min(N, (hi + 1) * B) - lo * B
+        p = (t % S) * F + t // S  # frame-major slot
+        lo, hi = kept_block_run(p // B, N, B, F, w_t)
+        total += min(N, (hi + 1) * B) - lo * B
+    return float(total)
+
+
 def stage_work(wl, kinds, pipe, pairs):
     """Algorithmic bytes (HBM stages) or executed flops (profiling) per call of each stage,
     and the number of exponentials the attention evaluates."""
@@ -126,15 +155,15 @@ def stage_work(wl, kinds, pipe, pairs):
            "mask": {"bytes": mask, "bound": "hbm"}}
     if wl.mode == "profiled":
         r = _lib.vsa_profile_rows(pipe.shape, pipe.params)
-        # tensor work of the profiling kernel: Q.K^T once and three P.V over all N keys
-        out["profile"] = {"flops": BH * 8.0 * d * r * N, "bound": "tensor", "rows": r}
+        # algorithmic work of profiling: per head the dense part (Q.K^T and P.V over all N keys,
+        # 4*d*r*N) plus one P.V per pattern over the keys that pattern allows each sampled row
+        allowed = profile_allowed_keys(wl, r, pipe.params.w_s, pipe.params.w_t)
+        alg = BH * (4.0 * d * r * N + 2.0 * d * allowed)
+        # executed: Q.K^T once and three full-width P.V (the masked ones lane-masked)
+        out["profile"] = {"flops": alg, "executed_flops": BH * 8.0 * d * r * N, "bound": "tensor", "rows": r,
+                          "allowed_keys_per_head": allowed}
     exp2 = float(pairs) * 128 * wl.block
     return out, exp2
-
-
-# fp32 FMA peak of the CUDA cores (not measured): 148 SMs x 128 lanes x 2 flops at the maximum
-# SM clock (1965 MHz); the k-means assignment runs there, not on the tensor cores
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
@@ -144,10 +173,10 @@ def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
         if t <= 0 or w.get("bytes", 1) == 0:
             continue
         if w["bound"] == "fp32":
+            # no measured fp32 FMA peak exists for this machine, so no fraction is reported
             tf = w["flops"] / t / 1e12
-            out[name] = {"bound": "alu", "flops": w["flops"], "achieved": tf, "peak": FP32_PEAK_TFLOPS,
-                         "unit": "TFLOP/s", "frac": tf / FP32_PEAK_TFLOPS,
-                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"}
+            out[name] = {"bound": "alu", "flops": w["flops"], "achieved": tf, "peak": None, "unit": "TFLOP/s",
+                         "frac": None}
         elif w["bound"] == "hbm":
             gbs = w["bytes"] / t / 1e9
             out[name] = {"bound": "hbm", "bytes": w["bytes"], "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
@@ -156,6 +185,9 @@ def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
             tf = w["flops"] / t / 1e12
             out[name] = {"bound": "tensor", "flops": w["flops"], "achieved": tf, "peak": tensor_tflops,
                          "unit": "TFLOP/s", "frac": tf / tensor_tflops}
+            if "executed_flops" in w:
+                out[name]["executed_flops"] = w["executed_flops"]
+                out[name]["executed_frac"] = w["executed_flops"] / t / 1e12 / tensor_tflops
     return out
 
 
@@ -610,7 +642,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="wan")
+    ap.add_argument("--config", default="hunyuan")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

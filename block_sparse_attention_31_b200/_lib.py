@@ -91,6 +91,7 @@ def _load():
         "vsa_semantic_attention": (st, [P(QKVO), P(Shape), P(SemParams), vp, sz, vp, vp]),
         "vsa_selftest_exp2": (st, [vp, vp, vp, i32, vp]),
         "vsa_selftest_wait_timeout": (st, [vp, vp, vp]),
+        "vsa_selftest_device_reset": (st, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -281,6 +282,10 @@ def vsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
 
 def vsa_selftest_wait_timeout(err, waited, stream=None):
     _check(lib.vsa_selftest_wait_timeout(_ptr(err), _ptr(waited), _stream(stream)), "vsa_selftest_wait_timeout")
+
+
+def vsa_selftest_device_reset():
+    _check(lib.vsa_selftest_device_reset(), "vsa_selftest_device_reset")
 
 
 # ---------------------------------------------------------------------------------------

@@ -5,11 +5,11 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <initializer_list>
-#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -413,7 +413,7 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   a.ucap = std::min(g.nblk, 2 * max_kv);
   a.gather = 0;
   a.nat_q = a.nat_k = a.nat_v = nullptr;
-  a.nat_o = nullptr;
+  a.nat_o = natural->o;  // written only for a head with an invalid kind byte (zero rows)
   const cudaError_t e = launch_sparse_attn(nat, perm, a, shape->d, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -809,29 +809,19 @@ vsa_status vsa_get_device_error(const int* d_err, cudaStream_t stream, int* host
 // acceptable.  For them vsa_profile_heads_static keeps its scratch in a fixed device array
 // of this file (kStaticProfileScratchBytes, held by every GPU that loads the library until
 // the process exits).  The array's host-side name is only a stand-in for the device
-// address, so the address is looked up once per device with cudaGetSymbolAddress and
-// passed to the kernels.
+// address.  Each call asks the runtime for the array's device address in the current context
+// (cudaGetSymbolAddress, a host-side lookup) and passes it to the kernels; no address is
+// cached, so a context that was reset and created again gets its own array's address.
 namespace vsa {
 constexpr size_t kStaticProfileScratchBytes = size_t(16) << 20;
-constexpr int kStaticMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_profile_scratch[kStaticProfileScratchBytes];
-static std::mutex g_profile_scratch_mu;
-static void* g_profile_scratch_ptr[kStaticMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up on first use).
+// Device address of the scratch array in the current device's context.
 static cudaError_t profile_scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_profile_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kStaticMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_profile_scratch_mu);
-  if (g_profile_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_profile_scratch);
-    if (e != cudaSuccess) return e;
-    g_profile_scratch_ptr[dev] = p;
-  }
-  *out = g_profile_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 }  // namespace vsa

@@ -113,7 +113,17 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
   const int pair = blockIdx.x - bh * npairs;
   const int kind = a.kinds[bh];
   if (kind > kCube || (a.gather && kind == kCube)) {  // in-kernel layout: cube heads need their copies
+    // The head's layout is unknown: its rows of the natural-order output (the buffer the caller
+    // reads) are written as zeros and LSE -inf, and the kind bit is raised.
     if (tid == 0 && pair == 0) atomicOr(a.err, kDevErrKind);
+    const int r0 = 2 * pair * BN, r1 = min(r0 + 2 * BN, a.nat_rows);
+    if (a.nat_o != nullptr)
+      for (int x = tid; x < (r1 - r0) * (D / 8); x += blockDim.x) {
+        const size_t row = static_cast<size_t>(bh) * a.nat_rows + r0 + x / (D / 8);
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.nat_o) + row * D)[x % (D / 8)] = make_uint4(0, 0, 0, 0);
+      }
+    if (a.lse_nat != nullptr)
+      for (int x = r0 + tid; x < r1; x += blockDim.x) a.lse_nat[static_cast<size_t>(bh) * a.nat_rows + x] = -INFINITY;
     return;
   }
   const int rows = layout_rows(g, kind);

@@ -52,3 +52,9 @@ extern "C" vsa_status vsa_selftest_exp2(const float* x, float* y_poly, float* y_
   vsa::exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
+
+// Test hook: reset the current device's primary context through this library's own CUDA
+// runtime, so that a test can check that later calls still find their device state.
+extern "C" vsa_status vsa_selftest_device_reset(void) {
+  return cudaDeviceReset() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}

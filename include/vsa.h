@@ -204,11 +204,17 @@ VSA_API vsa_status vsa_profile_heads(const void *q, const void *k, const void *v
  * pool, or a latency-critical path that must not call cudaMalloc.  The scratch lives in a
  * fixed array of vsa_profile_static_scratch_bytes() (16 MiB) inside the library, held by
  * every GPU that loads the library until the process exits; nothing is allocated.
- *   - Same arguments and results as vsa_profile_heads, minus ws / ws_bytes.
+ *   - Same arguments as vsa_profile_heads, minus ws / ws_bytes.
+ *   - To fit the array it may use fewer key-range splits than vsa_profile_heads, so its
+ *     fp32 partial sums combine in another order: the MSE values agree with those of
+ *     vsa_profile_heads within the profiling tolerance, and a head's kind can differ only
+ *     where its two MSEs are a near-tie.
  *   - Shapes whose scratch does not fit (after lowering the number of key-range splits to
  *     1) return VSA_ERR_WORKSPACE without launching anything.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the current context
+ *     (cudaGetSymbolAddress; nothing is cached, so a reset context is handled).  The first
+ *     call on a device may load the library's device code: make it before any stream
+ *     capture.
  *   - Every call shares the one array per device and leaves its contents behind; each call
  *     writes every scratch byte it reads, so no clearing is needed.  Calls that overlap on
  *     the GPU (different streams, or different host threads on the same device) race on
@@ -404,6 +410,13 @@ VSA_API vsa_status vsa_selftest_exp2(const float *x, float *y_poly, float *y_muf
  * returns; vsa_get_device_error then reports VSA_ERR_TIMEOUT and the context stays usable.
  *   d_err, d_waited  device ints (d_waited: 1 if the wait succeeded, 0 if it gave up) */
 VSA_API vsa_status vsa_selftest_wait_timeout(int *d_err, int *d_waited, cudaStream_t stream);
+
+/* Self-test hook (no counterpart in the pages): cudaDeviceReset of the current device through
+ * the library's own CUDA runtime.  It ends the calling process's context on that device, so
+ * every device buffer of the process becomes invalid; tests use it to check that entry points
+ * work again afterwards on new buffers (vsa_profile_heads_static looks its array's address up
+ * per call). */
+VSA_API vsa_status vsa_selftest_device_reset(void);
 
 /* Synchronise `stream`, copy the device error word to *host_err and map it to a status
  * (VSA_OK when zero, VSA_ERR_TIMEOUT when the timeout bit is set, else VSA_ERR_DEVICE). */

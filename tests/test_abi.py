@@ -34,8 +34,8 @@ def test_pattern_window_matches_oracle(wl, target):
         assert kept == pytest.approx(oracle.kept_fraction(kind, wl.F, wl.Hl, wl.Wl, wl.block, w), abs=1e-15)
 
 
-def test_survey_window_table():
-    # windows reached on the 21x30x52 grid (block 128), also listed in the design notes
+def test_wan_grid_window_table():
+    # the smallest windows reaching each kept fraction of the sweep on the 21x30x52 grid (block 128)
     shape = _lib.make_shape(1, 12, 21, 30, 52, 128, 128)
     got = {t: (_lib.vsa_pattern_window(shape, 0, t)[0], _lib.vsa_pattern_window(shape, 1, t)[0])
            for t in (1.0, 0.35, 0.18, 0.13, 0.05)}

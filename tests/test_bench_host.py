@@ -1,4 +1,6 @@
 """Host logic of bench.py that needs no GPU: the clock sampler's window filter."""
+import pytest
+
 import bench
 
 
@@ -86,5 +88,22 @@ def test_semantic_stage_work():
     assert exp2 == 1000 * 128 * 128
     roof = bench.stage_roofline(work, {"profile": 4.0, "permute": 0.1, "mask": 0.2, "unpermute": 0.05}, 6538.3,
                                 1631.1)
-    assert roof["profile"]["bound"] == "alu" and abs(roof["profile"]["peak"] - bench.FP32_PEAK_TFLOPS) < 1e-9
+    # no measured fp32 peak exists, so the k-means stage reports its rate without a fraction
+    assert roof["profile"]["bound"] == "alu" and roof["profile"]["peak"] is None and roof["profile"]["frac"] is None
     assert abs(roof["permute"]["achieved"] - work["permute"]["bytes"] / 1e-4 / 1e9) < 1e-6
+
+
+@pytest.mark.parametrize("F,Hl,Wl,block,w_s,w_t,r", [(6, 8, 16, 128, 1, 40, 37), (7, 5, 9, 64, 2, 7, 10),
+                                                     (21, 30, 52, 128, 2, 140, 328)])
+def test_profile_allowed_keys_matches_masks(F, Hl, Wl, block, w_s, w_t, r):
+    """The profiling stage's algorithmic work counts, per sampled row, the keys each pattern's
+    block mask allows (counted here from the oracle's masks and layouts)."""
+    wl = synthetic.Workload("p", 1, 1, F, Hl, Wl, 64, block, "bf16", "profiled")
+    N = wl.N
+    rows = [((2 * i + 1) * N) // (2 * r) for i in range(r)]
+    want = 0
+    for kind, w in ((oracle.SPATIAL, w_s), (oracle.TEMPORAL, w_t)):
+        keep = oracle.pattern_keep(kind, F, Hl, Wl, block, w)
+        blk = oracle.layout_slots(kind, F, Hl, Wl) // block
+        want += int(keep[blk[rows]][:, blk].sum())
+    assert bench.profile_allowed_keys(wl, r, w_s, w_t) == want

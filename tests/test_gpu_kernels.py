@@ -377,11 +377,15 @@ def test_attention_bad_lists_flag_error():
         order = torch.tensor(bad, dtype=torch.int32, device="cuda")
         _lib.vsa_sparse_attn_fwd(_lib.qkvo(q, q, q, o), None, kinds, good, ones, 2, shape, 0.0, err, order=order)
         assert _lib.vsa_get_device_error(err) & _lib.VSA_DEVERR_KV_RANGE, bad
-    # a bad kind byte
+    # a bad kind byte: the head's natural-order output rows are zero and its LSE is -inf
     err.zero_()
     kinds.fill_(9)
-    _lib.vsa_sparse_attn_fwd(_lib.qkvo(q, q, q, o), None, kinds, idx, cnt, 2, shape, 0.0, err)
+    o = torch.full_like(q, 5.0)
+    lse = torch.full((1, 1, wl.N), 5.0, dtype=torch.float32, device="cuda")
+    _lib.vsa_sparse_attn_fwd(_lib.qkvo(q, q, q, o, lse), None, kinds, idx, cnt, 2, shape, 0.0, err)
     assert _lib.vsa_get_device_error(err) & _lib.VSA_DEVERR_KIND
+    assert (o == 0).all()
+    assert torch.isneginf(lse).all()
 
 
 # ------------------------------------------------------------------------------------

@@ -6,8 +6,15 @@ can synchronise the device).  They cannot hand vsa_profile_heads a workspace, so
 offers a variant that keeps its scratch in a fixed array of its own.  This test calls that
 variant through the C ABI, twice in a row on the same inputs, and checks each result against
 the workspace-taking entry point.  It also checks that a shape too large for the fixed array
-is refused before anything is launched.  It lives in a file of its own so that it runs last.
+is refused before anything is launched, and that the variant still works after the device's
+context was reset (its array's address is looked up per call, never cached).  The file is
+collected last, so a run that stops at its first failure has run every other test before it.
 """
+import os
+import subprocess
+import sys
+import textwrap
+
 import numpy as np
 import pytest
 import torch
@@ -75,3 +82,67 @@ def test_static_scratch_refuses_oversized_shapes():
         _lib.vsa_profile_heads_static(dummy, dummy, dummy, shape, params, kinds, mse, err)
     assert exc.value.status == _lib.VSA_ERR_WORKSPACE
     assert _lib.vsa_get_device_error(err) == 0
+
+
+# Child process: device buffers come from the driver API (no torch CUDA state), the library
+# resets the context through its own runtime, and the same call on new buffers must give the
+# same bits as before the reset.
+_RESET_CHILD = textwrap.dedent("""
+    import ctypes, sys
+    import numpy as np
+    sys.path.insert(0, sys.argv[1])
+    import synthetic
+    from block_sparse_attention_31_b200 import _lib
+
+    cu = ctypes.CDLL("libcuda.so.1")
+    def ck(r):
+        assert r == 0, f"driver call failed: {r}"
+    def context():
+        dev, ctx = ctypes.c_int(), ctypes.c_void_p()
+        ck(cu.cuDeviceGet(ctypes.byref(dev), 0))
+        ck(cu.cuDevicePrimaryCtxRetain(ctypes.byref(ctx), dev))
+        ck(cu.cuCtxSetCurrent(ctx))
+    def upload(arr):
+        p = ctypes.c_uint64()
+        ck(cu.cuMemAlloc_v2(ctypes.byref(p), ctypes.c_size_t(max(arr.nbytes, 16))))
+        ck(cu.cuMemcpyHtoD_v2(ctypes.c_uint64(p.value), arr.ctypes.data_as(ctypes.c_void_p),
+                              ctypes.c_size_t(arr.nbytes)))
+        return p.value
+    def download(arr, p):
+        ck(cu.cuMemcpyDtoH_v2(arr.ctypes.data_as(ctypes.c_void_p), ctypes.c_uint64(p), ctypes.c_size_t(arr.nbytes)))
+
+    wl = synthetic.Workload("reset", 1, 4, 6, 8, 16, 128, 128, "bf16", "profiled")
+    q, k, v = (t.view(__import__("torch").int16).numpy().copy() for t in synthetic.make_qkv(wl))
+    shape = _lib.make_shape(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block)
+    params = _lib.make_params(1, 40, profile_frac=wl.profile_frac)
+
+    def run():
+        dq, dk, dv = upload(q), upload(k), upload(v)
+        kinds = np.full(wl.H, 7, dtype=np.uint8)
+        mse = np.full(2 * wl.H, -1.0, dtype=np.float32)
+        err = np.zeros(1, dtype=np.int32)
+        dkinds, dmse, derr = upload(kinds), upload(mse), upload(err)
+        _lib.vsa_profile_heads_static(dq, dk, dv, shape, params, dkinds, dmse, derr, stream=0)
+        assert _lib.vsa_get_device_error(derr, stream=0) == 0
+        download(kinds, dkinds)
+        download(mse, dmse)
+        return kinds, mse
+
+    ck(cu.cuInit(0))
+    context()
+    k1, m1 = run()
+    _lib.vsa_selftest_device_reset()
+    context()
+    k2, m2 = run()
+    assert np.array_equal(k1, k2), (k1, k2)
+    assert np.array_equal(m1.view(np.uint32), m2.view(np.uint32)), (m1, m2)
+    assert set(k1.tolist()) <= {0, 1} and (m1 >= 0).all()
+    print("reset ok", k1.tolist())
+""")
+
+
+def test_static_scratch_after_context_reset():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _RESET_CHILD, root], capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stdout[-2000:] + res.stderr[-4000:]
+    assert "reset ok" in res.stdout
