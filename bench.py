@@ -609,8 +609,12 @@ def oracle_sample(wl, seconds: float, seed: int = 0):
             rows_done += len(rows)
         n = min(n * 2, 4096)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    desc = (f"{rows_done} query rows of {heads} head(s) of {wl.name} (masks built for those heads in "
-            f"{mask_s:.1f} s, excluded), attention rows timed for {spent:.1f} s")
+    kinds_how = ("profiled by the oracle" if wl.mode == "profiled" and seconds > 60 else
+                 "the planted kinds (even heads spatial, odd temporal: what profiling picks on these inputs)"
+                 if wl.mode == "profiled" else "as the workload fixes them")
+    desc = (f"attention rows only (the dominant step; profiling, permutation and masks are not in the timed "
+            f"work): {rows_done} query rows of {heads} head(s) of {wl.name}, head kinds {kinds_how}, masks built "
+            f"for those heads in {mask_s:.1f} s (excluded), attention rows timed for {spent:.1f} s")
     return flops / spent, desc, cores, time.perf_counter() - t_begin
 
 

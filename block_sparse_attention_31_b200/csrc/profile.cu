@@ -35,6 +35,10 @@ constexpr int kProfThreads = 192;
 constexpr int kPM = 128;  // rows per tile
 constexpr int kNumSMs = 148;
 constexpr int kMaxSplits = 16;  // key-range splits per row tile, at most
+// A masked variant whose largest allowed logit lies more than this many base-2 units under
+// the dense running maximum is recomputed exactly: with a margin of 80, every probability the
+// 2^-126 flush can remove is below 2^-46 of the variant's own largest one.
+constexpr float kProfFlushMargin = 80.0f;
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -198,9 +202,12 @@ __device__ __forceinline__ void set_bit_range(uint32_t (&m)[BN / 32], int lo, in
 // probabilities are masked copies of the dense ones and each score is exponentiated once.
 // The spatial P.V reads the dense P with the rows outside the window disabled (the MMA's
 // output-lane mask); the temporal P.V reads a masked copy with rows that allow no key of the
-// block disabled.  Contributions more than 2^126 below the dense maximum flush to zero.
-// Both P tiles live in shared memory so that Q.K^T of block j+1 runs while the softmax of
-// block j computes.
+// block disabled.  Probabilities more than 2^126 below the running dense maximum flush to
+// zero, so each row also tracks the largest logit each masked variant allows: when that is
+// more than kProfFlushMargin (base 2) below the dense maximum, the variant's partial sum could
+// have lost weight to the flush, and the split marks it (l = -1) for the row-error kernel,
+// which then recomputes that variant of the row with its own maximum.  Both P tiles live in
+// shared memory so that Q.K^T of block j+1 runs while the softmax of block j computes.
 template <int D, int BN>
 __global__ void __launch_bounds__(kProfThreads, 1)
     profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
@@ -378,6 +385,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     const int ts_lo = rg.z / g.F, tf_lo = rg.z - (rg.z / g.F) * g.F;
     const int ts_hi = t_any ? (rg.w - 1) / g.F : -1, tf_hi = t_any ? (rg.w - 1) - ((rg.w - 1) / g.F) * g.F : -1;
     float m = -INFINITY, l[3] = {0.f, 0.f, 0.f};
+    float mv_s = -INFINITY, mv_t = -INFINITY;  // largest allowed logit (base 2) of each masked variant
     {  // the spatial and temporal accumulators only ever accumulate: start them at zero
       float z[32];
 #pragma unroll
@@ -440,6 +448,8 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
       uint64_t rs2[2] = {0ull, 0ull};
       float rt4[4] = {0.f, 0.f, 0.f, 0.f};
+      float tx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // temporal-allowed max of x
+      if (sp_on) mv_s = fmaxf(mv_s, mx * sl2);
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN / 2; ++c) {
@@ -452,6 +462,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         if (warp_tp) {
           const uint32_t b = (mt[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
           rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+          tx4[c & 3] = fmax3(tx4[c & 3], (b & 1u) ? x0 : -INFINITY, (b & 2u) ? x1 : -INFINITY);
         }
       }
       // the previous block's P.V products must be done: O stable, P tiles free
@@ -495,6 +506,10 @@ __global__ void __launch_bounds__(kProfThreads, 1)
           *reinterpret_cast<uint4*>(pPT + off) = make_uint4(m4[0], m4[1], m4[2], m4[3]);
         }
       }
+      {
+        const float tx = fmaxf(fmaxf(tx4[0], tx4[1]), fmaxf(tx4[2], tx4[3]));
+        if (tx != -INFINITY) mv_t = fmaxf(mv_t, tx + m_use);
+      }
       float rs0, rs1;
       f2_split(f2_add(rs2[0], rs2[1]), rs0, rs1);
       const float rs = rs0 + rs1;
@@ -515,14 +530,18 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
       tc_fence_after();
     }
-    // partials: (m, l) and unnormalised O of each variant
+    // partials: (m, l) and unnormalised O of each variant; l = -1 marks a masked variant
+    // whose allowed logits all sit more than kProfFlushMargin below the dense maximum
     const size_t base = ((static_cast<size_t>(bh) * a.splits + split) * 3) * a.r_pad + tile * kPM + row;
+    const bool low_s = mv_s != -INFINITY && mv_s < m - kProfFlushMargin;
+    const bool low_t = mv_t != -INFINITY && mv_t < m - kProfFlushMargin;
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
       const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
       const bool have = ok && cnt > 0;
+      const bool low = vv == 1 ? low_s : vv == 2 ? low_t : false;
       a.ml[prow * 2 + 0] = have ? m : -INFINITY;
-      a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
+      a.ml[prow * 2 + 1] = have ? (low ? -1.f : l[vv]) : 0.f;
       float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -544,11 +563,75 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+// Output x of one masked variant of sampled row i recomputed with the variant's own maximum
+// (used when a split marked the variant: its allowed logits sit far below the dense maximum).
+// The d threads of the CTA form d/32 warps; each warp takes every (d/32)-th allowed key, its
+// lanes hold d/32 dimensions each and reduce q.k with shuffles.  Two passes: the maximum, then the
+// exponentials, their sum and sum p*v.  Spatial keys are the natural tokens [lo, hi);
+// temporal keys the frame-major slots [lo, hi), slot p being token (p % F) * S + p / F.
+__device__ float profile_variant_exact(const __nv_bfloat16* __restrict__ qrow, const __nv_bfloat16* __restrict__ kh,
+                                       const __nv_bfloat16* __restrict__ vh, int lo, int hi, bool frame_major,
+                                       const Geom& g, int d, float scale_log2) {
+  __shared__ float red_m[4], red_l[4];
+  __shared__ float red_o[4][128];
+  const int x = threadIdx.x, warp = x >> 5, lane = x & 31, nw = blockDim.x >> 5;  // nw = d / 32
+  const int per = d / 32;  // dimensions per lane (2 or 4)
+  float qv[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) qv[e] = e < per ? __bfloat162float(qrow[lane * per + e]) : 0.f;
+  auto logit = [&](int slot) -> float {
+    const int t = frame_major ? (slot % g.F) * g.S + slot / g.F : slot;
+    const __nv_bfloat16* kr = kh + static_cast<size_t>(t) * d + lane * per;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (e < per) acc = fmaf(qv[e], __bfloat162float(kr[e]), acc);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    return acc * scale_log2;
+  };
+  float mx = -INFINITY;
+  for (int u = lo + warp; u < hi; u += nw) mx = fmaxf(mx, logit(u));
+  if (lane == 0) red_m[warp] = mx;
+  __syncthreads();
+  float M = red_m[0];
+  for (int w = 1; w < nw; ++w) M = fmaxf(M, red_m[w]);
+  float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  if (M != -INFINITY)
+    for (int u = lo + warp; u < hi; u += nw) {
+      const float p = exp2f(logit(u) - M);
+      L += p;
+      const int t = frame_major ? (u % g.F) * g.S + u / g.F : u;
+      const __nv_bfloat16* vr = vh + static_cast<size_t>(t) * d + lane * per;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e < per) o[e] = fmaf(p, __bfloat162float(vr[e]), o[e]);
+    }
+  if (lane == 0) red_l[warp] = L;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (e < per) red_o[warp][lane * per + e] = o[e];
+  __syncthreads();
+  float Lt = 0.f, ot = 0.f;
+  for (int w = 0; w < nw; ++w) {
+    Lt += red_l[w];
+    ot += red_o[w][x];
+  }
+  __syncthreads();  // the shared partials may be reused by the next call
+  return Lt > 0.f ? ot / Lt : 0.f;
+}
+
 // Merge the key splits of one sampled row of one head and accumulate its two squared errors
 // (one CTA of d threads per (row, head)); the per-row sums are reduced in fixed order below.
+// A masked variant that any split marked (l = -1) is recomputed with its own maximum.
 __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __restrict__ opart,
                                                                 const float* __restrict__ ml, int r_pad,
-                                                                int splits, int d, double* __restrict__ row_err) {
+                                                                int splits, int d, double* __restrict__ row_err,
+                                                                const __nv_bfloat16* __restrict__ qs,
+                                                                const __nv_bfloat16* __restrict__ k,
+                                                                const __nv_bfloat16* __restrict__ v,
+                                                                const int4* __restrict__ ranges, Geom g,
+                                                                float scale_log2) {
   __shared__ double red[2][4];
   const int i = blockIdx.x, bh = blockIdx.y, x = threadIdx.x;
   float o[3];
@@ -556,6 +639,7 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
   for (int vv = 0; vv < 3; ++vv) {
     // all splits' partials are loaded before they are combined (at most kMaxSplits)
     float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
+    bool low = false;
 #pragma unroll
     for (int sp = 0; sp < kMaxSplits; ++sp) {
       ms[sp] = -INFINITY;
@@ -565,7 +649,16 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
         ms[sp] = __ldg(ml + prow * 2);
         ls[sp] = __ldg(ml + prow * 2 + 1);
         os[sp] = __ldg(opart + prow * d + x);
+        low |= ls[sp] < 0.f;
       }
+    }
+    if (low) {  // uniform across the CTA: every thread read the same (m, l) partials
+      const int4 rg = ranges[i];
+      const bool tp = vv == 2;
+      o[vv] = profile_variant_exact(qs + (static_cast<size_t>(bh) * r_pad + i) * d,
+                                    k + static_cast<size_t>(bh) * g.N * d, v + static_cast<size_t>(bh) * g.N * d,
+                                    tp ? rg.z : rg.x, tp ? rg.w : rg.y, tp, g, d, scale_log2);
+      continue;
     }
     float M = -INFINITY;
 #pragma unroll
@@ -688,7 +781,10 @@ cudaError_t launch_profile(const void* q, const void* k, const void* v, const Ge
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;
   double* row_err = reinterpret_cast<double*>(w + plan.off_rowerr);
-  profile_row_error_kernel<<<dim3(plan.r, BH), d, 0, stream>>>(opart, ml, plan.r_pad, plan.splits, d, row_err);
+  profile_row_error_kernel<<<dim3(plan.r, BH), d, 0, stream>>>(opart, ml, plan.r_pad, plan.splits, d, row_err, qs,
+                                                                static_cast<const __nv_bfloat16*>(k),
+                                                                static_cast<const __nv_bfloat16*>(v), ranges, g,
+                                                                scale_log2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   profile_reduce_kernel<<<BH, kRedThreads, 0, stream>>>(row_err, plan.r, plan.r_pad, d, kinds_out, mse_out);

@@ -10,13 +10,15 @@
 //     an empty cluster keeps its centroid;
 //   - cluster-major order: slots sorted by (cluster, token);
 //   - weight of key cluster j for query cluster i: n_j exp(s_ij - max_j s_ij), s_ij = scale *
-//     cq_i . ck_j in fp64 (dimension order, fused multiply-adds); kept: the shortest prefix of
-//     the weights sorted in descending order (ties to the smaller j) whose running sum reaches
-//     top_p times the sum of all of them;
+//     cq_i . ck_j in fp64 (dimension order, fused multiply-adds; CUDA's fp64 exp); kept: the
+//     shortest prefix of the weights sorted in descending order (ties to the smaller j) whose
+//     running sum reaches top_p times the sum of all of them;
 //   - block pair (a, b) of the two cluster-major layouts is kept when some query slot of a
 //     and some key slot of b belong to a kept cluster pair.
 // Every floating-point step that decides an integer (assignment, order, top-p) is written
-// out with explicitly rounded operations, so the result does not depend on contraction.
+// out with explicitly rounded operations, so the result does not depend on contraction.  The
+// assignment's fp32 distances can differ from exact ones by a bounded amount: where two
+// centroids are that close to a tie, either label is a correct nearest-centroid choice.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -363,28 +365,6 @@ __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(const __nv_b
 // top-p budget
 // ---------------------------------------------------------------------------------------
 
-// exp(x) for x <= 0: Cody and Waite's reduction x = n ln2 + r (ln2 split into a 32-bit head
-// and a tail), Taylor series of e^r to degree 13 in Horner form, scaling by 2^n built from its
-// bit pattern; 0 below -700.
-__device__ double exp_neg(double x) {
-  const double ln2_hi = 0x1.62e42fee00000p-1, ln2_lo = 0x1.a39ef35793c76p-33;
-  const double inv_ln2 = 0x1.71547652b82fep+0;
-  const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1, 0x1.5555555555555p-3,
-                        0x1.5555555555555p-5, 0x1.1111111111111p-7, 0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13,
-                        0x1.a01a01a01a01ap-16, 0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
-                        0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
-  if (!(x > -700.0)) return 0.0;
-  if (x > 0.0) x = 0.0;
-  const double n = rint(__dmul_rn(x, inv_ln2));
-  double r = __fma_rn(-n, ln2_hi, x);
-  r = __fma_rn(-n, ln2_lo, r);
-  double p = c[13];
-#pragma unroll
-  for (int i = 12; i >= 0; --i) p = __fma_rn(p, r, c[i]);
-  const double two_n = __longlong_as_double(static_cast<long long>(static_cast<int>(n) + 1023) << 52);
-  return __dmul_rn(p, two_n);
-}
-
 // Kept key clusters of query cluster blockIdx.x of head blockIdx.y: keep[bh, i, ceil(Ck/32)].
 __global__ void __launch_bounds__(kKeepThreads) semantic_keep_kernel(const float* __restrict__ cq,
                                                                      const int32_t* __restrict__ nq, int Cq,
@@ -427,7 +407,7 @@ __global__ void __launch_bounds__(kKeepThreads) semantic_keep_kernel(const float
   for (int w = 1; w < kKeepThreads / 32; ++w) m = fmax(m, red[w]);
   for (int j = tid; j < n2; j += kKeepThreads) {
     if (ks_i[j] != kNone)
-      ks_w[j] = __dmul_rn(static_cast<double>(nkh[ks_i[j]]), exp_neg(__dsub_rn(ks_w[j], m)));
+      ks_w[j] = __dmul_rn(static_cast<double>(nkh[ks_i[j]]), exp(__dsub_rn(ks_w[j], m)));  // CUDA fp64 exp
     else
       ks_w[j] = -1.0;  // below every weight (weights are >= 0)
   }

@@ -60,12 +60,16 @@ def _load():
         lib.or_attention_rows.argtypes = [vp, vp, vp, i64, i64, dbl, vp, i64, vp, i64, vp, i64, vp, vp]
         lib.or_attention_rows_qk.restype = None
         lib.or_attention_rows_qk.argtypes = [vp, vp, vp, i64, i64, dbl, vp, vp, i64, vp, i64, vp, i64, vp, vp]
-        lib.or_exp_neg.restype = dbl
-        lib.or_exp_neg.argtypes = [dbl]
+        lib.or_kmeans_assign.restype = None
+        lib.or_kmeans_assign.argtypes = [vp, i64, i64, vp, i64, vp, vp]
+        lib.or_kmeans_update.restype = ctypes.c_int
+        lib.or_kmeans_update.argtypes = [vp, i64, i64, vp, i64, vp, vp]
         lib.or_kmeans.restype = ctypes.c_int
         lib.or_kmeans.argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
         lib.or_cluster_perm.restype = None
         lib.or_cluster_perm.argtypes = [vp, i64, i64, vp, vp]
+        lib.or_semantic_weights.restype = None
+        lib.or_semantic_weights.argtypes = [vp, vp, i64, vp, vp, i64, i64, dbl, vp]
         lib.or_semantic_keep.restype = None
         lib.or_semantic_keep.argtypes = [vp, vp, i64, vp, vp, i64, i64, dbl, dbl, vp]
         lib.or_profile_rows.restype = i64
@@ -177,11 +181,6 @@ def profile_head(q, k, v, F, Hl, Wl, block, w_s, w_t, frac=0.01, scale=None):
 # vsa_oracle.c next to the C functions.
 # ---------------------------------------------------------------------------------------
 
-def exp_neg(x: float) -> float:
-    """The oracle's own exp for x <= 0 (0 below -700)."""
-    return float(_load().or_exp_neg(float(x)))
-
-
 def _f32(x) -> np.ndarray:
     if hasattr(x, "detach"):
         x = x.detach().to("cpu").float().numpy()
@@ -198,6 +197,38 @@ def kmeans(x, C: int, iters: int):
     if _load().or_kmeans(_p(x), N, d, C, iters, _p(cent), _p(label), _p(count)) != 0:
         raise ValueError("oracle k-means: bad arguments or allocation failure")
     return cent, label, count
+
+
+def kmeans_assign(x, cent):
+    """One assignment step: (labels [N] of the nearest centroid by fp64 squared distance, ties
+    to the smaller index; gap [N] = second-nearest minus nearest distance)."""
+    x, cent = _f32(x), _f32(cent)
+    N, d = x.shape
+    label = np.empty(N, dtype=np.int32)
+    gap = np.empty(N, dtype=np.float64)
+    _load().or_kmeans_assign(_p(x), N, d, _p(cent), cent.shape[0], _p(label), _p(gap))
+    return label, gap
+
+
+def kmeans_update(x, label, prev_cent):
+    """One update step from given labels: (centroids [C, d] fp32, counts [C]); an empty
+    cluster keeps its row of ``prev_cent``."""
+    x = _f32(x)
+    N, d = x.shape
+    cent = np.array(_f32(prev_cent), copy=True)
+    label = np.ascontiguousarray(label, dtype=np.int32)
+    count = np.empty(cent.shape[0], dtype=np.int32)
+    if _load().or_kmeans_update(_p(x), N, d, _p(label), cent.shape[0], _p(cent), _p(count)) != 0:
+        raise MemoryError("oracle k-means update allocation failed")
+    return cent, count
+
+
+def kmeans_init(x, C: int):
+    """Initial centroids: the rows floor((2j+1)N/(2C)) of x."""
+    x = _f32(x)
+    N = x.shape[0]
+    rows = [((2 * j + 1) * N) // (2 * C) for j in range(C)]
+    return np.ascontiguousarray(x[rows])
 
 
 def cluster_perm(label, C: int):
@@ -219,6 +250,19 @@ def semantic_keep(cq, nq, ck, nk, scale: float, top_p: float) -> np.ndarray:
     keep = np.empty((Cq, Ck), dtype=np.uint8)
     _load().or_semantic_keep(_p(cq), _p(nq), Cq, _p(ck), _p(nk), Ck, d, float(scale), float(top_p), _p(keep))
     return keep.astype(bool)
+
+
+def semantic_weights(cq, nq, ck, nk, scale: float) -> np.ndarray:
+    """Criticality weights [Cq, Ck] (fp64): n_j exp(s_ij - max_j s_ij); -1 where a cluster is
+    empty."""
+    cq, ck = _f32(cq), _f32(ck)
+    nq = np.ascontiguousarray(nq, dtype=np.int32)
+    nk = np.ascontiguousarray(nk, dtype=np.int32)
+    Cq, d = cq.shape
+    Ck = ck.shape[0]
+    w = np.empty((Cq, Ck), dtype=np.float64)
+    _load().or_semantic_weights(_p(cq), _p(nq), Cq, _p(ck), _p(nk), Ck, d, float(scale), _p(w))
+    return w
 
 
 def semantic_block_keep(label_q, perm_q, label_k, perm_k, keep, block: int) -> np.ndarray:

@@ -22,8 +22,7 @@
  *          FlashAttention kernels, i.e. it is ordinary softmax(QK^T * scale) V restricted
  *          to the kept keys.
  *
- * Readings where the pages give no formula (each is listed with its reason in the
- * design notes of the repository):
+ * Readings where the pages give no formula:
  *   - attention is softmax(q.k / sqrt(d)) over the allowed keys, times V;
  *   - a head's layout maps token t = f*S + s (S = Hl*Wl) to a slot: identity for spatial
  *     heads, s*F + f for temporal heads (frame-major), and for cube heads
@@ -34,17 +33,16 @@
  *     those intervals are at most w apart (the block-level cover of |f_q - f_k| <= w_s,
  *     respectively |s_q - s_k| <= w_t);
  *   - the window is the smallest w whose kept-block fraction reaches the target;
- *   - cube selection: fp64 mean of Q and K over each cube's real tokens (summed in token
- *     order), score qbar_c . kbar_c' (summed in dimension order, one fused multiply-add
- *     per term), keep the top k per row (score descending, ties to the smaller index)
- *     together with the cube itself;
+ *   - cube selection: fp64 mean of Q and K over each cube's real tokens, score
+ *     qbar_c . kbar_c' (a plain fp64 dot product), keep the top k per row (score
+ *     descending, ties to the smaller index) together with the cube itself;
  *   - profiling rows rho_i = floor((2i+1) N / (2r)), r = ceil(frac * N); error = mean
  *     squared difference to dense attention on those rows under the block masks that
  *     would be executed; ties go to the spatial pattern;
  *   - a row with no allowed key has output 0 and log-sum-exp -inf.
  *
- * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no -ffast-math; the only fused
- * multiply-adds are the explicit fma() calls of the coarse scores).
+ * Build: gcc -O2 -fopenmp -shared -fPIC -ffp-contract=off (no -ffast-math, no fused
+ * multiply-adds: every product and sum is rounded on its own, as written).
  */
 #include <math.h>
 #include <stdint.h>
@@ -173,12 +171,12 @@ int or_cube_topk_keep(const double *q, const double *k, int64_t F, int64_t Hl, i
             qbar[c * d + x] /= (double)count[c];
             kbar[c * d + x] /= (double)count[c];
         }
-    /* coarse scores: fp64 dot products in dimension order, one fused multiply-add per term */
+    /* coarse scores: plain fp64 dot products */
 #pragma omp parallel for schedule(static)
     for (int64_t c = 0; c < C; ++c)
         for (int64_t c2 = 0; c2 < C; ++c2) {
             double acc = 0.0;
-            for (int64_t x = 0; x < d; ++x) acc = fma(qbar[c * d + x], kbar[c2 * d + x], acc);
+            for (int64_t x = 0; x < d; ++x) acc += qbar[c * d + x] * kbar[c2 * d + x];
             score[c * C + c2] = acc;
         }
     /* per row: pick the best remaining column topk times (selection by repeated max) */
@@ -314,63 +312,74 @@ int or_profile_head(const double *q, const double *k, const double *v, int64_t F
  * reordered so that each cluster is contiguous, and a top-p budget over the clusters
  * picks the critical key clusters of each query cluster.  The page gives no formulas;
  * the readings used here:
- *   - Lloyd's k-means per head, separately on Q and on K, `iters` rounds of assignment
- *     then update; initial centroids are the rows rho_j = floor((2j+1) N / (2C));
- *   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32 (both dot products summed in
- *     dimension order, one fused multiply-add per term), ties to the smaller j;
- *   - update: fp64 sum of the members in token order, divided by the member count and
- *     rounded to fp32; an empty cluster keeps its centroid;
+ *   - Lloyd's k-means per head, separately on Q and on K, `iters` rounds of assignment then
+ *     update; initial centroids are the rows rho_j = floor((2j+1) N / (2C));
+ *   - assignment: each row goes to the centroid at the smallest squared Euclidean
+ *     distance sum_x (x - c_j)^2, computed in fp64; exact ties to the smaller j;
+ *   - update: a centroid is the mean of its members, computed in fp64 and stored in fp32
+ *     (centroids are fp32 vectors); an empty cluster keeps its centroid;
  *   - cluster-major order: slots sorted by (cluster, token);
  *   - criticality of key cluster j for query cluster i: n_j exp(s_ij - max_j s_ij) with
- *     s_ij = scale * cq_i . ck_j (fp64, dimension order, fused multiply-adds); the kept
- *     clusters are the shortest prefix of the list sorted by weight (descending, ties to
- *     the smaller j) whose running sum reaches top_p times the sum of the whole list;
+ *     s_ij = scale * cq_i . ck_j (fp64); the kept clusters are the shortest prefix of the
+ *     list sorted by weight (descending, ties to the smaller j) whose running sum reaches
+ *     top_p times the sum of the whole list;
  *   - block pair (a, b) of the two cluster-major layouts is kept when some query slot of
  *     block a and some key slot of block b belong to a kept cluster pair.
- * The floating-point steps that decide an integer (assignment, top-p) are taken in the
- * precision and order stated above, which is also the CUDA path's.
  * ------------------------------------------------------------------------------------- */
 
-/* 2^n for an integer n in the normal range, built from its bit pattern (exact). */
-static double pow2i(int64_t n)
+/* Squared Euclidean distance of two fp32 vectors, in fp64. */
+static double dist2(const float *a, const float *b, int64_t d)
 {
-    uint64_t bits = (uint64_t)(n + 1023) << 52;
-    double r;
-    memcpy(&r, &bits, sizeof r);
-    return r;
+    double acc = 0.0;
+    for (int64_t x = 0; x < d; ++x) {
+        double t = (double)a[x] - (double)b[x];
+        acc += t * t;
+    }
+    return acc;
 }
 
 /*
- * exp(x) for x <= 0 (Cody and Waite's argument reduction, x = n ln2 + r with ln2 split into
- * a 32-bit head and a tail, then the Taylor series of e^r to degree 13, Horner form with
- * fused multiply-adds).  Below -700 the result is 0: weights that small do not matter and
- * the scaling stays exact.
+ * Assignment step: label[t] = the nearest of the C centroids cent [C, d] to row t of x [N, d]
+ * (fp64 squared distance, ties to the smaller index).  gap (optional, [N]) receives the
+ * distance of the second-nearest centroid minus that of the nearest (0 for C = 1 or a tie).
  */
-double or_exp_neg(double x)
+void or_kmeans_assign(const float *x, int64_t N, int64_t d, const float *cent, int64_t C, int32_t *label,
+                      double *gap)
 {
-    static const double ln2_hi = 0x1.62e42fee00000p-1, ln2_lo = 0x1.a39ef35793c76p-33;
-    static const double inv_ln2 = 0x1.71547652b82fep+0;
-    static const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1,
-                                 0x1.5555555555555p-3, 0x1.5555555555555p-5, 0x1.1111111111111p-7,
-                                 0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
-                                 0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
-                                 0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
-    if (!(x > -700.0)) return 0.0;
-    if (x > 0.0) x = 0.0;
-    double n = nearbyint(x * inv_ln2);
-    double r = fma(-n, ln2_hi, x);
-    r = fma(-n, ln2_lo, r);
-    double p = c[13];
-    for (int i = 12; i >= 0; --i) p = fma(p, r, c[i]);
-    return p * pow2i((int64_t)n);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        int64_t best = 0;
+        double bd = INFINITY, second = INFINITY;
+        for (int64_t j = 0; j < C; ++j) {
+            double dj = dist2(x + t * d, cent + j * d, d);
+            if (dj < bd) { second = bd; bd = dj; best = j; }
+            else if (dj < second) second = dj;
+        }
+        label[t] = (int32_t)best;
+        if (gap) gap[t] = C > 1 ? second - bd : 0.0;
+    }
 }
 
-/* Squared norm and dot product in fp32, dimension order, one fused multiply-add per term. */
-static float dot_f32(const float *a, const float *b, int64_t d)
+/*
+ * Update step: cent[j] = fp32 of the fp64 mean of the rows labelled j; an empty cluster keeps
+ * cent[j].  count [C] receives the member counts.  Returns 0, or -1 on allocation failure.
+ */
+int or_kmeans_update(const float *x, int64_t N, int64_t d, const int32_t *label, int64_t C, float *cent,
+                     int32_t *count)
 {
-    float acc = 0.0f;
-    for (int64_t x = 0; x < d; ++x) acc = fmaf(a[x], b[x], acc);
-    return acc;
+    double *sum = (double *)calloc((size_t)(C * d), sizeof(double));
+    if (!sum) return -1;
+    memset(count, 0, sizeof(int32_t) * (size_t)C);
+    for (int64_t t = 0; t < N; ++t) {
+        int64_t j = label[t];
+        count[j] += 1;
+        for (int64_t q = 0; q < d; ++q) sum[j * d + q] += (double)x[t * d + q];
+    }
+    for (int64_t j = 0; j < C; ++j)
+        if (count[j] > 0)
+            for (int64_t q = 0; q < d; ++q) cent[j * d + q] = (float)(sum[j * d + q] / (double)count[j]);
+    free(sum);
+    return 0;
 }
 
 /*
@@ -382,37 +391,14 @@ int or_kmeans(const float *x, int64_t N, int64_t d, int64_t C, int64_t iters, fl
               int32_t *count)
 {
     if (C < 1 || C > N || iters < 1) return -1;
-    float *nc = (float *)malloc(sizeof(float) * (size_t)C);
-    double *sum = (double *)malloc(sizeof(double) * (size_t)(C * d));
-    if (!nc || !sum) { free(nc); free(sum); return -1; }
     for (int64_t j = 0; j < C; ++j) {
         int64_t r = ((2 * j + 1) * N) / (2 * C);
         memcpy(cent + j * d, x + r * d, sizeof(float) * (size_t)d);
     }
     for (int64_t it = 0; it < iters; ++it) {
-        for (int64_t j = 0; j < C; ++j) nc[j] = dot_f32(cent + j * d, cent + j * d, d);
-#pragma omp parallel for schedule(static)
-        for (int64_t t = 0; t < N; ++t) {
-            int32_t best = 0;
-            float best_d = 0.0f;
-            for (int64_t j = 0; j < C; ++j) {
-                float dist = nc[j] - 2.0f * dot_f32(x + t * d, cent + j * d, d);
-                if (j == 0 || dist < best_d) { best = (int32_t)j; best_d = dist; }
-            }
-            label[t] = best;
-        }
-        memset(count, 0, sizeof(int32_t) * (size_t)C);
-        memset(sum, 0, sizeof(double) * (size_t)(C * d));
-        for (int64_t t = 0; t < N; ++t) {
-            int64_t j = label[t];
-            count[j] += 1;
-            for (int64_t q = 0; q < d; ++q) sum[j * d + q] += (double)x[t * d + q];
-        }
-        for (int64_t j = 0; j < C; ++j)
-            if (count[j] > 0)
-                for (int64_t q = 0; q < d; ++q) cent[j * d + q] = (float)(sum[j * d + q] / (double)count[j]);
+        or_kmeans_assign(x, N, d, cent, C, label, NULL);
+        if (or_kmeans_update(x, N, d, label, C, cent, count) != 0) return -1;
     }
-    free(nc); free(sum);
     return 0;
 }
 
@@ -434,6 +420,31 @@ void or_cluster_perm(const int32_t *label, int64_t N, int64_t C, int32_t *perm, 
  * member keeps nothing, an empty key cluster is never kept.  scale and p as described
  * above (0 < p <= 1).
  */
+/*
+ * Criticality weights of every key cluster for every query cluster: w[i * Ck + j] =
+ * n_j exp(s_ij - max_j s_ij), s_ij = scale * cq_i . ck_j (fp64), over the non-empty key
+ * clusters; -1 marks an empty key cluster (or every entry of an empty query cluster).
+ */
+void or_semantic_weights(const float *cq, const int32_t *nq, int64_t Cq, const float *ck, const int32_t *nk,
+                         int64_t Ck, int64_t d, double scale, double *w)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < Cq; ++i) {
+        double *row = w + i * Ck;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < Ck; ++j) {
+            row[j] = -1.0;
+            if (nq[i] == 0 || nk[j] == 0) continue;
+            double acc = 0.0;
+            for (int64_t x = 0; x < d; ++x) acc += (double)cq[i * d + x] * (double)ck[j * d + x];
+            row[j] = scale * acc;
+            if (row[j] > m) m = row[j];
+        }
+        for (int64_t j = 0; j < Ck; ++j)
+            if (nq[i] > 0 && nk[j] > 0) row[j] = (double)nk[j] * exp(row[j] - m);
+    }
+}
+
 void or_semantic_keep(const float *cq, const int32_t *nq, int64_t Cq, const float *ck, const int32_t *nk,
                       int64_t Ck, int64_t d, double scale, double p, uint8_t *keep)
 {
@@ -449,13 +460,13 @@ void or_semantic_keep(const float *cq, const int32_t *nq, int64_t Cq, const floa
         for (int64_t j = 0; j < Ck; ++j) {
             if (nk[j] == 0) continue;
             double acc = 0.0;
-            for (int64_t x = 0; x < d; ++x) acc = fma((double)cq[i * d + x], (double)ck[j * d + x], acc);
+            for (int64_t x = 0; x < d; ++x) acc += (double)cq[i * d + x] * (double)ck[j * d + x];
             w[j] = scale * acc;
             if (w[j] > m) m = w[j];
         }
         int64_t live = 0;
         for (int64_t j = 0; j < Ck; ++j)
-            if (nk[j] > 0) { w[j] = (double)nk[j] * or_exp_neg(w[j] - m); ++live; }
+            if (nk[j] > 0) { w[j] = (double)nk[j] * exp(w[j] - m); ++live; }
         /* the list sorted by weight, by repeated selection of the largest remaining entry */
         int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)(live > 0 ? live : 1));
         if (!order) { free(w); free(used); continue; }

@@ -28,3 +28,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report the GPU answers that were accepted at oracle near-ties (see tests/validity.py)."""
+    mod = sys.modules.get("validity")
+    if mod is None:
+        return
+    terminalreporter.write_line(mod.summary())
+    for cat, detail in mod.LOG[:50]:
+        terminalreporter.write_line(f"  {cat}: {detail}")

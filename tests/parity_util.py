@@ -46,3 +46,20 @@ def to_f64(t):
 
 def cuda_err():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# Profiling MSE tolerance.  The kernel forms each variant's output with P rounded to bf16
+# (relative error up to 2^-9 per probability) and fp32 accumulation, so an output element can
+# be off by about 2^-9 times the size of the outputs, and the difference of two variants by
+# twice that.  With eps = 2^-7 * max |O_dense| over the sampled outputs (a factor 2 of margin),
+# an MSE m computed from differences off by at most eps is within 2 sqrt(m) eps + eps^2 of the
+# exact one.
+MSE_EPS_REL = 2.0 ** -7
+MSE_LOG = []
+
+
+def mse_close(got: float, want: float, dense_rows, what=""):
+    eps = MSE_EPS_REL * float(np.abs(dense_rows).max())
+    bound = 2.0 * math.sqrt(max(want, 0.0)) * eps + eps * eps
+    MSE_LOG.append((what, got, want, abs(got - want) / max(bound, 1e-300)))
+    assert abs(got - want) <= bound, f"{what}: MSE {got!r} vs oracle {want!r}, bound {bound:.3e}"

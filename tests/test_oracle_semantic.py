@@ -2,9 +2,9 @@
 k-means clustering of tokens, cluster-major reordering, top-p budget over clusters).
 
 The checks take routes other than the oracle's own loops:
-- Python's math.exp for the exponential;
 - planted blobs whose clustering is known in closed form;
-- fp64 numpy distances and means for the assignment and update;
+- scipy's cdist distances and numpy means for the assignment and update;
+- a hand-built case that only exact (fp64) distances resolve;
 - bincount/argsort for the order;
 - numpy weights for the top-p prefix;
 - membership-matrix products for the block mask;
@@ -17,23 +17,6 @@ import pytest
 import torch
 
 import oracle
-
-
-# ------------------------------------------------------------------------------------
-# exp
-# ------------------------------------------------------------------------------------
-
-def test_exp_neg_matches_math_exp():
-    """Within 2 ulp of the library exp on [-700, 0]; exact at 0; 0 below -700."""
-    xs = np.concatenate([-np.random.default_rng(0).random(4000) * 700.0, -np.random.default_rng(1).random(4000),
-                         -np.arange(0, 700) * math.log(2.0), [0.0, -0.5, -1e-300, -699.9]])
-    worst = 0.0
-    for x in xs:
-        got, want = oracle.exp_neg(float(x)), math.exp(float(x))
-        worst = max(worst, abs(got - want) / want)
-    assert worst <= 2.0 ** -51, worst
-    assert oracle.exp_neg(0.0) == 1.0
-    assert oracle.exp_neg(-701.0) == 0.0 and oracle.exp_neg(-float("inf")) == 0.0
 
 
 # ------------------------------------------------------------------------------------
@@ -67,23 +50,47 @@ def test_kmeans_recovers_planted_blobs(N, C, d):
 
 
 def test_kmeans_assignment_and_update_rules():
-    """Round T assigns each row to a nearest centroid of round T-1 (fp64 distances, within
-    fp32 rounding), and round T's centroids are the fp32 means of those members."""
+    """Round T assigns each row to the nearest centroid of round T-1 (scipy's Euclidean
+    distances), and round T's centroids are the fp32 means of those members; the single
+    steps compose into the whole k-means."""
+    from scipy.spatial.distance import cdist
     rng = np.random.default_rng(3)
     x = rng.standard_normal((800, 32)).astype(np.float32)
     C = 12
     prev, _, _ = oracle.kmeans(x, C, 2)
     cent, label, count = oracle.kmeans(x, C, 3)
-    x64, p64 = x.astype(np.float64), prev.astype(np.float64)
-    dist = (x64 ** 2).sum(1)[:, None] + (p64 ** 2).sum(1)[None, :] - 2.0 * x64 @ p64.T
-    tol = 1e-5 * ((x64 ** 2).sum(1) + (p64 ** 2).sum(1).max())
-    assert np.all(dist[np.arange(len(x)), label] <= dist.min(axis=1) + tol)
+    dist = cdist(x.astype(np.float64), prev.astype(np.float64))
+    assert np.array_equal(label, np.argmin(dist, axis=1))
     assert np.array_equal(count, np.bincount(label, minlength=C))
     for j in range(C):
         if count[j]:
             np.testing.assert_array_max_ulp(cent[j], _fp32_mean(x[label == j]), maxulp=1)
         else:
             assert np.array_equal(cent[j], prev[j])
+    # the exposed steps: assign against round 2's centroids, update from those labels
+    lab, gap = oracle.kmeans_assign(x, prev)
+    assert np.array_equal(lab, label)
+    srt = np.sort(dist ** 2, axis=1)
+    np.testing.assert_allclose(gap, srt[:, 1] - srt[:, 0], rtol=1e-9, atol=1e-12)
+    c2, n2 = oracle.kmeans_update(x, lab, prev)
+    assert np.array_equal(c2.view(np.uint32), cent.view(np.uint32)) and np.array_equal(n2, count)
+    c0 = oracle.kmeans_init(x, C)
+    assert np.array_equal(c0, x[[(2 * j + 1) * 800 // (2 * C) for j in range(C)]])
+
+
+def test_kmeans_assignment_is_exact():
+    """Centroids 1 and 1 + 2^-21 and the row 1 + 3*2^-23 (all exact in fp32): the second
+    centroid is nearer (2^-23 against 3*2^-23), a gap that fp32's |c|^2 - 2 x.c form rounds
+    to a tie (which would pick the first); the oracle's fp64 distances resolve it."""
+    x = np.array([[1.0 + 3 * 2.0 ** -23], [1.0], [5.0], [1.0 + 2.0 ** -21]], dtype=np.float32)
+    assert float(x[0, 0]) == 1.0 + 3 * 2.0 ** -23 and float(x[3, 0]) == 1.0 + 2.0 ** -21
+    # the fp32 form of the distance ties
+    c = x[[1, 3], 0]
+    two = np.float32(2.0)
+    d32 = [np.float32(cj * cj) - np.float32(two * np.float32(x[0, 0] * cj)) for cj in c]
+    assert d32[0] == d32[1]
+    cent, label, count = oracle.kmeans(x, 2, 1)      # initial centroids: rows 1 and 3
+    assert label[0] == 1 and label[1] == 0 and label[3] == 1 and label[2] == 1
 
 
 def test_kmeans_ties_and_empty_clusters():
@@ -263,3 +270,14 @@ def test_semantic_head_token_level_brute_force():
     p = np.exp(s - s.max(axis=1, keepdims=True))
     want = (p / p.sum(axis=1, keepdims=True)) @ v.numpy()
     np.testing.assert_allclose(res["out"], want, atol=1e-12, rtol=0)
+
+
+def test_semantic_weights_match_numpy():
+    """The exposed criticality weights equal numpy's n_j exp(s_ij - max_j s_ij); empty
+    clusters are marked -1; the top-p rows are built from these weights."""
+    cq, nq, ck, nk = _centroids(13)
+    w = oracle.semantic_weights(cq, nq, ck, nk, 0.5)
+    want = _weights(cq, ck, nk, 0.5)
+    live = (nq[:, None] > 0) & (nk[None, :] > 0)
+    np.testing.assert_allclose(w[live], want[live], rtol=1e-13, atol=0)
+    assert np.all(w[~live] == -1.0)
