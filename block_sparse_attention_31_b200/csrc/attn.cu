@@ -5,19 +5,24 @@
 // compatible with FlashAttention kernels; "Sparse Video-Gen" summary, "Approach": block-wise
 // spatial and temporal masks).  Online softmax in the base-2 domain, fp32 accumulation.
 //
-// One CTA per pair of consecutive query blocks of a head (tiles 0 and 1), 320 threads:
-//   warp 0  (one lane)  TMA producer: both Q tiles once, then K and V of every key block in
-//                       the union of the two lists through a 2-stage ring (each K/V tile is
-//                       loaded once and serves both query tiles)
-//   warp 1  (one lane)  tcgen05 issuer, per union entry: P.V of tile 0's previous block, Q.K^T
-//                       of tile 0, then the same for tile 1; the tensor core works on one tile
-//                       while the other tile's softmax runs.  Warp 1 also owns TMEM.
-//   warps 2-5 / 6-9     softmax of tile 0 / tile 1, one query row per thread (TMEM lane = row):
-//                       S from TMEM, online max in the base-2 domain with lazy rescaling of O
-//                       (only when the max grows by more than 2^16), P = exp2(S*scale*log2e - m)
-//                       written as packed bf16 over the tile's S columns in TMEM, where the
-//                       P.V MMA reads it; at the end O / l goes through shared memory to a TMA
-//                       store.
+// One CTA per pair of query blocks of a head (tiles 0 and 1), 384 threads in three
+// warpgroups whose registers are rebalanced at the start (setmaxnreg: the softmax warpgroups
+// grow to kRegsSoftmax, the control warpgroup shrinks to kRegsCtl; the sum equals the launch's):
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1, one query row per thread (TMEM lane = row):
+//                    all of a key block's scores are read from TMEM with one wait, then the
+//                    row max, the lazy rescale of O (only when the max grows by more than
+//                    2^16), and P = exp2(S*scale*log2e - m) written as packed bf16 over the
+//                    tile's S columns in TMEM in two halves, each announced on its own
+//                    barrier so that the P.V of the first half overlaps the exponentials of
+//                    the second; at the end O / l goes through shared memory to a TMA store.
+//   warp 8 (one lane) TMA producer: both Q tiles once, then K and V of every key block in the
+//                    union of the two lists through a 2-stage ring (each K/V tile is loaded
+//                    once and serves both query tiles); with the in-kernel layout warp 8
+//                    gathers Q and K rows and warp 10 gathers V rows instead.
+//   warp 9 (one lane) tcgen05 issuer, per union entry: P.V of tile 0's previous block (first
+//                    half as soon as it is written), Q.K^T of tile 0, then the same for tile
+//                    1; the tensor core works on one tile while the other tile's softmax runs.
+//                    Warp 9 also owns TMEM.
 // TMEM: S0, S1 (BN columns each), O0, O1 (D columns each).
 //
 // Shared-memory operand tiles use the 128-byte swizzle (TMA SWIZZLE_128B == UMMA SWIZZLE_128B):
@@ -34,10 +39,16 @@
 
 namespace vsa {
 
-// warp 0 TMA (or Q and K gather), warp 1 MMA, warps 2-5 softmax tile 0, 6-9 tile 1, and for the
-// in-kernel layout warp 10 (V gather)
-constexpr int kAttnThreads = 320, kAttnThreadsGather = 352;
+// warps 0-3 softmax tile 0, 4-7 tile 1; warp 8 TMA (or Q and K gather), warp 9 MMA, warp 10 V
+// gather (in-kernel layout only), warp 11 idle
+constexpr int kAttnThreads = 384;
+constexpr int kWarpLoad = 8, kWarpMma = 9, kWarpVGather = 10;
 constexpr int kBM = 128;           // MMA M: query rows per tile
+// Register split: 384 threads launch with 168 registers each (64,512 in all); the control
+// warpgroup gives up 80 per thread and the two softmax warpgroups take 40 more each:
+// 2 * 128 * 208 + 128 * 88 = 64,512 (88 keeps the producer and issuer code free of spills).
+constexpr int kRegsSoftmax = 208, kRegsCtl = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl == 384 * 168, "register split must equal the launch total");
 
 template <int D, int BN>
 struct AttnCfg {
@@ -69,7 +80,8 @@ enum {
   B_S_FULL = 10,   // +tile
   B_P_FULL = 12,   // +tile
   B_O_FINAL = 14,  // +tile
-  B_DRAIN = 16
+  B_DRAIN = 16,
+  B_P_HALF = 17    // +tile: first half of P (keys 0..BN/2-1) written
 };
 constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kPartial = 1u << 29, kKbMask = (1u << 29) - 1u;
 // Probability pairs (2 columns) whose exponentials run on the FMA pipe: kPolyPairs8 in 8.
@@ -84,7 +96,7 @@ constexpr int kPolyPairs8 = VSA_POLY_PAIRS8;
 // tile) so the tensor core works on one tile while the other tile's softmax runs.  P is
 // written as packed bf16 over the tile's S columns in TMEM and read from there by the P.V MMA.
 template <int D, int BN>
-__global__ void __launch_bounds__(kAttnThreadsGather, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tq_n, const __grid_constant__ CUtensorMap tk_n,
                            const __grid_constant__ CUtensorMap tv_n, const __grid_constant__ CUtensorMap to_n,
                            const __grid_constant__ CUtensorMap tq_p, const __grid_constant__ CUtensorMap tk_p,
@@ -254,6 +266,7 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       mbar_init(bar(B_Q + t), nload);
       mbar_init(bar(B_S_FULL + t), 1);
       mbar_init(bar(B_P_FULL + t), 128);
+      mbar_init(bar(B_P_HALF + t), 128);
       mbar_init(bar(B_O_FINAL + t), 1);
     }
     for (int st = 0; st < C::NS; ++st) {
@@ -270,7 +283,7 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
     tma_prefetch_desc(tv);
     tma_prefetch_desc(to);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -280,9 +293,11 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int U = misc[2];
 
-  if ((warp == 0 || warp == 10) && gather) {
+  if (warp >= 8) {
+  setmaxnreg_dec<kRegsCtl>();
+  if ((warp == kWarpLoad || warp == kWarpVGather) && gather) {
     // ================= gather producers (temporal head, natural-order buffers) =================
-    // Warp 0 copies the Q and K tiles, warp 10 the V tiles, 16 bytes per copy: slot p of the
+    // Warp 8 copies the Q and K tiles, warp 10 the V tiles, 16 bytes per copy: slot p of the
     // frame-major layout is token (p % F) * S + p / F; copies land in the 128-byte-swizzled
     // layout a TMA tile load would produce, slots past N are zero-filled.  Each lane's copies
     // signal the stage's barrier when they land.  Lane l owns 16-byte column c = l % CPR of rows
@@ -317,16 +332,17 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       const __nv_bfloat16* gk = static_cast<const __nv_bfloat16*>(a.nat_k) + head;
       const __nv_bfloat16* gv = static_cast<const __nv_bfloat16*>(a.nat_v) + head;
       const int cnts[2] = {cnt0, cnt1};
-      if (warp == 0) {
+      const bool qk = warp == kWarpLoad;
+      if (qk) {
         for (int t = 0; t < 2; ++t) {
           if (cnts[t] == 0) continue;
           gather_tile(sbase + C::OFF_Q + t * C::Q_BYTES, kBM, (t ? qb1 : qb0) * BN, gq);
           cp_async_mbar_arrive_noinc(bar(B_Q + t));
         }
       }
-      const int eb = warp == 0 ? B_EMPTY_K : B_EMPTY_V, fb = warp == 0 ? B_FULL_K : B_FULL_V;
-      const uint32_t sdst0 = warp == 0 ? sK : sV;
-      const __nv_bfloat16* gsrc = warp == 0 ? gk : gv;
+      const int eb = qk ? B_EMPTY_K : B_EMPTY_V, fb = qk ? B_FULL_K : B_FULL_V;
+      const uint32_t sdst0 = qk ? sK : sV;
+      const __nv_bfloat16* gsrc = qk ? gk : gv;
       for (int n = 0; n < U; ++n) {
         const int st = n % C::NS;
         const uint32_t u = n / C::NS;
@@ -339,7 +355,7 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncwarp();
-  } else if (warp == 0) {
+  } else if (warp == kWarpLoad) {
     // ================= TMA producer =================
     if (lane == 0 && U > 0) {
       int nk = 0, nv = 0;  // copies issued
@@ -383,7 +399,7 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ================= tcgen05 issuer =================
     if (lane == 0 && U > 0) {
       const int cnts[2] = {cnt0, cnt1};
@@ -398,9 +414,11 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       const uint64_t dq1 = sdesc_sw128(sbase + C::OFF_Q + C::Q_BYTES, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::KV_BYTES, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::KV_BYTES, BN * 128, 1024);
+      // P.V of tile t's pending block: the first half of the keys as soon as its P is written,
+      // the second half after the rest
       auto issue_pv = [&](int t) -> bool {
         const int np = pend[t];
-        if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
+        if (!mbar_wait(bar(B_P_HALF + t), pvc[t] & 1, abort_flag, a.err)) return false;
         if (!mbar_wait(bar(B_FULL_V + np % C::NS), (np / C::NS) & 1, abort_flag, a.err)) return false;
         if (gather) fence_proxy_async_smem();  // cp.async data, written by the generic proxy
         tc_fence_after();
@@ -408,7 +426,12 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
         const uint32_t d_o = tmem + C::TMEM_O + t * D, a_p = tmem + C::TMEM_S + t * BN;
         tc_mma_ts(d_o, a_p, vd, C::IDESC_PV, pvc[t] > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < BN / 16; ++kk)
+        for (int kk = 1; kk < BN / 32; ++kk)
+          tc_mma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV, 1u);
+        if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = BN / 32; kk < BN / 16; ++kk)
           tc_mma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV, 1u);
         pend[t] = -1;
         if (++pvc[t] == cnts[t]) tc_commit(bar(B_O_FINAL + t));
@@ -458,9 +481,11 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
       mbar_wait_drain(bar(B_DRAIN), 0, a.err);
     }
     __syncwarp();
-  } else if (warp < 10) {
-    // ================= softmax: warps 2-5 tile 0, warps 6-9 tile 1; one row per thread =================
-    const int t = (warp - 2) >> 2;
+  }
+  } else {
+    // ================= softmax: warps 0-3 tile 0, warps 4-7 tile 1; one row per thread =================
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int t = warp >> 2;
     const int quad = warp & 3;          // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;   // query row within the tile
     if (t == 0 || has1) {
@@ -479,40 +504,34 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
         while (!(uni[cur] & tbit)) ++cur;
         const uint32_t ent = uni[cur];
         tc_fence_after();
-        if (ent & kPartial) {  // same block for every row: mask invalid key columns to -inf in TMEM
-#pragma unroll 1
+        // every score of the row with one wait
+        uint32_t r[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32_async(t_s + c * 32, r + c * 32);
+        tmem_wait_ld();
+        reg_fence<BN>(r);
+        if (ent & kPartial) {  // same block for every row: invalid key columns (tail, padding) -> -inf
+#pragma unroll
           for (int w = 0; w < BN / 32; ++w) {
             const uint32_t vb = uvalid[cur * (BN / 32) + w];
-            if (vb == 0xffffffffu) continue;
-            float v[32];
-            tmem_ld32(t_s + w * 32, v);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = ((vb >> x) & 1u) ? v[x] : -INFINITY;
-            tmem_st32(t_s + w * 32, v);
+            for (int x = 0; x < 32; ++x) r[w * 32 + x] = ((vb >> x) & 1u) ? r[w * 32 + x] : 0xff800000u;
           }
         }
         ++cur;
-        // pass 1: row max, 64 columns per wait; eight independent partial maxima keep the
-        // dependency chains short
+        // row max: eight independent partial maxima keep the dependency chains short
         float mx8[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {
-          uint32_t r[64];
-          tmem_ld32_async(t_s + h * 64, r);
-          tmem_ld32_async(t_s + h * 64 + 32, r + 32);
-          tmem_wait_ld();
-          reg_fence<64>(r);
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
-        }
+        for (int c = 0; c < BN / 2; ++c)
+          mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m, mx * sl2);
         // Rescale only when the running max grows by more than 2^kRescaleLog2; otherwise keep the
-        // old max (the final 1/l normalisation is exact either way).
+        // old max (the final 1/l normalisation is exact either way).  O is stable here: the
+        // Q.K^T whose completion signalled S was issued after the previous P.V of this tile.
         const bool grow = m_new > m + kRescaleLog2;
         if (k > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
           const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
@@ -530,38 +549,38 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
           m = m_new;
         }
         const float m_use = m == -INFINITY ? 0.f : m;
-        // pass 2: 64 scores at a time -> 32 packed bf16 pairs written over the consumed S columns;
-        // the row sum is kept in eight partial sums
-        // (scale and max subtraction, row sums and the polynomial exponentials on packed pairs)
+        // exponentials in two halves of the keys: each half's packed bf16 P goes over the
+        // consumed S columns and is announced on its own barrier, so the P.V of the first half
+        // runs while the second half is computed (scale and max subtraction, row sums and the
+        // polynomial exponentials on packed pairs)
         uint64_t rs4[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) rs4[x] = 0ull;
         const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
 #pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {
-          uint32_t r[64];
-          tmem_ld32_async(t_s + h * 64, r);
-          tmem_ld32_async(t_s + h * 64 + 32, r + 32);
-          tmem_wait_ld();
-          reg_fence<64>(r);
-          uint32_t pk[32];
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[BN / 4];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const uint64_t x = f2_fma(f2_make(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2x2, negm2);
+          for (int c = 0; c < BN / 4; ++c) {
+            const int cc = hf * (BN / 4) + c;  // key pair
+            const uint64_t x =
+                f2_fma(f2_make(__uint_as_float(r[2 * cc]), __uint_as_float(r[2 * cc + 1])), sl2x2, negm2);
             uint64_t p;
-            if ((c & 7) >= 8 - kPolyPairs8) {
+            if ((cc & 7) >= 8 - kPolyPairs8) {
               p = exp2_poly2(x);
             } else {
               float x0, x1;
               f2_split(x, x0, x1);
               p = f2_make(fast_exp2(x0), fast_exp2(x1));
             }
-            rs4[c & 3] = f2_add(rs4[c & 3], p);
+            rs4[cc & 3] = f2_add(rs4[cc & 3], p);
             float p0, p1;
             f2_split(p, p0, p1);
             pk[c] = pack_bf16x2(p0, p1);
           }
-          tmem_st32_u(t_s + h * 32, pk);
+          tmem_st_cols<BN / 4>(t_s + hf * (BN / 4), pk);
+          tc_fence_before();
+          mbar_arrive(bar((hf ? B_P_FULL : B_P_HALF) + t));
         }
         {
           const uint64_t s2 = f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3]));
@@ -569,8 +588,6 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
           f2_split(s2, s0, s1);
           l += s0 + s1;
         }
-        tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + t));
       }
       // ---- epilogue: O / l -> bf16 -> swizzled smem (over this tile's Q) -> TMA store ----
       if (ok && cnt > 0) {
@@ -633,7 +650,7 @@ __global__ void __launch_bounds__(kAttnThreadsGather, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == kWarpMma) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 template <int D, int BN>
@@ -647,7 +664,7 @@ static cudaError_t launch_attn_t(const AttnMaps& nat, const AttnMaps& perm, cons
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(a.BH) * ((a.g.nblk + 1) / 2);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), a.gather ? kAttnThreadsGather : kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
+  kern<<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
                                                                      perm.v, perm.o, a);
   return cudaGetLastError();
 }

@@ -203,11 +203,12 @@ __device__ __forceinline__ void set_bit_range(uint32_t (&m)[BN / 32], int lo, in
 // The spatial P.V reads the dense P with the rows outside the window disabled (the MMA's
 // output-lane mask); the temporal P.V reads a masked copy with rows that allow no key of the
 // block disabled.  Probabilities more than 2^126 below the running dense maximum flush to
-// zero, so each row also tracks the largest logit each masked variant allows: when that is
-// more than kProfFlushMargin (base 2) below the dense maximum, the variant's partial sum could
-// have lost weight to the flush, and the split marks it (l = -1) for the row-error kernel,
-// which then recomputes that variant of the row with its own maximum.  Both P tiles live in
-// shared memory so that Q.K^T of block j+1 runs while the softmax of block j computes.
+// zero, so each row also tracks the largest logit each masked variant allows in this split
+// and stores it as that variant's partial max (the dense partial max is the exponent base of
+// all three); the row-error kernel recomputes a variant with its own maximum when the
+// variant's largest logit over all splits lies more than kProfFlushMargin (base 2) below the
+// dense max of a split where the variant has keys.  Both P tiles live in shared memory so
+// that Q.K^T of block j+1 runs while the softmax of block j computes.
 template <int D, int BN>
 __global__ void __launch_bounds__(kProfThreads, 1)
     profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
@@ -530,18 +531,16 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
       tc_fence_after();
     }
-    // partials: (m, l) and unnormalised O of each variant; l = -1 marks a masked variant
-    // whose allowed logits all sit more than kProfFlushMargin below the dense maximum
+    // partials: the dense max m (the exponent base of all three variants) in the dense row,
+    // each masked variant's own largest allowed logit in its row, the sums l and the
+    // unnormalised O of each variant
     const size_t base = ((static_cast<size_t>(bh) * a.splits + split) * 3) * a.r_pad + tile * kPM + row;
-    const bool low_s = mv_s != -INFINITY && mv_s < m - kProfFlushMargin;
-    const bool low_t = mv_t != -INFINITY && mv_t < m - kProfFlushMargin;
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
       const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
       const bool have = ok && cnt > 0;
-      const bool low = vv == 1 ? low_s : vv == 2 ? low_t : false;
-      a.ml[prow * 2 + 0] = have ? m : -INFINITY;
-      a.ml[prow * 2 + 1] = have ? (low ? -1.f : l[vv]) : 0.f;
+      a.ml[prow * 2 + 0] = have ? (vv == 0 ? m : vv == 1 ? mv_s : mv_t) : -INFINITY;
+      a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
       float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -623,7 +622,11 @@ __device__ float profile_variant_exact(const __nv_bfloat16* __restrict__ qrow, c
 
 // Merge the key splits of one sampled row of one head and accumulate its two squared errors
 // (one CTA of d threads per (row, head)); the per-row sums are reduced in fixed order below.
-// A masked variant that any split marked (l = -1) is recomputed with its own maximum.
+// A split's sums are based on its dense max md; a masked variant's stored max is its own
+// largest allowed logit mv.  When the variant's largest logit over all splits, M_v, lies more
+// than kProfFlushMargin below md of a split where the variant has keys, that split's flush
+// at 2^-126 of md may have removed probabilities above 2^-46 of the variant's own maximum,
+// so the variant of this row is recomputed with its own maximum.
 __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __restrict__ opart,
                                                                 const float* __restrict__ ml, int r_pad,
                                                                 int splits, int d, double* __restrict__ row_err,
@@ -638,20 +641,26 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
 #pragma unroll
   for (int vv = 0; vv < 3; ++vv) {
     // all splits' partials are loaded before they are combined (at most kMaxSplits)
-    float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
-    bool low = false;
+    float ms[kMaxSplits], mv[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
+    float Mv = -INFINITY;
 #pragma unroll
     for (int sp = 0; sp < kMaxSplits; ++sp) {
-      ms[sp] = -INFINITY;
+      ms[sp] = mv[sp] = -INFINITY;
       ls[sp] = os[sp] = 0.f;
       if (sp < splits) {
         const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-        ms[sp] = __ldg(ml + prow * 2);
+        const size_t drow = ((static_cast<size_t>(bh) * splits + sp) * 3) * r_pad + i;
+        ms[sp] = __ldg(ml + drow * 2);  // the split's dense max: the base of its sums
+        mv[sp] = __ldg(ml + prow * 2);  // the variant's own largest logit (the dense max for vv 0)
         ls[sp] = __ldg(ml + prow * 2 + 1);
         os[sp] = __ldg(opart + prow * d + x);
-        low |= ls[sp] < 0.f;
+        Mv = fmaxf(Mv, mv[sp]);
       }
     }
+    bool low = false;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+      low |= vv > 0 && mv[sp] != -INFINITY && Mv < ms[sp] - kProfFlushMargin;
     if (low) {  // uniform across the CTA: every thread read the same (m, l) partials
       const int4 rg = ranges[i];
       const bool tp = vv == 2;
@@ -660,13 +669,16 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
                                     tp ? rg.z : rg.x, tp ? rg.w : rg.y, tp, g, d, scale_log2);
       continue;
     }
+    // reference: the largest dense max among the splits where the variant has keys, so that
+    // the variant's scaled sums stay far above the fp32 range's bottom
     float M = -INFINITY;
 #pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) M = fmaxf(M, ms[sp]);
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+      if (mv[sp] != -INFINITY) M = fmaxf(M, ms[sp]);
     float L = 0.f, acc = 0.f;
 #pragma unroll
     for (int sp = 0; sp < kMaxSplits; ++sp) {
-      if (ms[sp] == -INFINITY) continue;
+      if (mv[sp] == -INFINITY) continue;
       const float w = exp2f(ms[sp] - M);
       L += ls[sp] * w;
       acc += os[sp] * w;

@@ -72,6 +72,10 @@ def _load():
         lib.or_semantic_weights.argtypes = [vp, vp, i64, vp, vp, i64, i64, dbl, vp]
         lib.or_semantic_keep.restype = None
         lib.or_semantic_keep.argtypes = [vp, vp, i64, vp, vp, i64, i64, dbl, dbl, vp]
+        lib.or_e4m3_value.restype = dbl
+        lib.or_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.or_quantize_e4m3.restype = None
+        lib.or_quantize_e4m3.argtypes = [vp, i64, i64, i64, vp, vp]
         lib.or_profile_rows.restype = i64
         lib.or_profile_rows.argtypes = [i64, dbl]
         lib.or_profile_head.restype = ctypes.c_int
@@ -315,6 +319,42 @@ def semantic_head(q, k, v, cq: int, ck: int, iters: int, top_p: float, block: in
                                   scale=None if scale <= 0 else scale)
         res.update(out=out, lse=lse)
     return res
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 Q and K (Sparse Video-Gen summary page, "Measured effects": FP8 quantisation); the
+# readings are stated in vsa_oracle.c.
+# ---------------------------------------------------------------------------------------
+
+def quantize_e4m3(x, block: int):
+    """Per-block e4m3 quantisation of one head's rows x [rows, d]: (codes uint8 [rows, d],
+    scale exponents int32 [ceil(rows / block)])."""
+    x = _f64(x)
+    rows, d = x.shape
+    code = np.empty((rows, d), dtype=np.uint8)
+    exp = np.empty(-(-rows // block), dtype=np.int32)
+    _load().or_quantize_e4m3(_p(x), rows, d, block, _p(code), _p(exp))
+    return code, exp
+
+
+_E4M3_TABLE = None
+
+
+def e4m3_values(code) -> np.ndarray:
+    """fp64 values of e4m3 codes."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        lib = _load()
+        _E4M3_TABLE = np.array([lib.or_e4m3_value(c) for c in range(256)], dtype=np.float64)
+    return _E4M3_TABLE[np.asarray(code, dtype=np.uint8)]
+
+
+def dequantize_e4m3(code, exp, block: int) -> np.ndarray:
+    """The values the codes stand for: e4m3(code) * 2^e of the row's block."""
+    v = e4m3_values(code)
+    rows = v.shape[0]
+    e = np.repeat(np.asarray(exp, dtype=np.int64), block)[:rows]
+    return np.ldexp(v, e[:, None])
 
 
 # ---------------------------------------------------------------------------------------

@@ -490,3 +490,62 @@ void or_semantic_keep(const float *cq, const int32_t *nq, int64_t Cq, const floa
         free(order); free(w); free(used);
     }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * FP8 Q and K ("Sparse Video-Gen" summary page, "Measured effects": FP8 quantisation on top
+ * of the sparse attention).  The page gives no format details; the readings used here:
+ *   - e4m3 values (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest 448,
+ *     subnormals down to 2^-9), round to nearest with ties to even;
+ *   - one scale per block of `block` rows of a head's layout: the smallest power of two 2^e
+ *     with max |x| <= 448 * 2^e over the block (e = 0 for an all-zero block); the stored code
+ *     is e4m3(x / 2^e) and the value it stands for is e4m3(x / 2^e) * 2^e.
+ * ------------------------------------------------------------------------------------- */
+
+/* e4m3 code of y (|y| <= 448), rounded to the nearest value, ties to even. */
+static uint8_t e4m3_code(double y)
+{
+    uint8_t sign = (y < 0.0 || (y == 0.0 && signbit(y))) ? 0x80 : 0x00;
+    double a = fabs(y);
+    if (a < ldexp(1.0, -6)) {                       /* subnormal range: spacing 2^-9 */
+        double m = nearbyint(a / ldexp(1.0, -9));  /* 0..8; 8 is the smallest normal */
+        if (m >= 8.0) return (uint8_t)(sign | (1 << 3));
+        return (uint8_t)(sign | (int)m);
+    }
+    int E = (int)floor(log2(a));
+    if (ldexp(1.0, E) > a) E -= 1;                  /* guard log2 rounding */
+    if (ldexp(1.0, E + 1) <= a) E += 1;
+    double m = nearbyint(a / ldexp(1.0, E - 3));    /* 8..16 */
+    if (m >= 16.0) { m = 8.0; E += 1; }
+    return (uint8_t)(sign | ((E + 7) << 3) | ((int)m - 8));
+}
+
+/* Value of an e4m3 code. */
+double or_e4m3_value(uint8_t c)
+{
+    int e = (c >> 3) & 0xF, m = c & 7;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/*
+ * Quantise one head's rows x [rows, d] in blocks of `block` rows: code [rows, d] (e4m3) and
+ * scale_exp [ceil(rows / block)] (the block's power-of-two exponent e).
+ */
+void or_quantize_e4m3(const double *x, int64_t rows, int64_t d, int64_t block, uint8_t *code, int32_t *scale_exp)
+{
+    int64_t nb = ceil_div(rows, block);
+    for (int64_t b = 0; b < nb; ++b) {
+        int64_t r0 = b * block, r1 = (b + 1) * block < rows ? (b + 1) * block : rows;
+        double amax = 0.0;
+        for (int64_t i = r0 * d; i < r1 * d; ++i)
+            if (fabs(x[i]) > amax) amax = fabs(x[i]);
+        int e = 0;
+        if (amax > 0.0) {
+            e = (int)ceil(log2(amax / 448.0)) - 1;
+            while (amax > 448.0 * ldexp(1.0, e)) ++e;     /* smallest e with amax <= 448 * 2^e */
+            while (amax <= 448.0 * ldexp(1.0, e - 1)) --e;
+        }
+        scale_exp[b] = e;
+        for (int64_t i = r0 * d; i < r1 * d; ++i) code[i] = e4m3_code(ldexp(x[i], -e));
+    }
+}
