@@ -145,6 +145,8 @@ def stage_work(wl, kinds, pipe, pairs):
     # one of the R slots (padding zeroed); spatial bf16 heads are read in place (no copy)
     n_tc = 0 if pipe.in_kernel else n_t  # temporal heads copied (not gathered in the kernel)
     perm = 3.0 * (n_tc * 2 * N + n_c * (N + R)) * row
+    if getattr(pipe, "qk_fp8", False):  # e4m3 codes of Q and K: read bf16 rows, write one byte each
+        perm += 2.0 * BH * R * (row + d)
     unperm = (n_tc + n_c) * 2.0 * N * row
     nwords = -(-pipe.nblk // 32)
     mask = BH * pipe.nblk * (nwords + pipe.max_kv + 1) * 4.0
@@ -292,10 +294,11 @@ class ClockSampler:
 class Pipeline:
     """Buffers for the stage-by-stage path through the public entry points."""
 
-    def __init__(self, wl, device, in_kernel=False):
+    def __init__(self, wl, device, in_kernel=False, qk_fp8=False):
         import block_sparse_attention_31_b200 as vsa
         from block_sparse_attention_31_b200 import _lib
         self.vsa, self.lib, self.wl, self.dev = vsa, _lib, wl, device
+        self.qk_fp8 = bool(qk_fp8)
         self.in_kernel = bool(in_kernel) and wl.mode != "cube"  # cube heads always use their copies
         cube = wl.cube if wl.mode == "cube" else None
         self.shape = _lib.make_shape(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, cube)
@@ -330,7 +333,13 @@ class Pipeline:
         self.order = (torch.empty(wl.B * wl.H * self.nblk, dtype=torch.int32, device=device)
                       if wl.mode == "cube" else None)
         cube = wl.mode == "cube"
-        self.launches = ((4 if wl.mode == "profiled" else 0)                 # prep, attn3, row error, reduce
+        if self.qk_fp8:  # e4m3 codes of Q and K in every head's layout, one exponent per block
+            self.q8 = torch.empty(wl.B, wl.H, self.R, wl.d, dtype=torch.uint8, device=device)
+            self.k8 = torch.empty_like(self.q8)
+            self.qe = torch.empty(BH, self.nblk, dtype=torch.int32, device=device)
+            self.ke = torch.empty_like(self.qe)
+        self.launches = ((2 if self.qk_fp8 else 0)                          # quantise Q and K
+                         + (4 if wl.mode == "profiled" else 0)                 # prep, attn3, row error, reduce
                          + (0 if self.in_kernel else 6 if cube else 3)        # permutes
                          + (5 if cube else 1)                                 # masks (+ pool, score, top-k, order)
                          + 1                                                  # attention
@@ -348,6 +357,9 @@ class Pipeline:
         if not self.in_kernel:
             for src, dst in ((q, self.qp), (k, self.kp), (v, self.vp)):
                 L.vsa_permute(src, L.VSA_BF16, dst, self.kinds, self.shape, self.err, s)
+        if self.qk_fp8:  # the e4m3 codes of Q and K count with the layouts
+            L.vsa_quantize_fp8(q, self.qp, self.kinds, self.shape, self.q8, self.qe, self.err, s)
+            L.vsa_quantize_fp8(k, self.kp, self.kinds, self.shape, self.k8, self.ke, self.err, s)
         if ev is not None:
             ev[2].record()
         L.vsa_build_mask(self.kinds, self.qp, self.kp, self.shape, self.params, self.bits, self.kv_idx, self.kv_cnt,
@@ -356,7 +368,11 @@ class Pipeline:
             L.vsa_block_order(self.kinds, self.kv_idx, self.kv_cnt, self.max_kv, self.shape, self.order, s)
         if ev is not None:
             ev[3].record()
-        if self.in_kernel:  # temporal heads gathered through the frame-major map inside the kernel
+        if self.qk_fp8:
+            L.vsa_sparse_attn_fwd_fp8qk(L.qkvo(q, k, v, o), L.qkvo(self.qp, self.kp, self.vp, self.op), self.q8,
+                                        self.qe, self.k8, self.ke, self.kinds, self.kv_idx, self.kv_cnt, self.max_kv,
+                                        self.shape, 0.0, self.err, s, order=self.order)
+        elif self.in_kernel:  # temporal heads gathered through the frame-major map inside the kernel
             L.vsa_sparse_attn_fwd_natural(L.qkvo(q, k, v, o), self.kinds, self.kv_idx, self.kv_cnt, self.max_kv,
                                           self.shape, 0.0, self.err, s)
         else:
@@ -435,8 +451,10 @@ class SemanticPipeline:
             ev[5].record()
 
 
-def make_pipeline(wl, device, in_kernel=False):
-    return SemanticPipeline(wl, device) if wl.mode == "semantic" else Pipeline(wl, device, in_kernel=in_kernel)
+def make_pipeline(wl, device, in_kernel=False, qk_fp8=False):
+    if wl.mode == "semantic":
+        return SemanticPipeline(wl, device)
+    return Pipeline(wl, device, in_kernel=in_kernel, qk_fp8=qk_fp8)
 
 
 STAGES = ("profile", "permute", "mask", "attention", "unpermute")
@@ -466,7 +484,7 @@ def gpu_arm(args, wl, rank, world, device):
     q, k, v = synthetic.make_qkv(wl, seed=rank_seed(wl.seed, rank))
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     o = torch.empty_like(qd)
-    pipe = make_pipeline(wl, device, in_kernel=args.layout == "kernel")
+    pipe = make_pipeline(wl, device, in_kernel=args.layout == "kernel", qk_fp8=args.qk == "fp8")
     for _ in range(args.warmup):
         pipe.step(qd, kd, vd, o)
     torch.cuda.synchronize()
@@ -518,7 +536,8 @@ def e2e_arm(args, wl, q, k, v, device):
                                      ck=wl.clusters[1], iters=wl.kmeans_iters, top_p=wl.top_p, device=device)
         return _e2e_run(args, plan, q, k, v, None, "SemanticAttention.run_host")
     select = {"profiled": "profile", "fixed": "given", "cube": "cube"}[wl.mode]
-    kw = dict(select=select, dtype=q.dtype, device=device, layout_in_kernel=args.layout == "kernel")
+    kw = dict(select=select, dtype=q.dtype, device=device, layout_in_kernel=args.layout == "kernel",
+              qk_fp8=args.qk == "fp8")
     if wl.mode == "profiled":
         kw.update(target=wl.target, profile_frac=wl.profile_frac)
     elif wl.mode == "cube":
@@ -650,6 +669,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qk", default="bf16", choices=["bf16", "fp8"],
+                    help="Q.K^T in bf16, or on e4m3 codes with one power-of-two scale per block (P.V stays bf16)")
     ap.add_argument("--layout", default="copies", choices=["copies", "kernel"],
                     help="temporal heads: permuted into copies (faster at these sizes), or gathered inside "
                          "the attention kernel")
@@ -681,12 +702,22 @@ def main():
     peak_burst = float(peaks["bf16_tflops"])
     attn_s = res["stage_ms"]["attention"] / 1e3
     achieved = res["alg"] / attn_s / 1e12
+    # e4m3 Q.K^T: half the flops (Q.K^T) run at twice the bf16 rate (the nominal fp8 / bf16 ratio,
+    # 4.5 / 2.25), the other half (P.V) at the bf16 rate, so the attention's peak is the bf16
+    # peak / 0.75 (derived, not measured)
+    fp8 = args.qk == "fp8"
+    qk_factor = 1.0 / 0.75 if fp8 else 1.0
+    attn_peak, attn_peak_sust = peak_burst * qk_factor, peak_sust * qk_factor
+    attn_peak_src = (f"derived: {src} bf16_tflops (burst) / 0.75, Q.K^T at twice the bf16 rate (nominal "
+                     "fp8/bf16 ratio 4.5/2.25), P.V at the bf16 rate" if fp8 else
+                     f"{src} bf16_tflops (burst; the kernel runs at the maximum SM clock, see clocks)")
     value = aggregate_tflops(res["alg"], res["ms"], world)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["ms"], "ms_per_call": res["ms"], "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.F, wl.Hl, wl.Wl], "d": wl.d,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16, Q.K^T e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": wl.name + (", Q.K^T e4m3 per-block scales" if fp8 else ""), "B": wl.B, "H": wl.H,
+                   "grid": [wl.F, wl.Hl, wl.Wl], "d": wl.d,
                    "block": wl.block, "mode": wl.mode, "w_s": res["w_s"], "w_t": res["w_t"],
                    "kept_block_fraction": res["kept"], "head_kinds": res["kinds"],
                    "layout": ("cluster-major copies (Q by its k-means clusters, K and V by theirs)"
@@ -703,14 +734,13 @@ def main():
                             "(4*d*valid_q*valid_k per kept pair) / ms per call, summed over ranks",
         "dense_equiv_tflops": aggregate_tflops(res["dense"], res["ms"], world),
         "stage_ms": res["stage_ms"],
-        "roofline": {"kernel": "vsa_sparse_attn_fwd", "bound": "tensor", "achieved": achieved,
-                     "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
-                     "peak_source": f"{src} bf16_tflops (burst; the kernel runs at the maximum SM clock, "
-                                    "see clocks)",
-                     "frac_of_sustained_peak": achieved / peak_sust,
+        "roofline": {"kernel": "vsa_sparse_attn_fwd_fp8qk" if fp8 else "vsa_sparse_attn_fwd", "bound": "tensor",
+                     "achieved": achieved, "peak": attn_peak, "unit": "TFLOP/s", "frac": achieved / attn_peak,
+                     "peak_source": attn_peak_src,
+                     "frac_of_sustained_peak": achieved / attn_peak_sust,
                      "executed_tflops": res["exe"] / attn_s / 1e12,
-                     "executed_frac": res["exe"] / attn_s / 1e12 / peak_burst,
-                     "traffic": TRAFFIC.get(wl.name)},
+                     "executed_frac": res["exe"] / attn_s / 1e12 / attn_peak,
+                     "traffic": None if fp8 else TRAFFIC.get(wl.name)},
         "stage_roofline": stage_roofline(res["swork"], res["stage_ms"], float(peaks["hbm_gbs"]), peak_burst),
         "softmax_exp2_per_call": res["exp2"],
         "gpu_launches": res["launches"] * args.steps,

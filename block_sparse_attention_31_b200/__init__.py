@@ -18,6 +18,7 @@ from ._lib import (VSA_BF16, VSA_CUBE, VSA_F32, VSA_SELECT_CUBE, VSA_SELECT_GIVE
                    vsa_build_mask, vsa_get_device_error, vsa_layout_rows, vsa_mask_workspace_size, vsa_max_kv, vsa_num_blocks,
                    vsa_pattern_window, vsa_permute, vsa_profile_heads, vsa_profile_rows, vsa_profile_workspace_size,
                    vsa_sparse_attn_fwd, vsa_sparse_attn_fwd_natural, vsa_unpermute, SemParams, make_sem_params,
+                   vsa_quantize_fp8, vsa_sparse_attn_fwd_fp8qk,
                    vsa_gather_rows, vsa_kmeans, vsa_kmeans_workspace_size, vsa_scatter_rows, vsa_semantic_attention,
                    vsa_semantic_mask, vsa_semantic_mask_workspace_size, vsa_semantic_workspace_size)
 
@@ -96,13 +97,15 @@ class SparseAttention(_HostPipelined):
              smallest windows reaching it.
     layout_in_kernel: temporal heads are gathered through the frame-major map inside the
              attention kernel instead of being permuted into copies (bf16, no cube dims).
+    qk_fp8:  Q.K^T on e4m3 codes with one power-of-two scale per block; P.V stays bf16
+             (bf16, d = 128, block 128).
     """
 
     def __init__(self, B: int, H: int, F: int, Hl: int, Wl: int, d: int, block: int = 128, *,
                  dtype: torch.dtype = torch.bfloat16, select: str = "profile", w_s: Optional[int] = None,
                  w_t: Optional[int] = None, target: Optional[float] = None, topk: int = 0,
                  cube: Optional[Sequence[int]] = None, profile_frac: float = 0.01, scale: float = 0.0,
-                 with_lse: bool = False, layout_in_kernel: bool = False, device="cuda"):
+                 with_lse: bool = False, layout_in_kernel: bool = False, qk_fp8: bool = False, device="cuda"):
         if dtype not in _DTYPE:
             raise ValueError(f"unsupported dtype {dtype}")
         self.B, self.H, self.F, self.Hl, self.Wl, self.d, self.block = B, H, F, Hl, Wl, d, block
@@ -118,7 +121,7 @@ class SparseAttention(_HostPipelined):
             w_s = w_s_t if w_s is None else w_s
             w_t = w_t_t if w_t is None else w_t
         self.w_s, self.w_t = int(w_s or 0), int(w_t or 0)
-        self.params = make_params(self.w_s, self.w_t, profile_frac, topk, scale, layout_in_kernel)
+        self.params = make_params(self.w_s, self.w_t, profile_frac, topk, scale, layout_in_kernel, qk_fp8)
         self.ws_bytes = vsa_attention_workspace_size(self.shape, self.params, _DTYPE[dtype], self.select)
         if self.ws_bytes == 0:
             raise VsaError(_lib.VSA_ERR_INVALID_ARG, "vsa_attention_workspace_size")
@@ -221,5 +224,6 @@ __all__ = ["SparseAttention", "SemanticAttention", "attention", "SemParams", "ma
            "vsa_attention", "vsa_attention_workspace_layout", "vsa_attention_workspace_size", "vsa_block_order", "vsa_build_mask",
            "vsa_get_device_error", "vsa_layout_rows", "vsa_mask_workspace_size", "vsa_max_kv", "vsa_num_blocks",
            "vsa_pattern_window", "vsa_permute", "vsa_profile_heads", "vsa_profile_rows",
-           "vsa_profile_workspace_size", "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_natural", "vsa_unpermute", "VSA_SPATIAL", "VSA_TEMPORAL",
+           "vsa_profile_workspace_size", "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_natural", "vsa_unpermute",
+           "vsa_quantize_fp8", "vsa_sparse_attn_fwd_fp8qk", "VSA_SPATIAL", "VSA_TEMPORAL",
            "VSA_CUBE", "VSA_F32", "VSA_BF16", "VSA_SELECT_PROFILE", "VSA_SELECT_GIVEN", "VSA_SELECT_CUBE"]

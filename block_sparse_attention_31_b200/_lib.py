@@ -38,7 +38,8 @@ class Shape(ctypes.Structure):
 
 class Params(ctypes.Structure):
     _fields_ = [("w_s", ctypes.c_int), ("w_t", ctypes.c_int), ("profile_frac", ctypes.c_double),
-                ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("layout_in_kernel", ctypes.c_int)]
+                ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("layout_in_kernel", ctypes.c_int),
+                ("qk_fp8", ctypes.c_int)]
 
 
 class SemParams(ctypes.Structure):
@@ -77,6 +78,9 @@ def _load():
         "vsa_block_order": (st, [vp, vp, vp, i32, P(Shape), vp, vp]),
         "vsa_sparse_attn_fwd": (st, [P(QKVO), P(QKVO), vp, vp, vp, i32, vp, P(Shape), ctypes.c_float, vp, vp]),
         "vsa_sparse_attn_fwd_natural": (st, [P(QKVO), vp, vp, vp, i32, vp, P(Shape), ctypes.c_float, vp, vp]),
+        "vsa_quantize_fp8": (st, [vp, vp, vp, P(Shape), vp, vp, vp, vp]),
+        "vsa_sparse_attn_fwd_fp8qk": (st, [P(QKVO), P(QKVO), vp, vp, vp, vp, vp, vp, vp, i32, vp, P(Shape),
+                                           ctypes.c_float, vp, vp]),
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
@@ -140,8 +144,9 @@ def make_shape(B, H, F, Hl, Wl, d, block, cube=None) -> Shape:
     return Shape(B, H, F, Hl, Wl, d, block, cf, ch, cw)
 
 
-def make_params(w_s=0, w_t=0, profile_frac=0.01, topk=0, scale=0.0, layout_in_kernel=False) -> Params:
-    return Params(int(w_s), int(w_t), float(profile_frac), int(topk), float(scale), int(bool(layout_in_kernel)))
+def make_params(w_s=0, w_t=0, profile_frac=0.01, topk=0, scale=0.0, layout_in_kernel=False, qk_fp8=False) -> Params:
+    return Params(int(w_s), int(w_t), float(profile_frac), int(topk), float(scale), int(bool(layout_in_kernel)),
+                  int(bool(qk_fp8)))
 
 
 # ---------------------------------------------------------------------------------------
@@ -251,6 +256,20 @@ def vsa_sparse_attn_fwd(natural: QKVO, permuted, kinds, kv_idx, kv_cnt, max_kv, 
                                    _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt), int(max_kv), _ptr(order),
                                    ctypes.byref(shape), float(scale), _ptr(err), _stream(stream)),
            "vsa_sparse_attn_fwd")
+
+
+def vsa_quantize_fp8(natural, permuted, kinds, shape: Shape, dst, exps, err, stream=None):
+    _check(lib.vsa_quantize_fp8(_ptr(natural), _ptr(permuted), _ptr(kinds), ctypes.byref(shape), _ptr(dst), _ptr(exps),
+                                _ptr(err), _stream(stream)), "vsa_quantize_fp8")
+
+
+def vsa_sparse_attn_fwd_fp8qk(natural: QKVO, permuted, q8, qexp, k8, kexp, kinds, kv_idx, kv_cnt, max_kv,
+                              shape: Shape, scale, err, stream=None, order=None):
+    _check(lib.vsa_sparse_attn_fwd_fp8qk(ctypes.byref(natural),
+                                         ctypes.byref(permuted) if permuted is not None else None, _ptr(q8),
+                                         _ptr(qexp), _ptr(k8), _ptr(kexp), _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt),
+                                         int(max_kv), _ptr(order), ctypes.byref(shape), float(scale), _ptr(err),
+                                         _stream(stream)), "vsa_sparse_attn_fwd_fp8qk")
 
 
 def vsa_sparse_attn_fwd_natural(natural: QKVO, kinds, kv_idx, kv_cnt, max_kv, shape: Shape, scale, err, stream=None,

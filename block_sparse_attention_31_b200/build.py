@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libvsa.so")
-SOURCES = ["api.cu", "attn.cu", "mask.cu", "permute.cu", "profile.cu", "semantic.cu", "selftest.cu"]
+SOURCES = ["api.cu", "attn.cu", "fp8.cu", "mask.cu", "permute.cu", "profile.cu", "semantic.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -54,6 +54,21 @@ cudaError_t encode_rows_map(CUtensorMap* map, const void* base, int d, int rows,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_rows_map_u8(CUtensorMap* map, const void* base, int d, int rows, int BH, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  if (d != 128) return cudaErrorInvalidValue;  // one 128-byte swizzled row per box row
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows) * d};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -369,16 +384,30 @@ vsa_status vsa_block_order(const uint8_t* d_kind, const int32_t* d_kv_idx, const
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
-vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted, const uint8_t* d_kind,
-                               const int32_t* d_kv_idx, const int32_t* d_kv_cnt, int max_kv,
-                               const int32_t* d_order, const vsa_shape* shape, float scale, int* d_err,
-                               cudaStream_t stream) {
+// e4m3 Q and K for vsa_sparse_attn_fwd_fp8qk (all null for bf16).
+struct Fp8QK {
+  const uint8_t* q8;
+  const int32_t* qexp;
+  const uint8_t* k8;
+  const int32_t* kexp;
+};
+
+static vsa_status sparse_attn_fwd_impl(const vsa_qkvo* natural, const vsa_qkvo* permuted, const Fp8QK& f8,
+                                       const uint8_t* d_kind, const int32_t* d_kv_idx, const int32_t* d_kv_cnt,
+                                       int max_kv, const int32_t* d_order, const vsa_shape* shape, float scale,
+                                       int* d_err, cudaStream_t stream) {
   Geom g;
   vsa_status st = make_geom(shape, &g);
   if (st != VSA_OK) return st;
   if ((st = check_qkvo(natural)) != VSA_OK) return st;
   if (permuted != nullptr && (st = check_qkvo(permuted)) != VSA_OK) return st;
   if (!d_kind || !d_kv_idx || !d_kv_cnt || !d_err || max_kv <= 0 || !(scale >= 0.f)) return VSA_ERR_INVALID_ARG;
+  const bool qk8 = f8.q8 != nullptr;
+  if (qk8) {
+    if (!f8.qexp || !f8.k8 || !f8.kexp || !aligned16(f8.q8) || !aligned16(f8.k8)) return VSA_ERR_INVALID_ARG;
+    if (shape->d != 128 || shape->block != 128) return VSA_ERR_UNSUPPORTED;
+    if (!on_device({f8.q8, f8.qexp, f8.k8, f8.kexp})) return VSA_ERR_INVALID_ARG;
+  }
   const int BH = shape->B * shape->H;
   if (!on_device({natural->q, natural->k, natural->v, natural->o, natural->lse, d_kind, d_kv_idx, d_kv_cnt, d_order,
                   d_err}))
@@ -396,6 +425,12 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   } else {
     perm = nat;
   }
+  if (qk8) {  // every head's Q and K come from the e4m3 buffers (R rows per head, its own layout)
+    if (encode_rows_map_u8(&nat.q, f8.q8, shape->d, g.R, BH, 128) != cudaSuccess) return VSA_ERR_CUDA;
+    if (encode_rows_map_u8(&nat.k, f8.k8, shape->d, g.R, BH, g.block) != cudaSuccess) return VSA_ERR_CUDA;
+    perm.q = nat.q;
+    perm.k = nat.k;
+  }
   AttnArgs a;
   a.kinds = d_kind;
   a.kv_idx = d_kv_idx;
@@ -412,9 +447,44 @@ vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted
   a.nat_rows = nat_rows;
   a.ucap = std::min(g.nblk, 2 * max_kv);
   a.gather = 0;
+  a.qexp = qk8 ? f8.qexp : nullptr;
+  a.kexp = qk8 ? f8.kexp : nullptr;
   a.nat_q = a.nat_k = a.nat_v = nullptr;
   a.nat_o = natural->o;  // written only for a head with an invalid kind byte (zero rows)
   const cudaError_t e = launch_sparse_attn(nat, perm, a, shape->d, stream);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+vsa_status vsa_sparse_attn_fwd(const vsa_qkvo* natural, const vsa_qkvo* permuted, const uint8_t* d_kind,
+                               const int32_t* d_kv_idx, const int32_t* d_kv_cnt, int max_kv,
+                               const int32_t* d_order, const vsa_shape* shape, float scale, int* d_err,
+                               cudaStream_t stream) {
+  return sparse_attn_fwd_impl(natural, permuted, Fp8QK{nullptr, nullptr, nullptr, nullptr}, d_kind, d_kv_idx,
+                              d_kv_cnt, max_kv, d_order, shape, scale, d_err, stream);
+}
+
+vsa_status vsa_sparse_attn_fwd_fp8qk(const vsa_qkvo* natural, const vsa_qkvo* permuted, const uint8_t* q8,
+                                     const int32_t* d_qexp, const uint8_t* k8, const int32_t* d_kexp,
+                                     const uint8_t* d_kind, const int32_t* d_kv_idx, const int32_t* d_kv_cnt,
+                                     int max_kv, const int32_t* d_order, const vsa_shape* shape, float scale,
+                                     int* d_err, cudaStream_t stream) {
+  if (!q8) return VSA_ERR_INVALID_ARG;
+  return sparse_attn_fwd_impl(natural, permuted, Fp8QK{q8, d_qexp, k8, d_kexp}, d_kind, d_kv_idx, d_kv_cnt, max_kv,
+                              d_order, shape, scale, d_err, stream);
+}
+
+vsa_status vsa_quantize_fp8(const void* natural, const void* permuted, const uint8_t* d_kind,
+                            const vsa_shape* shape, uint8_t* dst, int32_t* d_exp, int* d_err, cudaStream_t stream) {
+  Geom g;
+  vsa_status st = make_geom(shape, &g);
+  if (st != VSA_OK) return st;
+  if (!natural || !d_kind || !dst || !d_exp || !d_err) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(natural) || (permuted && !aligned16(permuted)) || !aligned16(dst)) return VSA_ERR_INVALID_ARG;
+  if (shape->d != 128) return VSA_ERR_UNSUPPORTED;
+  if (!on_device({natural, permuted, d_kind, dst, d_exp, d_err})) return VSA_ERR_INVALID_ARG;
+  const int nat_rows = permuted != nullptr ? g.N : g.R;
+  const cudaError_t e = launch_quantize_e4m3(natural, permuted, d_kind, g, shape->B * shape->H, shape->d, nat_rows,
+                                             dst, d_exp, d_err, stream);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -449,6 +519,7 @@ vsa_status vsa_sparse_attn_fwd_natural(const vsa_qkvo* natural, const uint8_t* d
   a.nat_rows = g.N;
   a.ucap = std::min(g.nblk, 2 * max_kv);
   a.gather = 1;
+  a.qexp = a.kexp = nullptr;
   a.nat_q = natural->q;
   a.nat_k = natural->k;
   a.nat_v = natural->v;
@@ -651,7 +722,8 @@ vsa_status vsa_semantic_attention(const vsa_qkvo* io, const vsa_shape* shape, co
 // Whole call
 // ---------------------------------------------------------------------------------------
 struct AttnLayout {
-  size_t off_bits, off_idx, off_cnt, off_order, off_q, off_k, off_v, off_o, off_lse, off_prof, off_mask, bytes;
+  size_t off_bits, off_idx, off_cnt, off_order, off_q, off_k, off_v, off_o, off_lse, off_prof, off_mask;
+  size_t off_q8, off_k8, off_qe, off_ke, bytes;
   int max_kv;
 };
 
@@ -665,6 +737,9 @@ static vsa_status attention_layout(const vsa_shape* shape, const vsa_params* par
     return VSA_ERR_INVALID_ARG;
   if (select == VSA_SELECT_CUBE && g.ncubes == 0) return VSA_ERR_INVALID_ARG;
   if (select == VSA_SELECT_PROFILE && dtype != VSA_BF16) return VSA_ERR_UNSUPPORTED;
+  const bool qk8 = params->qk_fp8 != 0;
+  if (qk8 && (dtype != VSA_BF16 || shape->d != 128 || shape->block != 128 || params->layout_in_kernel != 0))
+    return VSA_ERR_UNSUPPORTED;
   int max_kv = 0;
   if ((st = vsa_max_kv(shape, params, &max_kv)) != VSA_OK) return st;
   if (max_kv <= 0) max_kv = 1;
@@ -695,6 +770,15 @@ static vsa_status attention_layout(const vsa_shape* shape, const vsa_params* par
   if (select == VSA_SELECT_PROFILE) off = align256(off + vsa_profile_workspace_size(shape, params));
   L->off_mask = off;
   off = align256(off + vsa_mask_workspace_size(shape, params));
+  // e4m3 Q and K with their per-block scale exponents
+  L->off_q8 = off;
+  if (qk8) off = align256(off + BH * g.R * d);
+  L->off_k8 = off;
+  if (qk8) off = align256(off + BH * g.R * d);
+  L->off_qe = off;
+  if (qk8) off = align256(off + BH * g.nblk * 4);
+  L->off_ke = off;
+  if (qk8) off = align256(off + BH * g.nblk * 4);
   L->bytes = off;
   L->max_kv = max_kv;
   return VSA_OK;
@@ -776,7 +860,14 @@ vsa_status vsa_attention(const vsa_qkvo* io, vsa_dtype dtype, const vsa_shape* s
     if ((st = vsa_block_order(d_kind, kv_idx, kv_cnt, L.max_kv, shape, order, stream)) != VSA_OK) return st;
   }
   const vsa_qkvo perm_set{pq, pk, pv, po, plse};
-  if (dtype == VSA_F32) {
+  if (params->qk_fp8 != 0) {  // e4m3 Q and K (bf16 inputs only, checked by attention_layout)
+    uint8_t *q8 = w + L.off_q8, *k8 = w + L.off_k8;
+    int32_t *qe = reinterpret_cast<int32_t*>(w + L.off_qe), *ke = reinterpret_cast<int32_t*>(w + L.off_ke);
+    if ((st = vsa_quantize_fp8(io->q, pq, d_kind, shape, q8, qe, d_err, stream)) != VSA_OK) return st;
+    if ((st = vsa_quantize_fp8(io->k, pk, d_kind, shape, k8, ke, d_err, stream)) != VSA_OK) return st;
+    st = vsa_sparse_attn_fwd_fp8qk(io, &perm_set, q8, qe, k8, ke, d_kind, kv_idx, kv_cnt, L.max_kv, order, shape,
+                                   params->scale, d_err, stream);
+  } else if (dtype == VSA_F32) {
     st = vsa_sparse_attn_fwd(&perm_set, nullptr, d_kind, kv_idx, kv_cnt, L.max_kv, order, shape, params->scale,
                              d_err, stream);
   } else {

@@ -50,22 +50,33 @@ constexpr int kBM = 128;           // MMA M: query rows per tile
 constexpr int kRegsSoftmax = 208, kRegsCtl = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl == 384 * 168, "register split must equal the launch total");
 
-template <int D, int BN>
+// QK8: Q and K are e4m3 codes with one power-of-two scale per block (Q.K^T on kind::f8f6f4);
+// V, P and O stay bf16.
+template <int D, int BN, bool QK8>
 struct AttnCfg {
   static constexpr int NS = 2;  // K/V ring stages
-  static constexpr int Q_BYTES = kBM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int QK_ES = QK8 ? 1 : 2;            // bytes per Q / K element
+  static constexpr int Q_BYTES = kBM * D * QK_ES;
+  static constexpr int K_BYTES = BN * D * QK_ES;
+  static constexpr int V_BYTES = BN * D * 2;
+  static constexpr int O_BYTES = kBM * D * 2;           // one tile of bf16 output
+  static constexpr int QK_PANEL = 128 / QK_ES;          // elements in one 128-byte swizzled row
+  static constexpr int QK_PANELS = D / QK_PANEL;
+  static constexpr int QK_KSTEP = QK8 ? 32 : 16;        // K of one MMA instruction (32 bytes)
   static constexpr int OFF_Q = 0;  // two Q tiles
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * K_BYTES;
+  // output staging: over the tile's Q buffer for bf16; a region of its own for e4m3 Q, whose
+  // tile is half the size of the bf16 output tile
+  static constexpr int OFF_OST = OFF_V + NS * V_BYTES;
+  static constexpr int OFF_BAR = OFF_OST + (QK8 ? 2 * O_BYTES : 0);
   static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_UNION = OFF_MISC + 64;  // union list, two bitsets, key-validity masks
   static constexpr int TMEM_S = 0;                  // S of tile t at t*BN (P aliases its first BN/2 columns)
   static constexpr int TMEM_O = 2 * BN;             // O of tile t at 2*BN + t*D
   static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
-  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBM, BN, false, false);
+  static constexpr uint32_t IDESC_QK = QK8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, false, true);
   static int smem_bytes(int ucap, int nwords) { return OFF_UNION + 4 * ucap + 8 * nwords + 4 * ucap * (BN / 32) + 1024; }
 };
@@ -95,14 +106,14 @@ constexpr int kPolyPairs8 = VSA_POLY_PAIRS8;
 // MMA issuer interleaves the tiles (P.V of one, then Q.K^T of the same tile, then the other
 // tile) so the tensor core works on one tile while the other tile's softmax runs.  P is
 // written as packed bf16 over the tile's S columns in TMEM and read from there by the P.V MMA.
-template <int D, int BN>
+template <int D, int BN, bool QK8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tq_n, const __grid_constant__ CUtensorMap tk_n,
                            const __grid_constant__ CUtensorMap tv_n, const __grid_constant__ CUtensorMap to_n,
                            const __grid_constant__ CUtensorMap tq_p, const __grid_constant__ CUtensorMap tk_p,
                            const __grid_constant__ CUtensorMap tv_p, const __grid_constant__ CUtensorMap to_p,
                            const AttnArgs a) {
-  using C = AttnCfg<D, BN>;
+  using C = AttnCfg<D, BN, QK8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
@@ -348,7 +359,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t u = n / C::NS;
         const int kb = static_cast<int>(uni[n] & kKbMask);
         if (n >= C::NS && !__all_sync(0xffffffffu, mbar_wait(bar(eb + st), (u - 1) & 1, abort_flag, a.err))) break;
-        gather_tile(sdst0 + st * C::KV_BYTES, BN, kb * BN, gsrc);
+        gather_tile(sdst0 + st * (qk ? C::K_BYTES : C::V_BYTES), BN, kb * BN, gsrc);
         cp_async_mbar_arrive_noinc(bar(fb + st));
       }
       // every copy lands before the CTA can exit (they always complete; nothing to bound)
@@ -364,8 +375,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (cnts[t] == 0) continue;
         mbar_arrive_expect_tx(bar(B_Q + t), C::Q_BYTES);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * 64,
+        for (int c = 0; c < C::QK_PANELS; ++c)
+          tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * C::QK_PANEL,
                       (t ? qb1 : qb0) * BN, bh);
       }
       for (int n = 0; n < U; ++n) {
@@ -373,16 +384,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t u = n / C::NS;
         const int kb = static_cast<int>(uni[n] & kKbMask);
         if (n >= C::NS && !mbar_wait(bar(B_EMPTY_K + st), (u - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(bar(B_FULL_K + st), C::KV_BYTES);
+        mbar_arrive_expect_tx(bar(B_FULL_K + st), C::K_BYTES);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK + st * C::KV_BYTES + c * BN * 128, tk, bar(B_FULL_K + st), c * 64, kb * BN, bh);
+        for (int c = 0; c < C::QK_PANELS; ++c)
+          tma_load_3d(sK + st * C::K_BYTES + c * BN * 128, tk, bar(B_FULL_K + st), c * C::QK_PANEL, kb * BN, bh);
         nk = n + 1;
         if (n >= C::NS && !mbar_wait(bar(B_EMPTY_V + st), (u - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(bar(B_FULL_V + st), C::KV_BYTES);
+        mbar_arrive_expect_tx(bar(B_FULL_V + st), C::V_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sV + st * C::KV_BYTES + c * BN * 128, tv, bar(B_FULL_V + st), c * 64, kb * BN, bh);
+          tma_load_3d(sV + st * C::V_BYTES + c * BN * 128, tv, bar(B_FULL_V + st), c * 64, kb * BN, bh);
         nv = n + 1;
       }
       if (*abort_flag) {
@@ -412,8 +423,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       static_assert(C::NS == 2, "descriptor selection below assumes two stages");
       const uint64_t dq0 = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
       const uint64_t dq1 = sdesc_sw128(sbase + C::OFF_Q + C::Q_BYTES, 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::KV_BYTES, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::KV_BYTES, BN * 128, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::K_BYTES, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::V_BYTES, BN * 128, 1024);
       // P.V of tile t's pending block: the first half of the keys as soon as its P is written,
       // the second half after the rest
       auto issue_pv = [&](int t) -> bool {
@@ -462,11 +473,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_after();
           const uint32_t d_s = tmem + C::TMEM_S + t * BN;
           const uint64_t qd = t ? dq1 : dq0, kd = st ? dk1 : dk0;
+          // each instruction takes 32 bytes of K: four per 128-byte swizzled row of a panel
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma_ss(d_s, qd + static_cast<uint64_t>(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) / 16),
-                      kd + static_cast<uint64_t>(((kk >> 2) * (BN * 128) + (kk & 3) * 32) / 16), C::IDESC_QK,
-                      kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / C::QK_KSTEP; ++kk) {
+            const uint64_t qa = qd + static_cast<uint64_t>(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) / 16);
+            const uint64_t kb_ = kd + static_cast<uint64_t>(((kk >> 2) * (BN * 128) + (kk & 3) * 32) / 16);
+            if constexpr (QK8) tc_mma_ss_f8(d_s, qa, kb_, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            else tc_mma_ss(d_s, qa, kb_, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
           tc_commit(bar(B_S_FULL + t));
           pend[t] = n;
         }
@@ -493,7 +507,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int qb = t ? qb1 : qb0;
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
       const uint32_t t_s = t_lane + C::TMEM_S + t * BN, t_o = t_lane + C::TMEM_O + t * D;
-      const float sl2 = a.scale_log2;
+      const float sl2_base = a.scale_log2;
+      // e4m3 Q and K: the block pair's scores carry the scales 2^(e_q + e_k)
+      const int eq = QK8 ? a.qexp[static_cast<size_t>(bh) * g.nblk + qb] : 0;
       float m = -INFINITY, l = 0.f;  // m: the (lazily updated) max used for the exponentials
       bool ok = true;
       int cur = 0;  // cursor into the union list (this tile's entries are the ones with its bit)
@@ -519,6 +535,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         ++cur;
+        const float sl2 = QK8 ? ldexpf(sl2_base, eq + a.kexp[static_cast<size_t>(bh) * g.nblk + (ent & kKbMask)])
+                              : sl2_base;
         // row max: eight independent partial maxima keep the dependency chains short
         float mx8[8];
 #pragma unroll
@@ -596,7 +614,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const bool have = ok && cnt > 0 && l > 0.f;
       const float inv = have ? 1.f / l : 0.f;
-      uint8_t* stage = smem + C::OFF_Q + t * C::Q_BYTES;
+      uint8_t* stage = smem + (QK8 ? C::OFF_OST + t * C::O_BYTES : C::OFF_Q + t * C::Q_BYTES);
       // in-kernel layout: this row's natural token (slot p -> (p % F) * S + p / F)
       const int slot = qb * BN + row;
       const bool row_live = row < BN && slot < rows;
@@ -634,7 +652,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         fence_proxy_async_smem();
         named_barrier_sync(1 + t, 128);
         if (quad == 2 && lane == 0) {
-          const uint32_t sstage = sbase + C::OFF_Q + t * C::Q_BYTES;
+          const uint32_t sstage = sbase + (QK8 ? C::OFF_OST + t * C::O_BYTES : C::OFF_Q + t * C::Q_BYTES);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) tma_store_3d(to, sstage + c * BN * 128, c * 64, qb * BN, bh);
           tma_store_commit();
@@ -653,10 +671,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == kWarpMma) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int D, int BN>
+template <int D, int BN, bool QK8>
 static cudaError_t launch_attn_t(const AttnMaps& nat, const AttnMaps& perm, const AttnArgs& a, cudaStream_t stream) {
-  using C = AttnCfg<D, BN>;
-  auto kern = sparse_attn_fwd_kernel<D, BN>;
+  using C = AttnCfg<D, BN, QK8>;
+  auto kern = sparse_attn_fwd_kernel<D, BN, QK8>;
   const int nwords = (a.g.nblk + 31) / 32;
   const int smem = C::smem_bytes(a.ucap, nwords);
   if (smem > 232448) return cudaErrorInvalidConfiguration;
@@ -664,18 +682,22 @@ static cudaError_t launch_attn_t(const AttnMaps& nat, const AttnMaps& perm, cons
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(a.BH) * ((a.g.nblk + 1) / 2);
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k,
-                                                                     perm.v, perm.o, a);
+  kern<<<static_cast<unsigned>(grid), kAttnThreads, smem, stream>>>(nat.q, nat.k, nat.v, nat.o, perm.q, perm.k, perm.v,
+                                                                   perm.o, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_attn(const AttnMaps& nat, const AttnMaps& perm, const AttnArgs& a, int d,
                                cudaStream_t stream) {
   const int bn = a.g.block;
-  if (d == 128 && bn == 128) return launch_attn_t<128, 128>(nat, perm, a, stream);
-  if (d == 64 && bn == 128) return launch_attn_t<64, 128>(nat, perm, a, stream);
-  if (d == 128 && bn == 64) return launch_attn_t<128, 64>(nat, perm, a, stream);
-  if (d == 64 && bn == 64) return launch_attn_t<64, 64>(nat, perm, a, stream);
+  if (a.qexp != nullptr) {  // e4m3 Q and K: d = 128, block 128, no in-kernel layout
+    if (d == 128 && bn == 128 && !a.gather) return launch_attn_t<128, 128, true>(nat, perm, a, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (d == 128 && bn == 128) return launch_attn_t<128, 128, false>(nat, perm, a, stream);
+  if (d == 64 && bn == 128) return launch_attn_t<64, 128, false>(nat, perm, a, stream);
+  if (d == 128 && bn == 64) return launch_attn_t<128, 64, false>(nat, perm, a, stream);
+  if (d == 64 && bn == 64) return launch_attn_t<64, 64, false>(nat, perm, a, stream);
   return cudaErrorInvalidValue;
 }
 

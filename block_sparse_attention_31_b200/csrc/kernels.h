@@ -70,6 +70,9 @@ struct AttnArgs {
   // In-kernel layout: temporal heads read Q, K, V and write O in natural order through the
   // frame-major slot map (no permuted copies); only with has_perm == 0.
   int gather;
+  // e4m3 Q and K (null for bf16): per (head, block) power-of-two exponents of their scales
+  const int32_t* qexp;
+  const int32_t* kexp;
   const void* nat_q;
   const void* nat_k;
   const void* nat_v;
@@ -96,5 +99,11 @@ cudaError_t launch_profile(const void* q, const void* k, const void* v, const Ge
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
 cudaError_t encode_rows_map(CUtensorMap* map, const void* base, int d, int rows, int BH, int box_rows);
+// The same for rows of d = 128 one-byte elements (e4m3 codes): one 128-byte box per row.
+cudaError_t encode_rows_map_u8(CUtensorMap* map, const void* base, int d, int rows, int BH, int box_rows);
+
+// Per-block e4m3 quantisation (fp8.cu): dst [BH, R, d] codes, exps [BH, nblk].
+cudaError_t launch_quantize_e4m3(const void* nat, const void* perm, const uint8_t* kinds, const Geom& g, int BH,
+                                 int d, int nat_rows, uint8_t* dst, int32_t* exps, int* err, cudaStream_t stream);
 
 }  // namespace vsa

@@ -114,6 +114,10 @@ typedef struct {
                                      in natural order through the frame-major map inside the
                                      attention kernel (no permute / unpermute copies); used
                                      for bf16 inputs without cube dims, ignored otherwise */
+    int qk_fp8;                   /* vsa_attention only: 1 = Q.K^T on e4m3 codes with one
+                                     power-of-two scale per block (vsa_quantize_fp8,
+                                     vsa_sparse_attn_fwd_fp8qk); bf16 inputs, d = 128, block 128,
+                                     not with layout_in_kernel (VSA_ERR_UNSUPPORTED otherwise) */
 } vsa_params;
 
 /* Pointers of one attention problem; o and lse are written. lse may be NULL. */
@@ -292,6 +296,42 @@ VSA_API vsa_status vsa_sparse_attn_fwd_natural(const vsa_qkvo *natural, const ui
                                                const int32_t *d_kv_idx, const int32_t *d_kv_cnt, int max_kv,
                                                const int32_t *d_order, const vsa_shape *shape, float scale,
                                                int *d_err, cudaStream_t stream);
+
+/*
+ * FP8 Q and K ("Sparse Video-Gen" summary page, "Measured effects": FP8 quantisation added to
+ * the sparse attention, 1.92x -> 2.33x end to end; its "Limitations" report no gain at head
+ * dimension 64).  The page gives no format; the reading used here: e4m3 codes (round to
+ * nearest even, saturating at 448) of x / 2^e, with one power-of-two scale 2^e per block of
+ * `block` rows of a head's layout, the smallest with max |x| <= 448 * 2^e (e = 0 for an
+ * all-zero block).  P.V stays bf16.
+ *
+ * vsa_quantize_fp8: codes of one tensor (Q or K) for every head, read as the attention reads
+ * them: spatial heads (or every head when `permuted` is NULL) from `natural`, temporal and cube
+ * heads from `permuted`.
+ *   natural   [B, H, N, d] bf16 (or [B, H, R, d] when permuted is NULL);  permuted [B, H, R, d]
+ *   dst       [B, H, R, d] e4m3 codes (caller-owned device memory); rows past a head's own
+ *             rows are zero
+ *   d_exp     [B*H, nblk] int32 out: the exponent e of every block's scale
+ * d must be 128 (VSA_ERR_UNSUPPORTED otherwise); a bad kind byte sets VSA_DEVERR_KIND.
+ */
+VSA_API vsa_status vsa_quantize_fp8(const void *natural, const void *permuted, const uint8_t *d_kind,
+                                    const vsa_shape *shape, uint8_t *dst, int32_t *d_exp, int *d_err,
+                                    cudaStream_t stream);
+
+/*
+ * vsa_sparse_attn_fwd with Q.K^T on e4m3 codes (tcgen05 kind::f8f6f4, fp32 accumulation): the
+ * scores of query block i and key block j are scaled by 2^(qexp[i] + kexp[j]) before the
+ * softmax; V, P and O are as in vsa_sparse_attn_fwd.
+ *   q8, k8          [B, H, R, d] e4m3 codes from vsa_quantize_fp8 (every head in its layout)
+ *   d_qexp, d_kexp  [B*H, nblk] their exponents
+ *   the rest        as vsa_sparse_attn_fwd (V, O and LSE from the natural / permuted sets)
+ * d = 128 and block = 128 only (VSA_ERR_UNSUPPORTED otherwise).
+ */
+VSA_API vsa_status vsa_sparse_attn_fwd_fp8qk(const vsa_qkvo *natural, const vsa_qkvo *permuted, const uint8_t *q8,
+                                             const int32_t *d_qexp, const uint8_t *k8, const int32_t *d_kexp,
+                                             const uint8_t *d_kind, const int32_t *d_kv_idx, const int32_t *d_kv_cnt,
+                                             int max_kv, const int32_t *d_order, const vsa_shape *shape,
+                                             float scale, int *d_err, cudaStream_t stream);
 
 /*
  * The whole call: kinds (profiled, given or cube) -> permute -> masks -> sparse attention
