@@ -86,13 +86,11 @@ enum {
   B_Q = 0,         // +tile
   B_FULL_K = 2,    // +stage
   B_FULL_V = 4,    // +stage
-  B_EMPTY_K = 6,   // +stage
-  B_EMPTY_V = 8,   // +stage
+  B_REL = 6,       // +entry parity: K of entry n and V of entry n - 1 consumed (one commit per entry)
   B_S_FULL = 10,   // +tile
   B_P_FULL = 12,   // +tile
   B_O_FINAL = 14,  // +tile
-  B_DRAIN = 16,
-  B_P_HALF = 17    // +tile: first half of P (keys 0..BN/2-1) written
+  B_DRAIN = 16
 };
 constexpr uint32_t kInTile0 = 1u << 30, kInTile1 = 1u << 31, kPartial = 1u << 29, kKbMask = (1u << 29) - 1u;
 // Probability pairs (2 columns) whose exponentials run on the FMA pipe: kPolyPairs8 in 8.
@@ -277,14 +275,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(B_Q + t), nload);
       mbar_init(bar(B_S_FULL + t), 1);
       mbar_init(bar(B_P_FULL + t), 128);
-      mbar_init(bar(B_P_HALF + t), 128);
       mbar_init(bar(B_O_FINAL + t), 1);
     }
     for (int st = 0; st < C::NS; ++st) {
       mbar_init(bar(B_FULL_K + st), nload);
       mbar_init(bar(B_FULL_V + st), nload);
-      mbar_init(bar(B_EMPTY_K + st), 1);
-      mbar_init(bar(B_EMPTY_V + st), 1);
+      mbar_init(bar(B_REL + st), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0;
@@ -351,14 +347,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           cp_async_mbar_arrive_noinc(bar(B_Q + t));
         }
       }
-      const int eb = qk ? B_EMPTY_K : B_EMPTY_V, fb = qk ? B_FULL_K : B_FULL_V;
+      const int fb = qk ? B_FULL_K : B_FULL_V;
       const uint32_t sdst0 = qk ? sK : sV;
       const __nv_bfloat16* gsrc = qk ? gk : gv;
       for (int n = 0; n < U; ++n) {
         const int st = n % C::NS;
-        const uint32_t u = n / C::NS;
         const int kb = static_cast<int>(uni[n] & kKbMask);
-        if (n >= C::NS && !__all_sync(0xffffffffu, mbar_wait(bar(eb + st), (u - 1) & 1, abort_flag, a.err))) break;
+        // K(n) replaces K(n-2): free after entry n-2's MMAs; V(n) replaces V(n-2): free after entry n-1's
+        const int re = qk ? n - 2 : n - 1;
+        if (n >= C::NS &&
+            !__all_sync(0xffffffffu, mbar_wait(bar(B_REL + re % C::NS), (re / C::NS) & 1, abort_flag, a.err)))
+          break;
         gather_tile(sdst0 + st * (qk ? C::K_BYTES : C::V_BYTES), BN, kb * BN, gsrc);
         cp_async_mbar_arrive_noinc(bar(fb + st));
       }
@@ -383,13 +382,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = n % C::NS;
         const uint32_t u = n / C::NS;
         const int kb = static_cast<int>(uni[n] & kKbMask);
-        if (n >= C::NS && !mbar_wait(bar(B_EMPTY_K + st), (u - 1) & 1, abort_flag, a.err)) break;
+        // K(n) goes where K(n-2) was: free once entry n-2's MMAs complete
+        if (n >= C::NS && !mbar_wait(bar(B_REL + st), (u - 1) & 1, abort_flag, a.err)) break;
         mbar_arrive_expect_tx(bar(B_FULL_K + st), C::K_BYTES);
 #pragma unroll
         for (int c = 0; c < C::QK_PANELS; ++c)
           tma_load_3d(sK + st * C::K_BYTES + c * BN * 128, tk, bar(B_FULL_K + st), c * C::QK_PANEL, kb * BN, bh);
         nk = n + 1;
-        if (n >= C::NS && !mbar_wait(bar(B_EMPTY_V + st), (u - 1) & 1, abort_flag, a.err)) break;
+        // V(n) goes where V(n-2) was: free once entry n-1's MMAs (which include P.V of n-2) complete
+        if (n >= C::NS && !mbar_wait(bar(B_REL + (n - 1) % C::NS), ((n - 1) / C::NS) & 1, abort_flag, a.err)) break;
         mbar_arrive_expect_tx(bar(B_FULL_V + st), C::V_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
@@ -425,32 +426,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq1 = sdesc_sw128(sbase + C::OFF_Q + C::Q_BYTES, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + C::K_BYTES, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sV, BN * 128, 1024), dv1 = sdesc_sw128(sV + C::V_BYTES, BN * 128, 1024);
-      // P.V of tile t's pending block: the first half of the keys as soon as its P is written,
-      // the second half after the rest
+      // P.V of tile t's pending block (its V was waited for at the start of the entry)
       auto issue_pv = [&](int t) -> bool {
         const int np = pend[t];
-        if (!mbar_wait(bar(B_P_HALF + t), pvc[t] & 1, abort_flag, a.err)) return false;
-        if (!mbar_wait(bar(B_FULL_V + np % C::NS), (np / C::NS) & 1, abort_flag, a.err)) return false;
+        if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
         if (gather) fence_proxy_async_smem();  // cp.async data, written by the generic proxy
         tc_fence_after();
         const uint64_t vd = (np & 1) ? dv1 : dv0;
         const uint32_t d_o = tmem + C::TMEM_O + t * D, a_p = tmem + C::TMEM_S + t * BN;
         tc_mma_ts(d_o, a_p, vd, C::IDESC_PV, pvc[t] > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < BN / 32; ++kk)
-          tc_mma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV, 1u);
-        if (!mbar_wait(bar(B_P_FULL + t), pvc[t] & 1, abort_flag, a.err)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = BN / 32; kk < BN / 16; ++kk)
+        for (int kk = 1; kk < BN / 16; ++kk)
           tc_mma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 16 * 128 / 16), C::IDESC_PV, 1u);
         pend[t] = -1;
         if (++pvc[t] == cnts[t]) tc_commit(bar(B_O_FINAL + t));
         return true;
       };
+      // Every wait and commit of this thread can leave the tensor core idle, so an entry makes
+      // few of them: K of the entry and V of the previous one up front, one P per tile, one
+      // S commit per tile and one release of both stages.
       for (int n = 0; ok && n < U; ++n) {
         const int st = n % C::NS;
-        if (!mbar_wait(bar(B_FULL_K + st), (n / C::NS) & 1, abort_flag, a.err)) {
+        if (!mbar_wait(bar(B_FULL_K + st), (n / C::NS) & 1, abort_flag, a.err) ||
+            (n >= 1 && !mbar_wait(bar(B_FULL_V + (n - 1) % C::NS), ((n - 1) / C::NS) & 1, abort_flag, a.err))) {
           ok = false;
           break;
         }
@@ -485,9 +483,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pend[t] = n;
         }
         if (!ok) break;
-        tc_commit(bar(B_EMPTY_K + st));
-        if (n >= 1) tc_commit(bar(B_EMPTY_V + (n - 1) % C::NS));
+        tc_commit(bar(B_REL + st));  // K(n) and V(n-1) are free once these MMAs complete
       }
+      if (ok && U >= 1 && !mbar_wait(bar(B_FULL_V + (U - 1) % C::NS), ((U - 1) / C::NS) & 1, abort_flag, a.err))
+        ok = false;
       for (int t = 0; ok && t < 2; ++t)
         if (pend[t] >= 0 && !issue_pv(t)) ok = false;
       // Drain: all MMAs issued by this thread complete before TMEM is released.
@@ -597,9 +596,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st_cols<BN / 4>(t_s + hf * (BN / 4), pk);
-          tc_fence_before();
-          mbar_arrive(bar((hf ? B_P_FULL : B_P_HALF) + t));
         }
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL + t));
         {
           const uint64_t s2 = f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3]));
           float s0, s1;
