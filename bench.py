@@ -546,7 +546,7 @@ def e2e_arm(args, wl, q, k, v, device):
         kw.update(w_s=wl.w_s, w_t=wl.w_t)
     plan = vsa.SparseAttention(wl.B, wl.H, wl.F, wl.Hl, wl.Wl, wl.d, wl.block, **kw)
     kinds = torch.tensor(list(wl.fixed_kinds), dtype=torch.uint8, device=device) if wl.mode == "fixed" else None
-    return _e2e_run(args, plan, q, k, v, kinds, "SparseAttention.run_host")
+    return _e2e_run(args, plan, q, k, v, kinds, "vsa_attention_host (C ABI, host batches) via SparseAttention.run_host")
 
 
 def _e2e_run(args, plan, q, k, v, kinds, api):
@@ -747,7 +747,7 @@ def main():
         "clocks": res["clocks"],
         "e2e": {"value": aggregate_tflops(res["alg"], res["e2e"]["ms_per_step"], world), "unit": "TFLOP/s",
                 "ms_per_step": res["e2e"]["ms_per_step"], "h2d_bytes_per_step": res["e2e"]["h2d_bytes_per_step"],
-                "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"]},
+                "d2h_bytes_per_step": res["e2e"]["d2h_bytes_per_step"], "api": res["e2e"]["api"]},
     }
     if not args.no_cpu_baseline and world == 1:
         v, desc, cores, _ = oracle_sample(wl, args.cpu_seconds)

@@ -3,7 +3,8 @@
 The compute lives in ``libvsa.so`` (hand-written CUDA for sm_100a behind the C ABI in
 ``include/vsa.h``).  This package is its thin Python binding: ``_lib`` mirrors each C entry
 point under the same name, and :class:`SparseAttention` owns the device buffers (from
-PyTorch) of one configured call and invokes ``vsa_attention``.
+PyTorch) of one configured call and invokes ``vsa_attention`` (``vsa_attention_host`` for
+host batches).
 """
 from __future__ import annotations
 
@@ -164,6 +165,49 @@ class SparseAttention(_HostPipelined):
 
     def clear_error(self):
         self.err.zero_()
+
+    def run_host(self, batches, outs=None, kinds: Optional[torch.Tensor] = None, timing=None):
+        """The call on a sequence of host batches through the library's vsa_attention_host: the
+        uploads of batch i+1 and the download of batch i-1 overlap the compute of batch i (three
+        streams, two device buffer sets owned here).  ``batches`` is a list of (q, k, v) CPU
+        tensors, which must be pinned for the copies to overlap; ``outs`` a list of CPU output
+        tensors (pinned ones are allocated when None).  Returns ``outs`` once every output has
+        arrived.  ``timing``, a pair of timing-enabled CUDA events, is recorded before the first
+        upload and after the last download."""
+        n = len(batches)
+        shape = (self.B, self.H, self.N, self.d)
+        if outs is None:
+            outs = [torch.empty(shape, dtype=self.dtype).pin_memory() for _ in range(n)]
+        if len(outs) != n:
+            raise ValueError("need one output tensor per batch")
+        for (q, k, v), o in zip(batches, outs):
+            for t in (q, k, v, o):
+                if t.device.type != "cpu" or t.dtype != self.dtype or tuple(t.shape) != shape or not t.is_contiguous():
+                    raise ValueError(f"contiguous host tensors of shape {shape} and dtype {self.dtype} expected")
+        if self.select == VSA_SELECT_GIVEN:
+            if kinds is None:
+                raise ValueError("select='given' needs kinds")
+            self.kinds.copy_(kinds.reshape(-1).to(torch.uint8))
+        if not hasattr(self, "_host_bufs"):
+            self._host_bufs = [[torch.empty(shape, dtype=self.dtype, device=self.device) for _ in range(4)]
+                               for _ in range(2)]  # q, k, v, o per buffer set
+            self._host_lse = ([torch.empty(self.B, self.H, self.N, dtype=torch.float32, device=self.device)
+                               for _ in range(2)] if self.with_lse else [None, None])
+            self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]  # upload, compute, download
+        up, comp, down = self._streams
+        cur = torch.cuda.current_stream(self.device)
+        up.wait_stream(cur)
+        comp.wait_stream(cur)
+        if timing is not None:
+            timing[0].record(up)
+        sets = [qkvo(b[0], b[1], b[2], b[3], lse) for b, lse in zip(self._host_bufs, self._host_lse)]
+        _lib.vsa_attention_host([(q, k, v, o) for (q, k, v), o in zip(batches, outs)], sets, _DTYPE[self.dtype],
+                                self.shape, self.params, self.select, self.kinds, self.mse, self.ws, self.ws_bytes,
+                                self.err, up, comp, down)
+        if timing is not None:
+            timing[1].record(down)
+        down.synchronize()
+        return outs
 
 
 class SemanticAttention(_HostPipelined):

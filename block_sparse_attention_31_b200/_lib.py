@@ -47,6 +47,10 @@ class SemParams(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
+class HostBatch(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p)]
+
+
 class QKVO(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
                 ("lse", ctypes.c_void_p)]
@@ -82,6 +86,8 @@ def _load():
         "vsa_sparse_attn_fwd_fp8qk": (st, [P(QKVO), P(QKVO), vp, vp, vp, vp, vp, vp, vp, i32, vp, P(Shape),
                                            ctypes.c_float, vp, vp]),
         "vsa_attention": (st, [P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp, vp]),
+        "vsa_attention_host": (st, [P(HostBatch), i32, P(QKVO), i32, P(Shape), P(Params), i32, vp, vp, vp, sz, vp,
+                                    vp, vp, vp]),
         "vsa_attention_workspace_layout": (st, [P(Shape), P(Params), i32, i32, P(sz), P(sz), P(sz), P(i32)]),
         "vsa_get_device_error": (st, [vp, vp, P(i32)]),
         "vsa_kmeans_workspace_size": (sz, [P(Shape), i32]),
@@ -277,6 +283,16 @@ def vsa_sparse_attn_fwd_natural(natural: QKVO, kinds, kv_idx, kv_cnt, max_kv, sh
     _check(lib.vsa_sparse_attn_fwd_natural(ctypes.byref(natural), _ptr(kinds), _ptr(kv_idx), _ptr(kv_cnt),
                                            int(max_kv), _ptr(order), ctypes.byref(shape), float(scale), _ptr(err),
                                            _stream(stream)), "vsa_sparse_attn_fwd_natural")
+
+
+def vsa_attention_host(batches, sets, dtype: int, shape: Shape, params: Params, select: int, kinds, mse, ws,
+                       ws_bytes, err, stream_up, stream_compute, stream_down):
+    """batches: sequence of (q, k, v, o) host tensors (pinned); sets: two QKVO of device buffers."""
+    arr = (HostBatch * len(batches))(*[HostBatch(_ptr(q), _ptr(k), _ptr(v), _ptr(o)) for q, k, v, o in batches])
+    sarr = (QKVO * 2)(*sets)
+    _check(lib.vsa_attention_host(arr, len(batches), sarr, dtype, ctypes.byref(shape), ctypes.byref(params), select,
+                                  _ptr(kinds), _ptr(mse), _ptr(ws), int(ws_bytes), _ptr(err), _stream(stream_up),
+                                  _stream(stream_compute), _stream(stream_down)), "vsa_attention_host")
 
 
 def vsa_attention(io: QKVO, dtype: int, shape: Shape, params: Params, select: int, kinds, mse, ws, ws_bytes, err,

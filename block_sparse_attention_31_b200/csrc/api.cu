@@ -879,6 +879,63 @@ vsa_status vsa_attention(const vsa_qkvo* io, vsa_dtype dtype, const vsa_shape* s
   return vsa_unpermute(po, plse, io->o, dtype, io->lse, d_kind, shape, d_err, stream);
 }
 
+vsa_status vsa_attention_host(const vsa_host_batch* host, int n, const vsa_qkvo* sets, vsa_dtype dtype,
+                              const vsa_shape* shape, const vsa_params* params, vsa_select select, uint8_t* d_kind,
+                              float* d_mse, void* ws, size_t ws_bytes, int* d_err, cudaStream_t stream_up,
+                              cudaStream_t stream_compute, cudaStream_t stream_down) {
+  if (host == nullptr || sets == nullptr || n < 0 || shape == nullptr) return VSA_ERR_INVALID_ARG;
+  if (dtype != VSA_F32 && dtype != VSA_BF16) return VSA_ERR_INVALID_ARG;
+  if (shape->B <= 0 || shape->H <= 0 || shape->F <= 0 || shape->Hl <= 0 || shape->Wl <= 0 || shape->d <= 0)
+    return VSA_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(shape->B) * shape->H * shape->F * shape->Hl * shape->Wl * shape->d *
+                       (dtype == VSA_F32 ? 4 : 2);
+  for (int i = 0; i < n; ++i)
+    if (!host[i].q || !host[i].k || !host[i].v || !host[i].o) return VSA_ERR_INVALID_ARG;
+  for (int s = 0; s < 2; ++s) {
+    vsa_status st = check_qkvo(&sets[s]);
+    if (st != VSA_OK) return st;
+  }
+  if (n == 0) return VSA_OK;
+  // events: uploaded[i], computed[i], downloaded[i] (host-side objects)
+  std::vector<cudaEvent_t> ev(3 * static_cast<size_t>(n), nullptr);
+  auto cleanup = [&]() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+  };
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      cleanup();
+      return VSA_ERR_CUDA;
+    }
+  vsa_status st = VSA_OK;
+  for (int i = 0; i < n && st == VSA_OK; ++i) {
+    const vsa_qkvo& d = sets[i % 2];
+    cudaEvent_t up = ev[3 * i], comp = ev[3 * i + 1], down = ev[3 * i + 2];
+    // upload: the set must no longer be read by batch i-2's compute
+    if (i >= 2 && cudaStreamWaitEvent(stream_up, ev[3 * (i - 2) + 1], 0) != cudaSuccess) st = VSA_ERR_CUDA;
+    if (st == VSA_OK &&
+        (cudaMemcpyAsync(const_cast<void*>(d.q), host[i].q, bytes, cudaMemcpyHostToDevice, stream_up) != cudaSuccess ||
+         cudaMemcpyAsync(const_cast<void*>(d.k), host[i].k, bytes, cudaMemcpyHostToDevice, stream_up) != cudaSuccess ||
+         cudaMemcpyAsync(const_cast<void*>(d.v), host[i].v, bytes, cudaMemcpyHostToDevice, stream_up) != cudaSuccess ||
+         cudaEventRecord(up, stream_up) != cudaSuccess))
+      st = VSA_ERR_CUDA;
+    // compute: inputs uploaded, and batch i-2's output has left this set's o
+    if (st == VSA_OK && cudaStreamWaitEvent(stream_compute, up, 0) != cudaSuccess) st = VSA_ERR_CUDA;
+    if (st == VSA_OK && i >= 2 && cudaStreamWaitEvent(stream_compute, ev[3 * (i - 2) + 2], 0) != cudaSuccess)
+      st = VSA_ERR_CUDA;
+    if (st == VSA_OK)
+      st = vsa_attention(&d, dtype, shape, params, select, d_kind, d_mse, ws, ws_bytes, d_err, stream_compute);
+    if (st == VSA_OK && cudaEventRecord(comp, stream_compute) != cudaSuccess) st = VSA_ERR_CUDA;
+    // download
+    if (st == VSA_OK && (cudaStreamWaitEvent(stream_down, comp, 0) != cudaSuccess ||
+                         cudaMemcpyAsync(host[i].o, d.o, bytes, cudaMemcpyDeviceToHost, stream_down) != cudaSuccess ||
+                         cudaEventRecord(down, stream_down) != cudaSuccess))
+      st = VSA_ERR_CUDA;
+  }
+  cleanup();
+  return st;
+}
+
 vsa_status vsa_get_device_error(const int* d_err, cudaStream_t stream, int* host_err) {
   if (d_err == nullptr) return VSA_ERR_INVALID_ARG;
   int h = 0;

@@ -14,7 +14,7 @@
 
 namespace vsa {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;
 
 // Smallest e with a <= 448 * 2^e for a > 0: with a = f * 2^E, f in [0.5, 1), and
 // 448 = 0.875 * 2^9, that is E - 9 when f <= 0.875 and E - 8 otherwise.
@@ -72,6 +72,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_e4m3_kernel(const __nv
   for (int w = 1; w < kQuantThreads / 32; ++w) m = fmaxf(m, red[w]);
   const int e = e4m3_block_exponent(m);
   if (tid == 0) exps[static_cast<size_t>(bh) * g.nblk + b] = e;
+  // 2^-e as a float (exact for -126 <= -e <= 127; other exponents go through ldexpf)
+  const bool plain = e >= -127 && e <= 126;
+  const float inv = plain ? __int_as_float((127 - e) << 23) : 1.f;
+  auto scaled = [&](float x) { return plain ? x * inv : ldexpf(x, -e); };
   // x / 2^e is exact (a power-of-two scaling of a bf16 value); the conversion rounds to the
   // nearest e4m3 value, ties to even, saturating at 448
 #pragma unroll
@@ -81,9 +85,9 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_e4m3_kernel(const __nv
     uint32_t packed[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float x0 = ldexpf(__uint_as_float(w[2 * h] << 16), -e), x1 = ldexpf(__uint_as_float(w[2 * h] & 0xffff0000u), -e);
-      const float x2 = ldexpf(__uint_as_float(w[2 * h + 1] << 16), -e),
-                  x3 = ldexpf(__uint_as_float(w[2 * h + 1] & 0xffff0000u), -e);
+      const float x0 = scaled(__uint_as_float(w[2 * h] << 16)), x1 = scaled(__uint_as_float(w[2 * h] & 0xffff0000u));
+      const float x2 = scaled(__uint_as_float(w[2 * h + 1] << 16)),
+                  x3 = scaled(__uint_as_float(w[2 * h + 1] & 0xffff0000u));
       const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
       const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x2, x3), __NV_SATFINITE, __NV_E4M3);
       packed[h] = (lo & 0xffffu) | (hi << 16);

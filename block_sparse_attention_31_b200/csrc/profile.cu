@@ -39,6 +39,9 @@ constexpr int kMaxSplits = 16;  // key-range splits per row tile, at most
 // the dense running maximum is recomputed exactly: with a margin of 80, every probability the
 // 2^-126 flush can remove is below 2^-46 of the variant's own largest one.
 constexpr float kProfFlushMargin = 80.0f;
+// Merged masked-variant sums below this (2^-60 of the dense maximum) trigger the recompute:
+// 60 + 18 (at most 2^18 keys) stays inside kProfFlushMargin.
+constexpr float kProfLowSum = 8.673617379884035e-19f;  // 2^-60
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -203,12 +206,9 @@ __device__ __forceinline__ void set_bit_range(uint32_t (&m)[BN / 32], int lo, in
 // The spatial P.V reads the dense P with the rows outside the window disabled (the MMA's
 // output-lane mask); the temporal P.V reads a masked copy with rows that allow no key of the
 // block disabled.  Probabilities more than 2^126 below the running dense maximum flush to
-// zero, so each row also tracks the largest logit each masked variant allows in this split
-// and stores it as that variant's partial max (the dense partial max is the exponent base of
-// all three); the row-error kernel recomputes a variant with its own maximum when the
-// variant's largest logit over all splits lies more than kProfFlushMargin (base 2) below the
-// dense max of a split where the variant has keys.  Both P tiles live in shared memory so
-// that Q.K^T of block j+1 runs while the softmax of block j computes.
+// zero; the row-error kernel detects a masked variant that could have lost weight that way
+// from its merged sum and recomputes it with its own maximum.  Both P tiles live in shared
+// memory so that Q.K^T of block j+1 runs while the softmax of block j computes.
 template <int D, int BN>
 __global__ void __launch_bounds__(kProfThreads, 1)
     profile_attn3_kernel(const __grid_constant__ CUtensorMap tqs, const __grid_constant__ CUtensorMap tk,
@@ -386,7 +386,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     const int ts_lo = rg.z / g.F, tf_lo = rg.z - (rg.z / g.F) * g.F;
     const int ts_hi = t_any ? (rg.w - 1) / g.F : -1, tf_hi = t_any ? (rg.w - 1) - ((rg.w - 1) / g.F) * g.F : -1;
     float m = -INFINITY, l[3] = {0.f, 0.f, 0.f};
-    float mv_s = -INFINITY, mv_t = -INFINITY;  // largest allowed logit (base 2) of each masked variant
     {  // the spatial and temporal accumulators only ever accumulate: start them at zero
       float z[32];
 #pragma unroll
@@ -449,8 +448,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
       uint64_t rs2[2] = {0ull, 0ull};
       float rt4[4] = {0.f, 0.f, 0.f, 0.f};
-      float tx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // temporal-allowed max of x
-      if (sp_on) mv_s = fmaxf(mv_s, mx * sl2);
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN / 2; ++c) {
@@ -463,7 +460,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         if (warp_tp) {
           const uint32_t b = (mt[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
           rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
-          tx4[c & 3] = fmax3(tx4[c & 3], (b & 1u) ? x0 : -INFINITY, (b & 2u) ? x1 : -INFINITY);
         }
       }
       // the previous block's P.V products must be done: O stable, P tiles free
@@ -507,10 +503,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
           *reinterpret_cast<uint4*>(pPT + off) = make_uint4(m4[0], m4[1], m4[2], m4[3]);
         }
       }
-      {
-        const float tx = fmaxf(fmaxf(tx4[0], tx4[1]), fmaxf(tx4[2], tx4[3]));
-        if (tx != -INFINITY) mv_t = fmaxf(mv_t, tx + m_use);
-      }
       float rs0, rs1;
       f2_split(f2_add(rs2[0], rs2[1]), rs0, rs1);
       const float rs = rs0 + rs1;
@@ -531,15 +523,13 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
       tc_fence_after();
     }
-    // partials: the dense max m (the exponent base of all three variants) in the dense row,
-    // each masked variant's own largest allowed logit in its row, the sums l and the
-    // unnormalised O of each variant
+    // partials: (m, l) and unnormalised O of each variant (m is the dense max for all three)
     const size_t base = ((static_cast<size_t>(bh) * a.splits + split) * 3) * a.r_pad + tile * kPM + row;
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
       const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
       const bool have = ok && cnt > 0;
-      a.ml[prow * 2 + 0] = have ? (vv == 0 ? m : vv == 1 ? mv_s : mv_t) : -INFINITY;
+      a.ml[prow * 2 + 0] = have ? m : -INFINITY;
       a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
       float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
 #pragma unroll 1
@@ -622,11 +612,12 @@ __device__ float profile_variant_exact(const __nv_bfloat16* __restrict__ qrow, c
 
 // Merge the key splits of one sampled row of one head and accumulate its two squared errors
 // (one CTA of d threads per (row, head)); the per-row sums are reduced in fixed order below.
-// A split's sums are based on its dense max md; a masked variant's stored max is its own
-// largest allowed logit mv.  When the variant's largest logit over all splits, M_v, lies more
-// than kProfFlushMargin below md of a split where the variant has keys, that split's flush
-// at 2^-126 of md may have removed probabilities above 2^-46 of the variant's own maximum,
-// so the variant of this row is recomputed with its own maximum.
+// Every split's sums are based on its dense max md.  A masked variant's merged sum L, taken
+// against the largest md, is at least 2^(M_v - max md) with M_v the variant's largest logit
+// (base 2), and at most its key count times that.  When L >= kProfLowSum, M_v lies within
+// -log2(kProfLowSum) + 18 < kProfFlushMargin of every split's md, so no probability above
+// 2^-46 of the variant's own maximum was flushed; otherwise the variant of this row is
+// recomputed with its own maximum.
 __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __restrict__ opart,
                                                                 const float* __restrict__ ml, int r_pad,
                                                                 int splits, int d, double* __restrict__ row_err,
@@ -641,47 +632,36 @@ __global__ void __launch_bounds__(128) profile_row_error_kernel(const float* __r
 #pragma unroll
   for (int vv = 0; vv < 3; ++vv) {
     // all splits' partials are loaded before they are combined (at most kMaxSplits)
-    float ms[kMaxSplits], mv[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
-    float Mv = -INFINITY;
+    float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
 #pragma unroll
     for (int sp = 0; sp < kMaxSplits; ++sp) {
-      ms[sp] = mv[sp] = -INFINITY;
+      ms[sp] = -INFINITY;
       ls[sp] = os[sp] = 0.f;
       if (sp < splits) {
         const size_t prow = ((static_cast<size_t>(bh) * splits + sp) * 3 + vv) * r_pad + i;
-        const size_t drow = ((static_cast<size_t>(bh) * splits + sp) * 3) * r_pad + i;
-        ms[sp] = __ldg(ml + drow * 2);  // the split's dense max: the base of its sums
-        mv[sp] = __ldg(ml + prow * 2);  // the variant's own largest logit (the dense max for vv 0)
+        ms[sp] = __ldg(ml + prow * 2);
         ls[sp] = __ldg(ml + prow * 2 + 1);
         os[sp] = __ldg(opart + prow * d + x);
-        Mv = fmaxf(Mv, mv[sp]);
       }
     }
-    bool low = false;
+    float M = -INFINITY;
 #pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      low |= vv > 0 && mv[sp] != -INFINITY && Mv < ms[sp] - kProfFlushMargin;
-    if (low) {  // uniform across the CTA: every thread read the same (m, l) partials
+    for (int sp = 0; sp < kMaxSplits; ++sp) M = fmaxf(M, ms[sp]);
+    float L = 0.f, acc = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      if (ms[sp] == -INFINITY) continue;
+      const float w = exp2f(ms[sp] - M);
+      L += ls[sp] * w;
+      acc += os[sp] * w;
+    }
+    if (vv > 0 && !(L >= kProfLowSum)) {  // uniform across the CTA: every thread read the same sums
       const int4 rg = ranges[i];
       const bool tp = vv == 2;
       o[vv] = profile_variant_exact(qs + (static_cast<size_t>(bh) * r_pad + i) * d,
                                     k + static_cast<size_t>(bh) * g.N * d, v + static_cast<size_t>(bh) * g.N * d,
                                     tp ? rg.z : rg.x, tp ? rg.w : rg.y, tp, g, d, scale_log2);
       continue;
-    }
-    // reference: the largest dense max among the splits where the variant has keys, so that
-    // the variant's scaled sums stay far above the fp32 range's bottom
-    float M = -INFINITY;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      if (mv[sp] != -INFINITY) M = fmaxf(M, ms[sp]);
-    float L = 0.f, acc = 0.f;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-      if (mv[sp] == -INFINITY) continue;
-      const float w = exp2f(ms[sp] - M);
-      L += ls[sp] * w;
-      acc += os[sp] * w;
     }
     o[vv] = L > 0.f ? acc / L : 0.f;
   }

@@ -345,6 +345,33 @@ VSA_API vsa_status vsa_attention(const vsa_qkvo *io, vsa_dtype dtype, const vsa_
                          vsa_select select, uint8_t *d_kind, float *d_mse, void *ws, size_t ws_bytes, int *d_err,
                          cudaStream_t stream);
 
+/*
+ * The whole call on host batches: for every batch i, upload q, k, v from host memory into a
+ * device buffer set, run vsa_attention on it and download o back to host memory.  Two buffer
+ * sets alternate so that the upload of batch i+1 and the download of batch i-1 overlap the
+ * compute of batch i, on three caller streams.  Returns once everything is enqueued; the
+ * caller synchronises stream_down (the last download is on it) before reading the outputs.
+ * The library allocates no device memory: the sets and the workspace are the caller's.
+ *   host      [n] host pointers: q, k, v (read), o (written), each [B, H, N, d] in dtype; they
+ *             should be pinned (cudaHostAlloc or registered), else the copies do not overlap
+ *   sets      [2] device buffer sets: q, k, v, o [B, H, N, d] in dtype (lse NULL or [B, H, N])
+ *   the rest  as vsa_attention (one workspace, kind and MSE array for every batch: batches run
+ *             one after the other on stream_compute); for VSA_SELECT_GIVEN the kinds in d_kind
+ *             serve every batch
+ * Events that order the three streams are created and destroyed inside the call (host-side
+ * objects; the destroy calls release them once their work has completed).
+ */
+typedef struct {
+    const void *q, *k, *v;
+    void *o;
+} vsa_host_batch;
+
+VSA_API vsa_status vsa_attention_host(const vsa_host_batch *host, int n, const vsa_qkvo *sets, vsa_dtype dtype,
+                                      const vsa_shape *shape, const vsa_params *params, vsa_select select,
+                                      uint8_t *d_kind, float *d_mse, void *ws, size_t ws_bytes, int *d_err,
+                                      cudaStream_t stream_up, cudaStream_t stream_compute,
+                                      cudaStream_t stream_down);
+
 /* Byte offsets of the mask arrays inside vsa_attention's workspace (for inspection). */
 VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const vsa_params *params, vsa_dtype dtype,
                                           vsa_select select, size_t *off_bits, size_t *off_kv_idx,
