@@ -78,7 +78,9 @@ struct AttnCfg {
   static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_QK = QK8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, false, true);
-  static int smem_bytes(int ucap, int nwords) { return OFF_UNION + 4 * ucap + 8 * nwords + 4 * ucap * (BN / 32) + 1024; }
+  static int smem_bytes(int ucap, int nwords) {
+    return OFF_UNION + 4 * ucap + 8 * nwords + 4 * ucap * (BN / 32) + 4 * nwords + 1024;
+  }
 };
 
 // Barrier slots.
@@ -209,35 +211,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     __syncthreads();
   }
+  // Union of the two lists in ascending order: warp 0 turns the per-word counts of the OR-ed
+  // bitsets into word offsets; then every thread places the blocks of its bit positions.
+  uint32_t* woff = uvalid + a.ucap * (BN / 32);  // [nwords] offset of each word's first entry
   if (warp == 0) {
     int base = 0;
     for (int w0 = 0; w0 < nwords; w0 += 32) {
       const int w = w0 + lane;
-      const uint32_t u0 = w < nwords ? bits0[w] : 0u, u1 = w < nwords ? bits1[w] : 0u;
-      uint32_t u = u0 | u1;
-      const int c = __popc(u);
+      const int c = w < nwords ? __popc(bits0[w] | bits1[w]) : 0;
       int incl = c;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int n = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += n;
       }
-      int pos = base + incl - c;
-      while (u) {
-        const int b = __ffs(u) - 1;
-        u &= u - 1u;
-        const int kb = w * 32 + b;
-        uni[pos++] = static_cast<uint32_t>(kb) | (((u0 >> b) & 1u) ? kInTile0 : 0u) |
-                     (((u1 >> b) & 1u) ? kInTile1 : 0u) | (block_full(g, kind, kb) ? 0u : kPartial);
-      }
+      if (w < nwords) woff[w] = static_cast<uint32_t>(base + incl - c);
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) misc[2] = base;
-    __syncwarp();
-    // valid-key bits of the blocks that are not full (ragged tail, cube padding).  A cube
-    // block is one cube (V == BN); its slot r = (df*ch + dh)*cw + dw holds a token when the
-    // offsets fall inside the cube's real extent, and the offsets of r = 32w + lane are the
-    // same for every cube, so they are computed once.
+  }
+  __syncthreads();
+  for (int kb = tid; kb < nwords * 32; kb += nthr) {
+    const uint32_t u0 = bits0[kb >> 5], u1 = bits1[kb >> 5], b = kb & 31;
+    const uint32_t u = u0 | u1;
+    if (!((u >> b) & 1u)) continue;
+    const int pos = static_cast<int>(woff[kb >> 5]) + __popc(u & ((1u << b) - 1u));
+    uni[pos] = static_cast<uint32_t>(kb) | (((u0 >> b) & 1u) ? kInTile0 : 0u) | (((u1 >> b) & 1u) ? kInTile1 : 0u) |
+               (block_full(g, kind, kb) ? 0u : kPartial);
+  }
+  __syncthreads();
+  {
+    // valid-key bits of the blocks that are not full (ragged tail, cube padding), one union
+    // entry per warp at a time.  A cube block is one cube (V == BN); its slot
+    // r = (df*ch + dh)*cw + dw holds a token when the offsets fall inside the cube's real
+    // extent, and the offsets of r = 32w + lane are the same for every cube.
+    const int base = misc[2];
     int cdw[BN / 32], cdh[BN / 32], cdf[BN / 32];
     if (kind == kCube) {
 #pragma unroll
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         cdf[w] = r / (g.cw * g.ch);
       }
     }
-    for (int n = 0; n < base; ++n) {
+    for (int n = warp; n < base; n += nthr >> 5) {
       const uint32_t e = uni[n];
       if (!(e & kPartial)) continue;
       const int kb = static_cast<int>(e & kKbMask);
