@@ -42,6 +42,7 @@ constexpr float kProfFlushMargin = 80.0f;
 // Merged masked-variant sums below this (2^-60 of the dense maximum) trigger the recompute:
 // 60 + 18 (at most 2^18 keys) stays inside kProfFlushMargin.
 constexpr float kProfLowSum = 8.673617379884035e-19f;  // 2^-60
+static_assert(60.0f + 18.0f < kProfFlushMargin, "low-sum threshold outside the flush margin");
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 

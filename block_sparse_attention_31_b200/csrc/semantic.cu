@@ -4,8 +4,10 @@
 // cluster attends to.  The page gives no formulas; the readings used here:
 //   - Lloyd's k-means per head on the bf16 rows (as fp32), `iters` rounds of assignment then
 //     update, initial centroids the rows rho_j = floor((2j+1) N / (2C));
-//   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32, both dot products summed in dimension
-//     order with one fused multiply-add per term, ties to the smaller j;
+//   - assignment: argmin_j |c_j|^2 - 2 x.c_j, ties to the smaller j: |c_j|^2 in fp32 (fused
+//     multiply-adds in dimension order), x.c_j on the tensor cores as x.c_hi + x.c_lo with
+//     c = c_hi + c_lo + r split into two bf16 vectors (|r| <= 2^-18 |c| per element; the bf16
+//     products are exact and accumulate in fp32);
 //   - update: fp64 sum of the members in token order, divided by the count, rounded to fp32;
 //     an empty cluster keeps its centroid;
 //   - cluster-major order: slots sorted by (cluster, token);
@@ -31,18 +33,8 @@ namespace vsa {
 
 namespace {
 
-constexpr int kKmTile = 128;     // tokens and centroids per assignment tile
-constexpr int kKmThreads = 256;  // 16 x 16 threads; thread (ty, tx): tokens ty + 16i, centroids tx + 16j
 constexpr int kKeepThreads = 256;
 constexpr int kRowThreads = 256;
-
-constexpr int kKmLd = kKmTile + 4;   // centroid tile [D][kKmLd] fp32: 16-byte aligned rows
-constexpr int kKmLdB = kKmTile + 8;  // token tile [D][kKmLdB] bf16: 16-byte aligned rows
-
-template <int D>
-constexpr size_t assign_smem_bytes() {  // about 100 KB at D = 128: two CTAs per SM
-  return sizeof(float) * (D * kKmLd + kKmTile) + sizeof(__nv_bfloat16) * D * kKmLdB;
-}
 
 // |c|^2 of one centroid held in shared memory: fp32, dimension order, one fused multiply-add
 // per term (the first term of the assignment's distance).
@@ -63,128 +55,146 @@ __device__ __forceinline__ bool better(float dist, int j, float bd, int bj) {
 
 // cent[bh, j] = x[bh, rho_j] as fp32, and its squared norm.  128 threads, d <= 128.
 __global__ void __launch_bounds__(128) kmeans_init_kernel(const __nv_bfloat16* __restrict__ x, int N, int d, int C,
-                                                          float* __restrict__ cent, float* __restrict__ cnorm) {
+                                                          float* __restrict__ cent, float* __restrict__ cnorm,
+                                                          __nv_bfloat16* __restrict__ chi,
+                                                          __nv_bfloat16* __restrict__ clo) {
   __shared__ float row_s[128];
   const int j = blockIdx.x, bh = blockIdx.y;
   const long long r = ((2LL * j + 1) * N) / (2LL * C);
   const __nv_bfloat16* src = x + (static_cast<size_t>(bh) * N + r) * d;
   float* dst = cent + (static_cast<size_t>(bh) * C + j) * d;
+  const size_t o = (static_cast<size_t>(bh) * C + j) * d;
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
     const float v = __bfloat162float(src[k]);
     dst[k] = v;
     row_s[k] = v;
+    chi[o + k] = src[k];  // a bf16 row splits exactly: hi = the row, lo = 0
+    clo[o + k] = __float2bfloat16_rn(0.f);
   }
   __syncthreads();
   if (threadIdx.x == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(row_s, d);
 }
 
-// label[bh, t] = nearest centroid of token t.  One CTA: 128 tokens of one head against all
-// centroids, 128 at a time.  Thread (ty, tx) holds tokens ty*8 + i and centroids tx*8 + j
-// (i, j < 8); the tiles are stored transposed ([dimension][token or centroid]) so that each
-// thread reads its 8 values of one dimension with two 16-byte loads.
+// label[bh, t] on the tensor cores: one CTA of 128 threads per 128 tokens of one head.  For each
+// tile of 128 centroids, thread 0 loads the token tile (once) and the centroids' bf16 halves
+// with TMA and issues S = X C_hi^T + X C_lo^T (tcgen05, M128 N128 K16, fp32 in TMEM); then every
+// thread (one token, TMEM lane = token) reads its 128 scores and keeps the running argmin of
+// |c|^2 - 2 s (one rounding), ties to the smaller index.  Tokens past N and centroids past C
+// are zero rows of the TMA boxes; the latter are skipped.
+constexpr int kTcRows = 128;
+
 template <int D>
-__global__ void __launch_bounds__(kKmThreads, 2)
-    kmeans_assign_kernel(const __nv_bfloat16* __restrict__ x, int N, int C, const float* __restrict__ cent,
-                         const float* __restrict__ cnorm, int32_t* __restrict__ label) {
-  extern __shared__ __align__(16) float km_smem[];
-  float* cs = km_smem;            // [D][kKmLd]
-  float* nc = cs + D * kKmLd;     // [128]
-  uint16_t* xs = reinterpret_cast<uint16_t*>(nc + kKmTile);  // [D][kKmLdB] bf16 bits
-  const int bh = blockIdx.y, t0 = blockIdx.x * kKmTile;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * N * D;
-  const float* chd = cent + static_cast<size_t>(bh) * C * D;
-  // token tile: thread e loads 8 dimensions of row e % 128
-  for (int e = tid; e < kKmTile * (D / 8); e += kKmThreads) {
-    const int r = e & (kKmTile - 1), c8 = e / kKmTile;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (t0 + r < N) w = *reinterpret_cast<const uint4*>(xh + static_cast<size_t>(t0 + r) * D + c8 * 8);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      xs[(c8 * 8 + 2 * q) * kKmLdB + r] = static_cast<uint16_t>(ww[q] & 0xffffu);
-      xs[(c8 * 8 + 2 * q + 1) * kKmLdB + r] = static_cast<uint16_t>(ww[q] >> 16);
-    }
+struct KmTcCfg {
+  static constexpr int X_BYTES = kTcRows * D * 2;
+  static constexpr int C_BYTES = kTcRows * D * 2;
+  static constexpr int OFF_X = 0, OFF_HI = X_BYTES, OFF_LO = X_BYTES + C_BYTES, OFF_BAR = X_BYTES + 2 * C_BYTES;
+  static constexpr int SMEM = OFF_BAR + 64 + 1024;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(kTcRows, kTcRows, false, false);
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tx,
+                                                               const __grid_constant__ CUtensorMap thi,
+                                                               const __grid_constant__ CUtensorMap tlo, int N, int C,
+                                                               const float* __restrict__ cnorm,
+                                                               int32_t* __restrict__ label, int* err) {
+  using K = KmTcCfg<D>;
+  extern __shared__ uint8_t km_raw[];
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  __shared__ float cn[kTcRows];
+  const uint32_t raw = smem_u32(km_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  const uint32_t sX = sb + K::OFF_X, sHi = sb + K::OFF_HI, sLo = sb + K::OFF_LO;
+  const uint32_t bLoad = sb + K::OFF_BAR, bMma = bLoad + 8;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y, t0 = blockIdx.x * kTcRows;
+  volatile int* abort_flag = &abort_s;
+  if (tid == 0) {
+    mbar_init(bLoad, 1);
+    mbar_init(bMma, 1);
+    mbar_init_fence();
+    abort_s = 0;
   }
-  float best_d[8];
-  int best_j[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    best_d[i] = 0.f;
-    best_j[i] = -1;
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_s), 128);
+    tmem_relinquish();
   }
-  for (int c0 = 0; c0 < C; c0 += kKmTile) {
-    __syncthreads();  // the previous tile's reads of cs and nc are done
-    for (int e = tid; e < kKmTile * (D / 4); e += kKmThreads) {
-      const int r = e & (kKmTile - 1), c4 = e / kKmTile;
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + r < C) w = *reinterpret_cast<const float4*>(chd + static_cast<size_t>(c0 + r) * D + c4 * 4);
-      cs[(c4 * 4 + 0) * kKmLd + r] = w.x;
-      cs[(c4 * 4 + 1) * kKmLd + r] = w.y;
-      cs[(c4 * 4 + 2) * kKmLd + r] = w.z;
-      cs[(c4 * 4 + 3) * kKmLd + r] = w.w;
-    }
-    if (tid < kKmTile) nc[tid] = c0 + tid < C ? cnorm[static_cast<size_t>(bh) * C + c0 + tid] : 0.f;
-    __syncthreads();
-    // acc2[i][p] packs the sums of centroids tx*8 + 2p and tx*8 + 2p + 1; every lane of
-    // fma.rn.f32x2 is one correctly rounded fused multiply-add, as __fmaf_rn
-    uint64_t acc2[8][4];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  float best_d = 0.f;
+  int best_j = -1;
+  bool ok = true;
+  const int ntiles = (C + kTcRows - 1) / kTcRows;
+  for (int ct = 0; ct < ntiles && ok; ++ct) {
+    const int c0 = ct * kTcRows;
+    if (tid == 0) {
+      const uint32_t bytes = (ct == 0 ? K::X_BYTES : 0) + 2 * K::C_BYTES;
+      mbar_arrive_expect_tx(bLoad, bytes);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+      for (int c = 0; c < D / 64; ++c) {
+        if (ct == 0) tma_load_3d(sX + c * kTcRows * 128, &tx, bLoad, c * 64, t0, bh);
+        tma_load_3d(sHi + c * kTcRows * 128, &thi, bLoad, c * 64, c0, bh);
+        tma_load_3d(sLo + c * kTcRows * 128, &tlo, bLoad, c * 64, c0, bh);
+      }
+      if (mbar_wait(bLoad, ct & 1, abort_flag, err)) {
+        tc_fence_after();
+        const uint64_t dx = sdesc_sw128(sX, 16, 1024), dh = sdesc_sw128(sHi, 16, 1024),
+                       dl = sdesc_sw128(sLo, 16, 1024);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) acc2[i][p] = 0ull;
-#pragma unroll 2
-    for (int k = 0; k < D; ++k) {
-      const uint4 aw = *reinterpret_cast<const uint4*>(xs + k * kKmLdB + ty * 8);  // 8 bf16 tokens
-      const ulonglong2 b_lo = *reinterpret_cast<const ulonglong2*>(cs + k * kKmLd + tx * 8);
-      const ulonglong2 b_hi = *reinterpret_cast<const ulonglong2*>(cs + k * kKmLd + tx * 8 + 4);
-      const uint64_t b2[4] = {b_lo.x, b_lo.y, b_hi.x, b_hi.y};
-      const uint32_t awv[4] = {aw.x, aw.y, aw.z, aw.w};
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (kTcRows * 128) + (kk & 3) * 32) / 16);
+          tc_mma_ss(tmem, dx + off, dh + off, K::IDESC, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float a = __uint_as_float((i & 1) ? (awv[i >> 1] & 0xffff0000u) : (awv[i >> 1] << 16));
-        const uint64_t a2 = f2_make(a, a);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) acc2[i][p] = f2_fma(a2, b2[p], acc2[i][p]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (kTcRows * 128) + (kk & 3) * 32) / 16);
+          tc_mma_ss(tmem, dx + off, dl + off, K::IDESC, 1u);
+        }
+        tc_commit(bMma);
+      } else {
+        mbar_wait_drain(bLoad, ct & 1, err);  // the copies land before the CTA moves on
       }
     }
-    __syncthreads();  // nc visible to every thread
+    cn[tid] = c0 + tid < C ? cnorm[static_cast<size_t>(bh) * C + c0 + tid] : 0.f;
+    ok = __syncthreads_and(!*abort_flag);
+    if (!ok) break;
+    ok = __syncthreads_and(mbar_wait(bMma, ct & 1, abort_flag, err));
+    if (!ok) {
+      if (tid == 0) mbar_wait_drain(bMma, ct & 1, err);  // the MMAs were issued: let them finish
+      break;
+    }
+    tc_fence_after();
+    const int nc = min(kTcRows, C - c0);
+#pragma unroll 1
+    for (int q = 0; q < kTcRows / 32; ++q) {
+      if (q * 32 >= nc) break;
+      float sv[32];
+      tmem_ld32(t_lane + q * 32, sv);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int jl = tx * 8 + 2 * p + h, cj = c0 + jl;
-        if (cj < C) {
-          const float n = nc[jl];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float lo, hi;
-            f2_split(acc2[i][p], lo, hi);
-            const float dist = __fmaf_rn(-2.f, h ? hi : lo, n);  // n - 2 dot, rounded once
-            if (better(dist, cj, best_d[i], best_j[i])) {
-              best_d[i] = dist;
-              best_j[i] = cj;
-            }
+      for (int x = 0; x < 32; ++x) {
+        const int jl = q * 32 + x;
+        if (jl < nc) {
+          const float dist = __fmaf_rn(-2.f, sv[x], cn[jl]);  // |c|^2 - 2 s, rounded once
+          if (better(dist, c0 + jl, best_d, best_j)) {
+            best_d = dist;
+            best_j = c0 + jl;
           }
         }
       }
     }
+    tc_fence_before();
+    __syncthreads();  // every thread has read S and cn before the next tile overwrites them
   }
-  // the 16 threads of a half-warp share their tokens: reduce (distance, index) lexicographically
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) {
-      const float od = __shfl_xor_sync(0xffffffffu, best_d[i], off);
-      const int oj = __shfl_xor_sync(0xffffffffu, best_j[i], off);
-      if (oj >= 0 && better(od, oj, best_d[i], best_j[i])) {
-        best_d[i] = od;
-        best_j[i] = oj;
-      }
-    }
-    const int t = t0 + ty * 8 + i;
-    if (tx == 0 && t < N) label[static_cast<size_t>(bh) * N + t] = best_j[i];
-  }
+  const int t = t0 + tid;
+  if (ok && t < N) label[static_cast<size_t>(bh) * N + t] = best_j;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // Counts, offsets and the stable cluster-major order of one head.  The head's tokens are cut
@@ -306,7 +316,9 @@ __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(const __nv_b
                                                                     const int32_t* __restrict__ offsets,
                                                                     const int32_t* __restrict__ perm,
                                                                     float* __restrict__ cent,
-                                                                    float* __restrict__ cnorm) {
+                                                                    float* __restrict__ cnorm,
+                                                                    __nv_bfloat16* __restrict__ chi,
+                                                                    __nv_bfloat16* __restrict__ clo) {
   extern __shared__ __align__(16) uint4 upd_smem[];
   constexpr int VPR = D * 2 / 16;                        // 16-byte pieces per row
   constexpr int PER_T = kUpdRows * VPR / kUpdThreads;    // pieces per thread per stage
@@ -354,8 +366,12 @@ __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(const __nv_b
   float* cnew = reinterpret_cast<float*>(upd_smem);  // the staged rows are no longer read
   if (tid < D) {
     const float c = __double2float_rn(__ddiv_rn(s, static_cast<double>(n)));
-    cent[(static_cast<size_t>(bh) * C + j) * D + tid] = c;
+    const size_t o = (static_cast<size_t>(bh) * C + j) * D + tid;
+    cent[o] = c;
     cnew[tid] = c;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(c);
+    chi[o] = hi;
+    clo[o] = __float2bfloat16_rn(__fsub_rn(c, __bfloat162float(hi)));
   }
   __syncthreads();
   if (tid == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(cnew, D);
@@ -582,45 +598,63 @@ int rows_grid_x(int N, int vpr, int BH) {
 
 template <int D>
 cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, float* cent, int32_t* label,
-                     int32_t* counts, int32_t* perm, int32_t* offsets, float* cnorm, int* err, cudaStream_t stream) {
-  constexpr size_t smem = assign_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                     int32_t* counts, int32_t* perm, int32_t* offsets, float* cnorm, __nv_bfloat16* chi,
+                     __nv_bfloat16* clo, int* err, cudaStream_t stream) {
+  using K = KmTcCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
   const size_t ssmem = sizeof(int) * (kSortWarps + 1) * static_cast<size_t>(C);
   if (ssmem > 48 * 1024) {
     e = cudaFuncSetAttribute(kmeans_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem));
     if (e != cudaSuccess) return e;
   }
-  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, cnorm);
+  CUtensorMap tx, thi, tlo;
+  if ((e = encode_rows_map(&tx, x, D, N, BH, kTcRows)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(&thi, chi, D, C, BH, kTcRows)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(&tlo, clo, D, C, BH, kTcRows)) != cudaSuccess) return e;
+  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, cnorm, chi, clo);
   constexpr size_t usmem = update_smem_bytes<D>();
   e = cudaFuncSetAttribute(kmeans_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(usmem));
   if (e != cudaSuccess) return e;
-  const dim3 agrid((N + kKmTile - 1) / kKmTile, BH), ugrid(C, BH);
+  const dim3 agrid((N + kTcRows - 1) / kTcRows, BH), ugrid(C, BH);
   for (int it = 0; it < iters; ++it) {
-    kmeans_assign_kernel<D><<<agrid, kKmThreads, smem, stream>>>(x, N, C, cent, cnorm, label);
+    kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, cnorm, label, err);
     kmeans_sort_kernel<<<BH, kSortWarps * 32, ssmem, stream>>>(label, N, C, counts, offsets, perm, err);
-    kmeans_update_kernel<D><<<ugrid, kUpdThreads, usmem, stream>>>(x, N, C, counts, offsets, perm, cent, cnorm);
+    kmeans_update_kernel<D><<<ugrid, kUpdThreads, usmem, stream>>>(x, N, C, counts, offsets, perm, cent, cnorm, chi,
+                                                                   clo);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t kmeans_workspace_bytes(int BH, int C) {
-  const size_t offs = (static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
-  return offs + ((static_cast<size_t>(BH) * C * sizeof(float) + 255) & ~static_cast<size_t>(255));
+namespace {
+constexpr size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+}  // namespace
+
+size_t kmeans_workspace_bytes(int BH, int C, int d) {
+  const size_t offs = round256(static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t));
+  const size_t norms = round256(static_cast<size_t>(BH) * C * sizeof(float));
+  const size_t half = round256(static_cast<size_t>(BH) * C * d * sizeof(__nv_bfloat16));
+  return offs + norms + 2 * half;
 }
 
 cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
                           int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream) {
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  int32_t* offsets = static_cast<int32_t*>(ws);
-  const size_t offs = (static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
-  float* cnorm = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + offs);
-  if (d == 128) return kmeans_d<128>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, err, stream);
-  if (d == 64) return kmeans_d<64>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, err, stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const size_t offs = round256(static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t));
+  const size_t norms = round256(static_cast<size_t>(BH) * C * sizeof(float));
+  const size_t half = round256(static_cast<size_t>(BH) * C * d * sizeof(__nv_bfloat16));
+  int32_t* offsets = reinterpret_cast<int32_t*>(w);
+  float* cnorm = reinterpret_cast<float*>(w + offs);
+  __nv_bfloat16* chi = reinterpret_cast<__nv_bfloat16*>(w + offs + norms);
+  __nv_bfloat16* clo = reinterpret_cast<__nv_bfloat16*>(w + offs + norms + half);
+  if (d == 128)
+    return kmeans_d<128>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, chi, clo, err, stream);
+  if (d == 64)
+    return kmeans_d<64>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, chi, clo, err, stream);
   return cudaErrorInvalidValue;
 }
 

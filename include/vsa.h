@@ -383,8 +383,10 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
  * formulas; the readings:
  *   - Lloyd's k-means per head on the bf16 rows (as fp32), `iters` rounds of assignment then
  *     update, starting from the rows floor((2j+1) N / (2C)), j < C;
- *   - assignment: argmin_j |c_j|^2 - 2 x.c_j in fp32, both dot products summed in dimension
- *     order with one fused multiply-add per term, ties to the smaller j;
+ *   - assignment: argmin_j |c_j|^2 - 2 x.c_j, ties to the smaller j; |c_j|^2 in fp32 (fused
+ *     multiply-adds in dimension order), x.c_j on the tensor cores from the two bf16 halves
+ *     of c_j (c_hi + c_lo, within 2^-18 |c_j| per element), fp32 accumulation.  Where two
+ *     centroids are within the rounding error of a tie, either label is a correct answer;
  *   - update: fp64 sum of the members in token order / count, rounded to fp32; an empty
  *     cluster keeps its centroid;
  *   - cluster-major order: slots sorted by (cluster, token);
@@ -397,8 +399,9 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
  * rows, 1 <= C <= min(N, 1024) clusters and 1 <= iters <= 1000.
  * ------------------------------------------------------------------------------------- */
 
-/* Scratch bytes of vsa_kmeans (cluster offsets and centroid norms); 0 for an invalid shape or
- * count. */
+/* Scratch bytes of vsa_kmeans: cluster offsets [B*H, C+1] int32, centroid norms [B*H, C] fp32
+ * and the centroids' bf16 halves [B*H, C, d] twice, each 256-byte aligned; 0 for an invalid
+ * shape or count. */
 VSA_API size_t vsa_kmeans_workspace_size(const vsa_shape *shape, int n_clusters);
 
 /*

@@ -168,9 +168,9 @@ def test_semantic_entry_points_validate_before_launch():
     s = ctypes.c_void_p(0)
     shape = _lib.make_shape(1, 2, 4, 8, 8, 64, 64)          # N = 256
     cube = _lib.make_shape(1, 2, 8, 8, 8, 64, 128, (4, 4, 8))
-    # offsets B*H*(C+1) int32 and norms B*H*C fp32, each 256-aligned
-    assert _lib.vsa_kmeans_workspace_size(shape, 16) == 256 + 256
-    assert _lib.vsa_kmeans_workspace_size(shape, 64) == 768 + 512
+    # offsets B*H*(C+1) int32, norms B*H*C fp32 and two bf16 halves B*H*C*d, each 256-aligned
+    assert _lib.vsa_kmeans_workspace_size(shape, 16) == 256 + 256 + 2 * 4096
+    assert _lib.vsa_kmeans_workspace_size(shape, 64) == 768 + 512 + 2 * 16384
     assert _lib.vsa_kmeans_workspace_size(shape, 0) == 0
     assert _lib.vsa_kmeans_workspace_size(shape, 257) == 0   # more clusters than rows
     assert _lib.vsa_kmeans_workspace_size(cube, 16) == 0

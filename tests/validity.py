@@ -33,11 +33,16 @@ def _log(category: str, detail: str):
 
 
 def labels_valid(x, cent, lab_gpu, what: str = "") -> int:
-    """k-means labels.  The kernel computes D_j = |c_j|^2 - 2 x.c_j with fp32 fused
-    multiply-add chains of d terms (and one rounding of the final combination), so its error
-    is at most E_j = gamma_d (|c_j|^2 + 2 sum_i |x_i c_ji|) + u |D_j|, gamma_d = d u / (1 - d u).
-    A label j_g other than the oracle's j_o is accepted when the fp64 distances satisfy
-    dist(j_g) - dist(j_o) <= 2 (E_jg + E_jo).  Returns the number of accepted differences."""
+    """k-means labels.  The kernel computes D_j = fl(|c_j|^2 - 2 s_j) with one rounding, where
+    |c_j|^2 is an fp32 fused multiply-add chain of d terms (error <= gamma_d |c_j|^2) and
+    s_j = x.c_hi + x.c_lo comes from the tensor cores: c_j = c_hi + c_lo + r with bf16 halves,
+    |r_i| <= 2^-18 |c_ji|, every product exact, 2d of them accumulated in fp32.  Allowing each
+    accumulation step an error of 2u (a truncating adder), |s_j - x.c_j| <= (gamma'_2d
+    (1 + 2^-8) + 2^-18) sum_i |x_i c_ji| with gamma'_2d = 4du / (1 - 4du).  So the error of D_j
+    is at most E_j = gamma_d |c_j|^2 + 2 (gamma'_2d (1 + 2^-8) + 2^-18) sum_i |x_i c_ji| + u |D_j|
+    (gamma_d = du / (1 - du), u = 2^-24).  A label j_g other than the oracle's j_o is accepted
+    when the fp64 distances satisfy dist(j_g) - dist(j_o) <= 2 (E_jg + E_jo).  Returns the
+    number of accepted differences."""
     x = np.asarray(x, dtype=np.float32)
     cent = np.asarray(cent, dtype=np.float32)
     lab_gpu = np.asarray(lab_gpu)
@@ -47,12 +52,14 @@ def labels_valid(x, cent, lab_gpu, what: str = "") -> int:
         return 0
     d = x.shape[1]
     gamma = d * U32 / (1 - d * U32)
+    gamma_tc = 4 * d * U32 / (1 - 4 * d * U32)
     x64, c64 = x.astype(np.float64), cent.astype(np.float64)
 
     def err(t, j):
         c = c64[j]
         D = c @ c - 2.0 * (x64[t] @ c)
-        return gamma * (c @ c + 2.0 * np.abs(x64[t] * c).sum()) + U32 * abs(D)
+        dot = (gamma_tc * (1 + 2.0 ** -8) + 2.0 ** -18) * np.abs(x64[t] * c).sum()
+        return gamma * (c @ c) + 2.0 * dot + U32 * abs(D)
 
     for t in diff:
         jg, jo = int(lab_gpu[t]), int(lab_o[t])
