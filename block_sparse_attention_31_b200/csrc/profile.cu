@@ -15,7 +15,8 @@
 //   attn3    one CTA per (head, 128-row tile, key split): S = Q K^T on tcgen05 into TMEM,
 //            one online softmax whose probabilities serve the dense, spatial-masked and
 //            temporal-masked variants, and three P.V products into three TMEM accumulators
-//            (the masked ones with rows switched off by the MMA's lane mask); writes the
+//            (the masked ones with rows switched off by the MMA's lane mask); the softmax runs
+//            on two warpgroups, each owning one half of every row's columns; writes the
 //            partial (max, sum, unnormalised O) of each variant;
 //   row_error one CTA per (sampled row, head): merges the splits, forms the three outputs and
 //            the row's two squared errors (fp64);
@@ -31,7 +32,7 @@
 
 namespace vsa {
 
-constexpr int kProfThreads = 192;
+constexpr int kProfThreads = 320;  // producer, MMA issuer, two softmax warpgroups
 constexpr int kPM = 128;  // rows per tile
 constexpr int kNumSMs = 148;
 constexpr int kMaxSplits = 16;  // key-range splits per row tile, at most
@@ -168,7 +169,8 @@ struct ProfCfg {
   static constexpr int OFF_PT = OFF_PD + P_BYTES;     // temporal-masked P
   static constexpr int OFF_BAR = OFF_PT + P_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
-  static constexpr int BYTES = OFF_MISC + 128;
+  static constexpr int OFF_XMAX = OFF_MISC + 128;     // [2 halves][kPM] partial row maxima
+  static constexpr int BYTES = OFF_XMAX + 2 * kPM * 4;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   // TMEM: S, then O of dense, spatial, temporal
   static constexpr int TMEM_S = 0, TMEM_O = BN;
@@ -178,7 +180,7 @@ struct ProfCfg {
 };
 
 enum { PB_Q = 0, PB_FULL_K = 1, PB_FULL_V = 3, PB_EMPTY_K = 5, PB_EMPTY_V = 7, PB_S_FULL = 9, PB_S_FREE = 10,
-       PB_P_FULL = 11, PB_O_DONE = 12, PB_DRAIN = 13 };
+       PB_P_FULL = 11, PB_O_DONE = 12, PB_DRAIN = 13, PB_X_FULL = 14 };
 
 struct ProfArgs {
   const int4* ranges;
@@ -223,6 +225,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   const uint32_t sPD = sbase + C::OFF_PD, sPT = sbase + C::OFF_PT;
   uint8_t* pPD = smem + C::OFF_PD;
   uint8_t* pPT = smem + C::OFF_PT;
+  volatile float* xmax = reinterpret_cast<volatile float*>(smem + C::OFF_XMAX);
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
@@ -250,10 +253,11 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       mbar_init(bar(PB_EMPTY_V + st), 1);
     }
     mbar_init(bar(PB_S_FULL), 1);
-    mbar_init(bar(PB_S_FREE), 128);
-    mbar_init(bar(PB_P_FULL), 128);
+    mbar_init(bar(PB_S_FREE), 256);
+    mbar_init(bar(PB_P_FULL), 256);
     mbar_init(bar(PB_O_DONE), 1);
     mbar_init(bar(PB_DRAIN), 1);
+    mbar_init(bar(PB_X_FULL), 256);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -375,8 +379,15 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     }
     __syncwarp();
   } else {
-    const int quad = warp & 3;
+    // Two softmax warpgroups split every S row by columns: warp w (2..9) serves the TMEM lane
+    // quarter w % 4 and the column half h = (w - 2) / 4.  The two threads of a row exchange
+    // their halves' maxima through shared memory (so they take the same rescale decisions),
+    // exponentiate their own half, write their half of each P tile and keep partial sums,
+    // which are added at the end (half 0 + half 1).
+    constexpr int HB = BN / 2;
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
+    const int c_own = half * HB;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t t_s = t_lane + C::TMEM_S, t_o = t_lane + C::TMEM_O;
     const float sl2 = a.scale_log2;
@@ -392,35 +403,47 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int x = 0; x < 32; ++x) z[x] = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 2 * D / 32; ++c) tmem_st32(t_o + D + c * 32, z);
+      for (int c = 0; c < D / 32; ++c) tmem_st32(t_o + D + half * D + c * 32, z);
     }
     bool ok = true;
     for (int j = 0; j < cnt; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_S_FULL), j & 1, abort_flag, a.err));
       if (!ok) break;
       tc_fence_after();
-      float s[BN];
+      uint32_t rs_own[HB];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, s + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar(PB_S_FREE));  // S may be overwritten by the next block's Q.K^T
+      for (int c = 0; c < HB / 32; ++c) tmem_ld32_async(t_s + c_own + c * 32, rs_own + c * 32);
+      tmem_wait_ld();
+      reg_fence<HB>(rs_own);
       const int t0 = (kb0 + j) * BN;
       const int nvalid = min(BN, g.N - t0);
-      if (nvalid < BN) {
+      float s[HB];
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c >= nvalid) s[c] = -INFINITY;
+      for (int c = 0; c < HB; ++c) s[c] = __uint_as_float(rs_own[c]);
+      if (nvalid < BN) {  // the ragged last block
+#pragma unroll
+        for (int c = 0; c < HB; ++c)
+          if (c_own + c >= nvalid) s[c] = -INFINITY;
       }
       float mx8[8];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
+      for (int x = 0; x < 8; ++x) mx8[x] = fmax3(s[2 * x], s[2 * x + 1], -INFINITY);
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 16; c < HB; c += 2) mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
+      // the row maximum: exchange the two halves' partial maxima (every thread has read the
+      // other half's value before it releases S, so the next block's writes come after it)
+      xmax[half * kPM + row] = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                     fmaxf(mx8[6], mx8[7]));
+      mbar_arrive(bar(PB_X_FULL));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_X_FULL), j & 1, abort_flag, a.err));
+      if (!ok) break;
+      const float mx = fmaxf(xmax[row], xmax[kPM + row]);
+      tc_fence_before();
+      mbar_arrive(bar(PB_S_FREE));  // S may be overwritten by the next block's Q.K^T
       const float m_new = fmaxf(m, mx * sl2);
       const bool grow = m_new > m + kRescaleLog2;
       // masks: spatial whole block; temporal as contiguous column ranges per frame segment
+      // (the whole row, so both halves know whether the row uses the temporal P tile)
       const bool sp_on = t0 >= rg.x && t0 < rg.y;
       uint32_t mt[BN / 32];
 #pragma unroll
@@ -441,17 +464,20 @@ __global__ void __launch_bounds__(kProfThreads, 1)
 #pragma unroll
       for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
       const bool tp_on = tany != 0u;
-      // Exponentials first, into registers (packed bf16 pairs): this overlaps the previous
-      // block's P.V products, which still read the P tiles.
+      uint32_t mh[HB / 32];  // this half's mask words (static indexing below)
+#pragma unroll
+      for (int w = 0; w < HB / 32; ++w) mh[w] = half ? mt[HB / 32 + w] : mt[w];
+      // Exponentials of this half first, into registers (packed bf16 pairs): this overlaps the
+      // previous block's P.V products, which still read the P tiles.
       const float m_next = grow ? m_new : m;
       const float m_use = m_next == -INFINITY ? 0.f : m_next;
       const bool warp_tp = __any_sync(0xffffffffu, tp_on);
       const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
       uint64_t rs2[2] = {0ull, 0ull};
       float rt4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[BN / 2];
+      uint32_t pk[HB / 2], pt[HB / 2];  // packed P and its temporal-masked copy
 #pragma unroll
-      for (int c = 0; c < BN / 2; ++c) {
+      for (int c = 0; c < HB / 2; ++c) {
         const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
         float x0, x1;
         f2_split(x, x0, x1);
@@ -459,8 +485,9 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
         pk[c] = pack_bf16x2(p0, p1);
         if (warp_tp) {
-          const uint32_t b = (mt[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
+          const uint32_t b = (mh[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
           rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+          pt[c] = pk[c] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
         }
       }
       // the previous block's P.V products must be done: O stable, P tiles free
@@ -470,14 +497,16 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         tc_fence_after();
       }
       if (j > 0 && __any_sync(0xffffffffu, grow && m != -INFINITY)) {
+        // this half rescales its 3D/2 of the three accumulators' columns
         const float alpha = grow ? fast_exp2(m - m_new) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 3 * D / 32; ++c) {
+        for (int c = 0; c < 3 * D / 64; ++c) {
           float o[32];
-          tmem_ld32(t_o + c * 32, o);
+          const uint32_t col = static_cast<uint32_t>(half * (3 * D / 2) + c * 32);
+          tmem_ld32(t_o + col, o);
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] *= alpha;
-          tmem_st32(t_o + c * 32, o);
+          tmem_st32(t_o + col, o);
         }
       }
       if (grow) {
@@ -488,21 +517,14 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         m = m_new;
       }
 #pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {  // 8 probabilities -> one 16-byte chunk of each P tile
+      for (int ch = 0; ch < HB / 8; ++ch) {  // 8 probabilities -> one 16-byte chunk of each P tile
+        const int gch = half * (HB / 8) + ch;
         const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        const int kc = ch >> 3, cc = ch & 7;
+        const int kc = gch >> 3, cc = gch & 7;
         const int off = kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(pPD + off) = v4;
-        if (tp_on) {
-          uint32_t m4[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int col = ch * 8 + 2 * x;
-            const uint32_t b = (mt[col >> 5] >> (col & 31)) & 3u;
-            m4[x] = pk[4 * ch + x] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
-          }
-          *reinterpret_cast<uint4*>(pPT + off) = make_uint4(m4[0], m4[1], m4[2], m4[3]);
-        }
+        if (tp_on)
+          *reinterpret_cast<uint4*>(pPT + off) = make_uint4(pt[4 * ch], pt[4 * ch + 1], pt[4 * ch + 2], pt[4 * ch + 3]);
       }
       float rs0, rs1;
       f2_split(f2_add(rs2[0], rs2[1]), rs0, rs1);
@@ -512,7 +534,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       if (sp_on) l[1] += rs;
       l[2] += rt;
       const uint32_t bs = __ballot_sync(0xffffffffu, sp_on), bt = __ballot_sync(0xffffffffu, tp_on);
-      if (lane == 0) {
+      if (lane == 0 && half == 0) {
         rowuse[(j & 1) * 8 + quad] = bs;
         rowuse[(j & 1) * 8 + 4 + quad] = bt;
       }
@@ -524,20 +546,35 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_O_DONE), (cnt - 1) & 1, abort_flag, a.err));
       tc_fence_after();
     }
-    // partials: (m, l) and unnormalised O of each variant (m is the dense max for all three)
+    const bool have = ok && cnt > 0;
+    // the halves' partial sums, added as half 0 + half 1 (the last P.V has read the dense P
+    // tile, which now holds half 1's sums)
+    float* lx = reinterpret_cast<float*>(pPD);
+    if (half == 1) {
+#pragma unroll
+      for (int vv = 0; vv < 3; ++vv) lx[vv * kPM + row] = have ? l[vv] : 0.f;
+    }
+    named_barrier_sync(1, 8 * 32);
+    if (half == 0) {
+#pragma unroll
+      for (int vv = 0; vv < 3; ++vv) l[vv] += lx[vv * kPM + row];
+    }
+    // partials: (m, l) and unnormalised O of each variant (m is the dense max for all three);
+    // each half writes its D/2 output columns
     const size_t base = ((static_cast<size_t>(bh) * a.splits + split) * 3) * a.r_pad + tile * kPM + row;
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
       const size_t prow = base + static_cast<size_t>(vv) * a.r_pad;
-      const bool have = ok && cnt > 0;
-      a.ml[prow * 2 + 0] = have ? m : -INFINITY;
-      a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
-      float4* dst = reinterpret_cast<float4*>(a.opart + prow * D);
+      if (half == 0) {
+        a.ml[prow * 2 + 0] = have ? m : -INFINITY;
+        a.ml[prow * 2 + 1] = have ? l[vv] : 0.f;
+      }
+      float4* dst = reinterpret_cast<float4*>(a.opart + prow * D + half * (D / 2));
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         float o[32];
         if (have) {
-          tmem_ld32(t_o + vv * D + c * 32, o);
+          tmem_ld32(t_o + vv * D + half * (D / 2) + c * 32, o);
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] = 0.f;
