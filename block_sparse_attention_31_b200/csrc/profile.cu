@@ -476,18 +476,29 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       uint64_t rs2[2] = {0ull, 0ull};
       float rt4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[HB / 2], pt[HB / 2];  // packed P and its temporal-masked copy
+      if (warp_tp) {  // one branch per block, not per pair
 #pragma unroll
-      for (int c = 0; c < HB / 2; ++c) {
-        const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
-        float x0, x1;
-        f2_split(x, x0, x1);
-        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-        rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
-        pk[c] = pack_bf16x2(p0, p1);
-        if (warp_tp) {
+        for (int c = 0; c < HB / 2; ++c) {
+          const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
+          float x0, x1;
+          f2_split(x, x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
           const uint32_t b = (mh[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
           rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
           pt[c] = pk[c] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < HB / 2; ++c) {
+          const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
+          float x0, x1;
+          f2_split(x, x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+          pt[c] = 0u;
         }
       }
       // the previous block's P.V products must be done: O stable, P tiles free
@@ -523,7 +534,9 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         const int kc = gch >> 3, cc = gch & 7;
         const int off = kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(pPD + off) = v4;
-        if (tp_on)
+        // every row, so that no lane branches (rows without a temporal key are switched off
+        // in the temporal P.V anyway)
+        if (warp_tp)
           *reinterpret_cast<uint4*>(pPT + off) = make_uint4(pt[4 * ch], pt[4 * ch + 1], pt[4 * ch + 2], pt[4 * ch + 3]);
       }
       float rs0, rs1;
