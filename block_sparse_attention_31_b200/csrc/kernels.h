@@ -88,7 +88,7 @@ struct ProfilePlan {
   int r_pad;    // rounded up to the 128-row tile
   int tiles;    // r_pad / 128
   int splits;   // key-range splits per tile
-  size_t off_qs, off_ranges, off_opart, off_ml, off_rowerr, bytes;
+  size_t off_qs, off_ranges, off_order, off_opart, off_ml, off_rowerr, bytes;
 };
 ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac);
 // Same layout as profile_plan but with an explicit number of key-range splits (>= 1).

@@ -80,6 +80,8 @@ ProfilePlan profile_plan(const Geom& g, int BH, int d, double frac) {
   off = align256(off + static_cast<size_t>(BH) * p.r_pad * d * 2);
   p.off_ranges = off;
   off = align256(off + static_cast<size_t>(p.r_pad) * 4 * sizeof(int));
+  p.off_order = off;
+  off = align256(off + static_cast<size_t>(p.r_pad) * sizeof(int));
   p.off_opart = off;
   off = align256(off + static_cast<size_t>(BH) * splits * 3 * p.r_pad * d * sizeof(float));
   p.off_ml = off;
@@ -129,18 +131,39 @@ __device__ __forceinline__ void kept_block_range(int i, int N, int B, int G, int
   hi = l - 1;
 }
 
+// Order of the sampled rows inside each 128-row tile: ascending temporal slot (spatial
+// position, then frame), padding rows last.  Rows that share a warp then have nearby
+// temporal key ranges, so whole 32-key words of a block fall outside all of them and the
+// softmax skips their temporal masking.  One CTA of 128 threads per tile; order[slot] = row.
+__global__ void __launch_bounds__(kPM) profile_order_kernel(Geom g, int r, int32_t* __restrict__ order) {
+  __shared__ long long key_s[kPM];
+  const int p = threadIdx.x, i = blockIdx.x * kPM + p;
+  long long key = (1LL << 40) + i;
+  if (i < r) {
+    const long long t = (static_cast<long long>(2 * i + 1) * g.N) / (2LL * r);
+    key = static_cast<long long>(slot_of_token(g, kTemporal, static_cast<int>(t))) * kPM + p;
+  }
+  key_s[p] = key;
+  __syncthreads();
+  int rank = 0;
+  for (int q = 0; q < kPM; ++q) rank += key_s[q] < key ? 1 : 0;  // keys are distinct
+  order[blockIdx.x * kPM + rank] = i;
+}
+
+// Slot s of the sampled-row buffers holds row order[s] (profile_order_kernel).
 __global__ void __launch_bounds__(256) profile_prep_kernel(const __nv_bfloat16* __restrict__ q, Geom g, int d, int r,
-                                                           int r_pad, int w_s, int w_t,
+                                                           int r_pad, int w_s, int w_t, const int32_t* __restrict__ order,
                                                            __nv_bfloat16* __restrict__ qs, int4* __restrict__ ranges) {
   const int bh = blockIdx.y;
   const int vpr = d / 8;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const int i = idx / vpr, v = idx - (idx / vpr) * vpr;
-  if (i >= r_pad) return;
+  const int slot = idx / vpr, v = idx - (idx / vpr) * vpr;
+  if (slot >= r_pad) return;
+  const int i = order[slot];
   const long long t = i < r ? (static_cast<long long>(2 * i + 1) * g.N) / (2LL * r) : -1;
   uint4 val = make_uint4(0, 0, 0, 0);
   if (t >= 0) val = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<size_t>(bh) * g.N + t) * d + v * 8));
-  *reinterpret_cast<uint4*>(qs + (static_cast<size_t>(bh) * r_pad + i) * d + v * 8) = val;
+  *reinterpret_cast<uint4*>(qs + (static_cast<size_t>(bh) * r_pad + slot) * d + v * 8) = val;
   if (bh == 0 && v == 0) {
     int4 rg = make_int4(0, 0, 0, 0);
     if (t >= 0) {
@@ -153,7 +176,7 @@ __global__ void __launch_bounds__(256) profile_prep_kernel(const __nv_bfloat16* 
       rg.z = lo * g.block;
       rg.w = min(g.N, (hi + 1) * g.block);
     }
-    ranges[i] = rg;
+    ranges[slot] = rg;
   }
 }
 
@@ -476,29 +499,34 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       uint64_t rs2[2] = {0ull, 0ull};
       float rt4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[HB / 2], pt[HB / 2];  // packed P and its temporal-masked copy
-      if (warp_tp) {  // one branch per block, not per pair
 #pragma unroll
-        for (int c = 0; c < HB / 2; ++c) {
-          const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
-          float x0, x1;
-          f2_split(x, x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
-          const uint32_t b = (mh[(2 * c) >> 5] >> ((2 * c) & 31)) & 3u;
-          rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
-          pt[c] = pk[c] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
-        }
-      } else {
+      for (int w = 0; w < HB / 32; ++w) {
+        // one branch per 32-key word: the masking runs only where some row of the warp has
+        // a temporal key
+        if (__any_sync(0xffffffffu, mh[w] != 0u)) {
 #pragma unroll
-        for (int c = 0; c < HB / 2; ++c) {
-          const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
-          float x0, x1;
-          f2_split(x, x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
-          pt[c] = 0u;
+          for (int c = 16 * w; c < 16 * w + 16; ++c) {
+            const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
+            float x0, x1;
+            f2_split(x, x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+            const uint32_t b = (mh[w] >> ((2 * c) & 31)) & 3u;
+            rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
+            pt[c] = pk[c] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
+          }
+        } else {
+#pragma unroll
+          for (int c = 16 * w; c < 16 * w + 16; ++c) {
+            const uint64_t x = f2_fma(f2_make(s[2 * c], s[2 * c + 1]), sl2x2, negm2);
+            float x0, x1;
+            f2_split(x, x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+            pt[c] = 0u;
+          }
         }
       }
       // the previous block's P.V products must be done: O stable, P tiles free
@@ -789,14 +817,16 @@ cudaError_t launch_profile(const void* q, const void* k, const void* v, const Ge
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(w + plan.off_qs);
   int4* ranges = reinterpret_cast<int4*>(w + plan.off_ranges);
+  int32_t* order = reinterpret_cast<int32_t*>(w + plan.off_order);
   float* opart = reinterpret_cast<float*>(w + plan.off_opart);
   float* ml = reinterpret_cast<float*>(w + plan.off_ml);
   if (plan.splits < 1 || plan.splits > kMaxSplits) return cudaErrorInvalidValue;
   {
     const int vpr = d / 8;
+    profile_order_kernel<<<plan.tiles, kPM, 0, stream>>>(g, plan.r, order);
     dim3 grid((plan.r_pad * vpr + 255) / 256, BH);
     profile_prep_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), g, d, plan.r, plan.r_pad,
-                                                  w_s, w_t, qs, ranges);
+                                                  w_s, w_t, order, qs, ranges);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
