@@ -192,8 +192,7 @@ struct ProfCfg {
   static constexpr int OFF_PT = OFF_PD + P_BYTES;     // temporal-masked P
   static constexpr int OFF_BAR = OFF_PT + P_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
-  static constexpr int OFF_XMAX = OFF_MISC + 128;     // [2 halves][kPM] partial row maxima
-  static constexpr int BYTES = OFF_XMAX + 2 * kPM * 4;
+  static constexpr int BYTES = OFF_MISC + 128;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   // TMEM: S, then O of dense, spatial, temporal
   static constexpr int TMEM_S = 0, TMEM_O = BN;
@@ -203,7 +202,7 @@ struct ProfCfg {
 };
 
 enum { PB_Q = 0, PB_FULL_K = 1, PB_FULL_V = 3, PB_EMPTY_K = 5, PB_EMPTY_V = 7, PB_S_FULL = 9, PB_S_FREE = 10,
-       PB_P_FULL = 11, PB_O_DONE = 12, PB_DRAIN = 13, PB_X_FULL = 14 };
+       PB_P_FULL = 11, PB_O_DONE = 12, PB_DRAIN = 13 };
 
 struct ProfArgs {
   const int4* ranges;
@@ -248,7 +247,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
   const uint32_t sPD = sbase + C::OFF_PD, sPT = sbase + C::OFF_PT;
   uint8_t* pPD = smem + C::OFF_PD;
   uint8_t* pPT = smem + C::OFF_PT;
-  volatile float* xmax = reinterpret_cast<volatile float*>(smem + C::OFF_XMAX);
   auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
   volatile int* misc = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   volatile int* abort_flag = misc + 1;
@@ -280,7 +278,6 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     mbar_init(bar(PB_P_FULL), 256);
     mbar_init(bar(PB_O_DONE), 1);
     mbar_init(bar(PB_DRAIN), 1);
-    mbar_init(bar(PB_X_FULL), 256);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -403,10 +400,10 @@ __global__ void __launch_bounds__(kProfThreads, 1)
     __syncwarp();
   } else {
     // Two softmax warpgroups split every S row by columns: warp w (2..9) serves the TMEM lane
-    // quarter w % 4 and the column half h = (w - 2) / 4.  The two threads of a row exchange
-    // their halves' maxima through shared memory (so they take the same rescale decisions),
-    // exponentiate their own half, write their half of each P tile and keep partial sums,
-    // which are added at the end (half 0 + half 1).
+    // quarter w % 4 and the column half h = (w - 2) / 4.  Both threads of a row read the whole
+    // row for its maximum (so they take the same rescale decisions without exchanging
+    // anything), exponentiate their own half, write their half of each P tile and keep partial
+    // sums, which are added at the end (half 0 + half 1).
     constexpr int HB = BN / 2;
     const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
@@ -433,36 +430,45 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_S_FULL), j & 1, abort_flag, a.err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t rs_own[HB];
+      // both halves of the row: this thread's own, and the other one for the row maximum only
+      // (reading it costs less than exchanging partial maxima between the warps)
+      uint32_t rs_own[HB], rs_oth[HB];
 #pragma unroll
-      for (int c = 0; c < HB / 32; ++c) tmem_ld32_async(t_s + c_own + c * 32, rs_own + c * 32);
+      for (int c = 0; c < HB / 32; ++c) {
+        tmem_ld32_async(t_s + c_own + c * 32, rs_own + c * 32);
+        tmem_ld32_async(t_s + (HB - c_own) + c * 32, rs_oth + c * 32);
+      }
       tmem_wait_ld();
       reg_fence<HB>(rs_own);
+      reg_fence<HB>(rs_oth);
+      tc_fence_before();
+      mbar_arrive(bar(PB_S_FREE));  // S may be overwritten by the next block's Q.K^T
       const int t0 = (kb0 + j) * BN;
       const int nvalid = min(BN, g.N - t0);
-      float s[HB];
+      float s[HB], so[HB];
 #pragma unroll
-      for (int c = 0; c < HB; ++c) s[c] = __uint_as_float(rs_own[c]);
+      for (int c = 0; c < HB; ++c) {
+        s[c] = __uint_as_float(rs_own[c]);
+        so[c] = __uint_as_float(rs_oth[c]);
+      }
       if (nvalid < BN) {  // the ragged last block
 #pragma unroll
-        for (int c = 0; c < HB; ++c)
+        for (int c = 0; c < HB; ++c) {
           if (c_own + c >= nvalid) s[c] = -INFINITY;
+          if (HB - c_own + c >= nvalid) so[c] = -INFINITY;
+        }
       }
       float mx8[8];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) mx8[x] = fmax3(s[2 * x], s[2 * x + 1], -INFINITY);
+      for (int x = 0; x < 8; ++x) mx8[x] = fmax3(s[2 * x], s[2 * x + 1], so[2 * x]);
 #pragma unroll
-      for (int c = 16; c < HB; c += 2) mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
-      // the row maximum: exchange the two halves' partial maxima (every thread has read the
-      // other half's value before it releases S, so the next block's writes come after it)
-      xmax[half * kPM + row] = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                     fmaxf(mx8[6], mx8[7]));
-      mbar_arrive(bar(PB_X_FULL));
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(PB_X_FULL), j & 1, abort_flag, a.err));
-      if (!ok) break;
-      const float mx = fmaxf(xmax[row], xmax[kPM + row]);
-      tc_fence_before();
-      mbar_arrive(bar(PB_S_FREE));  // S may be overwritten by the next block's Q.K^T
+      for (int x = 0; x < 8; ++x) mx8[x] = fmax3(mx8[x], so[2 * x + 1], -INFINITY);
+#pragma unroll
+      for (int c = 16; c < HB; c += 2) {
+        mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
+        mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], so[c], so[c + 1]);
+      }
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m, mx * sl2);
       const bool grow = m_new > m + kRescaleLog2;
       // masks: spatial whole block; temporal as contiguous column ranges per frame segment
