@@ -474,28 +474,27 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       // masks: spatial whole block; temporal as contiguous column ranges per frame segment
       // (the whole row, so both halves know whether the row uses the temporal P tile)
       const bool sp_on = t0 >= rg.x && t0 < rg.y;
-      uint32_t mt[BN / 32];
+      // this half's temporal mask words (bit c = own column c); tp_on: the row has a temporal
+      // key anywhere in the block (both halves compute it the same way)
+      uint32_t mh[HB / 32];
 #pragma unroll
-      for (int w = 0; w < BN / 32; ++w) mt[w] = 0u;
+      for (int w = 0; w < HB / 32; ++w) mh[w] = 0u;
+      bool tp_on = false;
       if (t_any) {
         int f = t0 / g.S, s0 = t0 - (t0 / g.S) * g.S;
         for (int c = 0; c < nvalid;) {
           const int seg = min(nvalid - c, g.S - s0);
           const int lo_s = ts_lo + (f < tf_lo ? 1 : 0), hi_s = ts_hi - (f > tf_hi ? 1 : 0);
           const int x0 = max(lo_s, s0), x1 = min(hi_s, s0 + seg - 1);
-          if (x0 <= x1) set_bit_range<BN>(mt, c + x0 - s0, c + x1 - s0);
+          if (x0 <= x1) {
+            tp_on = true;
+            set_bit_range<HB>(mh, c + x0 - s0 - c_own, c + x1 - s0 - c_own);
+          }
           c += seg;
           ++f;
           s0 = 0;
         }
       }
-      uint32_t tany = 0u;
-#pragma unroll
-      for (int w = 0; w < BN / 32; ++w) tany |= mt[w];
-      const bool tp_on = tany != 0u;
-      uint32_t mh[HB / 32];  // this half's mask words (static indexing below)
-#pragma unroll
-      for (int w = 0; w < HB / 32; ++w) mh[w] = half ? mt[HB / 32 + w] : mt[w];
       // Exponentials of this half first, into registers (packed bf16 pairs): this overlaps the
       // previous block's P.V products, which still read the P tiles.
       const float m_next = grow ? m_new : m;
