@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kProfThreads, 1)
       const bool warp_tp = __any_sync(0xffffffffu, tp_on);
       const uint64_t sl2x2 = f2_make(sl2, sl2), negm2 = f2_make(-m_use, -m_use);
       uint64_t rs2[2] = {0ull, 0ull};
-      float rt4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t rt2[2] = {0ull, 0ull};
       uint32_t pk[HB / 2], pt[HB / 2];  // packed P and its temporal-masked copy
 #pragma unroll
       for (int w = 0; w < HB / 32; ++w) {
@@ -518,8 +518,9 @@ __global__ void __launch_bounds__(kProfThreads, 1)
             rs2[c & 1] = f2_add(rs2[c & 1], f2_make(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
             const uint32_t b = (mh[w] >> ((2 * c) & 31)) & 3u;
-            rt4[c & 3] += ((b & 1u) ? p0 : 0.f) + ((b & 2u) ? p1 : 0.f);
-            pt[c] = pk[c] & (((b & 1u) ? 0x0000ffffu : 0u) | ((b & 2u) ? 0xffff0000u : 0u));
+            const float q0 = (b & 1u) ? p0 : 0.f, q1 = (b & 2u) ? p1 : 0.f;  // temporal-masked pair
+            rt2[c & 1] = f2_add(rt2[c & 1], f2_make(q0, q1));
+            pt[c] = pack_bf16x2(q0, q1);
           }
         } else {
 #pragma unroll
@@ -560,22 +561,29 @@ __global__ void __launch_bounds__(kProfThreads, 1)
         l[2] *= alpha;
         m = m_new;
       }
+      // 8 probabilities -> one 16-byte chunk of each P tile; the temporal tile is written for
+      // every row of a warp with some temporal key (rows without one are switched off in the
+      // temporal P.V)
 #pragma unroll
-      for (int ch = 0; ch < HB / 8; ++ch) {  // 8 probabilities -> one 16-byte chunk of each P tile
+      for (int ch = 0; ch < HB / 8; ++ch) {
         const int gch = half * (HB / 8) + ch;
-        const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        const int kc = gch >> 3, cc = gch & 7;
-        const int off = kc * (kPM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(pPD + off) = v4;
-        // every row, so that no lane branches (rows without a temporal key are switched off
-        // in the temporal P.V anyway)
-        if (warp_tp)
+        const int off = (gch >> 3) * (kPM * 128) + row * 128 + (((gch & 7) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(pPD + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      }
+      if (warp_tp) {
+#pragma unroll
+        for (int ch = 0; ch < HB / 8; ++ch) {
+          const int gch = half * (HB / 8) + ch;
+          const int off = (gch >> 3) * (kPM * 128) + row * 128 + (((gch & 7) ^ (row & 7)) << 4);
           *reinterpret_cast<uint4*>(pPT + off) = make_uint4(pt[4 * ch], pt[4 * ch + 1], pt[4 * ch + 2], pt[4 * ch + 3]);
+        }
       }
       float rs0, rs1;
       f2_split(f2_add(rs2[0], rs2[1]), rs0, rs1);
       const float rs = rs0 + rs1;
-      const float rt = (rt4[0] + rt4[1]) + (rt4[2] + rt4[3]);
+      float rt0, rt1;
+      f2_split(f2_add(rt2[0], rt2[1]), rt0, rt1);
+      const float rt = rt0 + rt1;
       l[0] += rs;
       if (sp_on) l[1] += rs;
       l[2] += rt;
