@@ -129,9 +129,11 @@ def stage_work(wl, kinds, pipe, pairs):
         nwords = -(-pipe.nblk // 32)
         cq, ck = wl.clusters
         out = {
-            # k-means: per round one fp32 dot product per (row, centroid) pair (2*d flops) for
-            # Q and K; the update, order and the rest are lower-order
-            "profile": {"flops": BH * wl.kmeans_iters * 2.0 * d * N * (cq + ck), "bound": "fp32"},
+            # k-means: per round one dot product per (row, centroid) pair (2*d flops) for Q and
+            # K, on the tensor cores as two bf16 halves of each centroid (executed twice that);
+            # the update, order and the rest are lower-order
+            "profile": {"flops": BH * wl.kmeans_iters * 2.0 * d * N * (cq + ck), "bound": "tensor",
+                        "executed_flops": BH * wl.kmeans_iters * 4.0 * d * N * (cq + ck)},
             "permute": {"bytes": BH * 3.0 * 2 * N * row, "bound": "hbm"},
             "mask": {"bytes": BH * pipe.nblk * (nwords + pipe.max_kv + 1) * 4.0, "bound": "hbm"},
             "unpermute": {"bytes": BH * 2.0 * N * row, "bound": "hbm"},
@@ -174,12 +176,7 @@ def stage_roofline(work, stage_ms, hbm_gbs, tensor_tflops):
         t = stage_ms[name] / 1e3
         if t <= 0 or w.get("bytes", 1) == 0:
             continue
-        if w["bound"] == "fp32":
-            # no measured fp32 FMA peak exists for this machine, so no fraction is reported
-            tf = w["flops"] / t / 1e12
-            out[name] = {"bound": "alu", "flops": w["flops"], "achieved": tf, "peak": None, "unit": "TFLOP/s",
-                         "frac": None}
-        elif w["bound"] == "hbm":
+        if w["bound"] == "hbm":
             gbs = w["bytes"] / t / 1e9
             out[name] = {"bound": "hbm", "bytes": w["bytes"], "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": gbs / hbm_gbs}

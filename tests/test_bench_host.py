@@ -88,8 +88,11 @@ def test_semantic_stage_work():
     assert exp2 == 1000 * 128 * 128
     roof = bench.stage_roofline(work, {"profile": 4.0, "permute": 0.1, "mask": 0.2, "unpermute": 0.05}, 6538.3,
                                 1631.1)
-    # no measured fp32 peak exists, so the k-means stage reports its rate without a fraction
-    assert roof["profile"]["bound"] == "alu" and roof["profile"]["peak"] is None and roof["profile"]["frac"] is None
+    # the k-means distances run on the tensor cores: algorithmic and executed (two bf16 halves)
+    # rates against the bf16 peak
+    assert roof["profile"]["bound"] == "tensor" and roof["profile"]["peak"] == 1631.1
+    assert abs(roof["profile"]["frac"] - work["profile"]["flops"] / 4e-3 / 1e12 / 1631.1) < 1e-12
+    assert work["profile"]["executed_flops"] == 2 * work["profile"]["flops"]
     assert abs(roof["permute"]["achieved"] - work["permute"]["bytes"] / 1e-4 / 1e9) < 1e-6
 
 
