@@ -544,7 +544,7 @@ static bool clusters_ok(const Geom& g, int C) { return C >= 1 && C <= kMaxCluste
 size_t vsa_kmeans_workspace_size(const vsa_shape* shape, int n_clusters) {
   Geom g;
   if (semantic_geom(shape, &g) != VSA_OK || !clusters_ok(g, n_clusters)) return 0;
-  return kmeans_workspace_bytes(shape->B * shape->H, n_clusters, shape->d);
+  return kmeans_workspace_bytes(shape->B * shape->H, g.N, n_clusters, shape->d);
 }
 
 vsa_status vsa_kmeans(const void* x, const vsa_shape* shape, int n_clusters, int iters, float* d_centroids,
@@ -651,7 +651,7 @@ static vsa_status semantic_layout(const vsa_shape* shape, const vsa_semantic_par
   L->lab_k = take(BH * N * 4);
   L->cnt_k = take(BH * sp->ck * 4);
   L->perm_k = take(BH * N * 4);
-  L->offs = take(kmeans_workspace_bytes(static_cast<int>(BH), std::max(sp->cq, sp->ck), static_cast<int>(d)));
+  L->offs = take(kmeans_workspace_bytes(static_cast<int>(BH), g.N, std::max(sp->cq, sp->ck), static_cast<int>(d)));
   L->keep = take(BH * sp->cq * kwords * 4);
   L->bits = take(BH * nb * bwords * 4);
   L->idx = take(BH * nb * nb * 4);

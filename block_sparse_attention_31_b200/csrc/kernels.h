@@ -29,9 +29,10 @@ cudaError_t launch_block_order(const uint8_t* kinds, const Geom& g, int BH, cons
 // Semantic-aware permutation (see semantic.cu).  At most kMaxClusters clusters per tensor.
 constexpr int kMaxClusters = 1024;
 // k-means of x [BH, N, d] bf16: cent [BH, C, d] f32, label [BH, N], counts [BH, C], perm [BH, N]
-// (slot -> token, cluster-major).  ws (kmeans_workspace_bytes): the cluster offsets
-// [BH, C + 1], the centroids' squared norms [BH, C] and their bf16 halves [BH, C, d] twice.
-size_t kmeans_workspace_bytes(int BH, int C, int d);
+// (slot -> token, cluster-major).  ws (kmeans_workspace_bytes): the cluster offsets and
+// partial-sum chunk offsets [BH, C + 1], the centroids' squared norms [BH, C], their bf16
+// halves [BH, C, d] twice, and the update's chunk sums [BH, ceil(N / 128) + C, d].
+size_t kmeans_workspace_bytes(int BH, int N, int C, int d);
 cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
                           int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream);
 // Workspace of launch_semantic_mask: the cluster range of every query and key block.

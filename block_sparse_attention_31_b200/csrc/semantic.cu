@@ -204,10 +204,12 @@ __global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_cons
 // __match_any_sync).  Shared memory: (kSortWarps + 1) * C ints.
 constexpr int kSortWarps = 16;
 constexpr int kSortPrefetch = 8;  // 32-token steps whose labels are loaded ahead
+constexpr int kUpdChunk = 128;    // member rows per partial-sum CTA of the update
 
 __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int32_t* __restrict__ label, int N, int C,
                                                                       int32_t* __restrict__ counts,
                                                                       int32_t* __restrict__ offsets,
+                                                                      int32_t* __restrict__ chunk_off,
                                                                       int32_t* __restrict__ perm, int* err) {
   extern __shared__ int sort_smem[];
   int* hist = sort_smem;              // [kSortWarps][C]: counts, then first free slot, per segment
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int3
       counts[static_cast<size_t>(bh) * C + j] = 0;
       offsets[static_cast<size_t>(bh) * (C + 1) + j] = 0;
     }
+    for (int j = tid; j <= C; j += kSortWarps * 32) chunk_off[static_cast<size_t>(bh) * (C + 1) + j] = 0;
     return;
   }
   for (int j = tid; j < C; j += kSortWarps * 32) {
@@ -241,25 +244,36 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int3
     counts[static_cast<size_t>(bh) * C + j] = sum;
   }
   __syncthreads();
-  // exclusive scan of tot over the clusters (warp 0, 32 clusters per step)
+  // exclusive scans over the clusters (warp 0, 32 clusters per step): of tot (the offsets) and
+  // of each cluster's number of kUpdChunk-row chunks (the update's partial sums)
   if (warp == 0) {
-    int carry = 0;
+    int carry = 0, ccarry = 0;
     for (int j0 = 0; j0 < C; j0 += 32) {
       const int j = j0 + lane;
       const int v = j < C ? tot[j] : 0;
-      int incl = v;
+      const int cv = (v + kUpdChunk - 1) / kUpdChunk;
+      int incl = v, cincl = cv;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
+        const int co = __shfl_up_sync(0xffffffffu, cincl, off);
+        if (lane >= off) {
+          incl += o;
+          cincl += co;
+        }
       }
       if (j < C) {
         tot[j] = carry + incl - v;
         offsets[static_cast<size_t>(bh) * (C + 1) + j] = carry + incl - v;
+        chunk_off[static_cast<size_t>(bh) * (C + 1) + j] = ccarry + cincl - cv;
       }
       carry += __shfl_sync(0xffffffffu, incl, 31);
+      ccarry += __shfl_sync(0xffffffffu, cincl, 31);
     }
-    if (lane == 0) offsets[static_cast<size_t>(bh) * (C + 1) + C] = carry;
+    if (lane == 0) {
+      offsets[static_cast<size_t>(bh) * (C + 1) + C] = carry;
+      chunk_off[static_cast<size_t>(bh) * (C + 1) + C] = ccarry;
+    }
   }
   __syncthreads();
   for (int j = tid; j < C; j += kSortWarps * 32) {
@@ -298,81 +312,165 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int3
   }
 }
 
-// New centroids: one CTA per (cluster, head).  The members' rows stream through shared memory
-// kUpdRows at a time (double-buffered; every thread loads 16-byte pieces of the next stage
-// while the current one is summed); thread x < D adds dimension x of the staged rows in token
-// order, in fp64.
-constexpr int kUpdThreads = 256;
-constexpr int kUpdRows = 128;
+// New centroids.  The reading is the members' fp64 sum in token order, divided by the count.
+// That sum is computed in parallel and still exactly: every member value is a bf16 number, so
+// all of a cluster's values in one dimension are integer multiples of 2^q, q the smallest
+// unit in the last place among them (ulp(v) = 2^(E - 7) for a normal bf16 value of exponent
+// E, 2^-133 for a subnormal one).  Every partial sum, in any order, is then a multiple of 2^q
+// of magnitude at most A = sum |v|, and fp64 holds every such number exactly while
+// A < 2^(q + 53).  Under that condition the ordered sum and any grouping of it are the same
+// exact number.  kmeans_partial_kernel sums chunks of kUpdChunk members (and their |v| and
+// q); kmeans_combine_kernel adds a cluster's chunks, checks the condition, and where it fails
+// (values spread over more than 53 binades, an infinity or a NaN) adds the members again one
+// by one in token order.  A sum of non-negative fp64 numbers reaches 2^(q+53) in floating
+// point exactly when it does in exact arithmetic, so the check itself is exact.
+constexpr int kNoUlp = 1000;  // q of a dimension with no nonzero member
 
-template <int D>
-constexpr size_t update_smem_bytes() {
-  return 2 * static_cast<size_t>(kUpdRows) * D * sizeof(__nv_bfloat16);
+// ulp exponent of a nonzero bf16 value from its bits (kNoUlp for +-0)
+__device__ __forceinline__ int bf16_ulp_exp(uint32_t bits) {
+  const int be = static_cast<int>((bits >> 7) & 0xffu);
+  if ((bits & 0x7fffu) == 0u) return kNoUlp;
+  return be == 0 ? -133 : be - 134;
 }
 
+// One CTA of kPartThreads per chunk k of a head's chunk list (the chunk's cluster is the last j
+// with chunk_off[j] <= k; empty clusters own no chunk).  The chunk's member indices go to
+// shared memory first; thread (row lane rl, dimension group g) then loads 16-byte pieces (8
+// dimensions) of rows rl, rl + RL, ... all independently, and the row lanes' partial sums
+// are added through shared memory (any order: see above).
+constexpr int kPartThreads = 128;
+
 template <int D>
-__global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
-                                                                    const int32_t* __restrict__ counts,
-                                                                    const int32_t* __restrict__ offsets,
-                                                                    const int32_t* __restrict__ perm,
-                                                                    float* __restrict__ cent,
-                                                                    float* __restrict__ cnorm,
-                                                                    __nv_bfloat16* __restrict__ chi,
-                                                                    __nv_bfloat16* __restrict__ clo) {
-  extern __shared__ __align__(16) uint4 upd_smem[];
-  constexpr int VPR = D * 2 / 16;                        // 16-byte pieces per row
-  constexpr int PER_T = kUpdRows * VPR / kUpdThreads;    // pieces per thread per stage
+__global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv_bfloat16* __restrict__ x, int N,
+                                                                      int C, const int32_t* __restrict__ offsets,
+                                                                      const int32_t* __restrict__ chunk_off,
+                                                                      const int32_t* __restrict__ perm, int max_chunks,
+                                                                      double* __restrict__ psum,
+                                                                      double* __restrict__ pabs,
+                                                                      int32_t* __restrict__ pq) {
+  constexpr int G = D / 8;               // dimension groups of 8
+  constexpr int RL = kPartThreads / G;   // row lanes
+  constexpr int PER = kUpdChunk / RL;    // rows per thread
+  __shared__ int rows_s[kUpdChunk];
+  __shared__ double red_s[RL][D];
+  __shared__ double reda_s[RL][D];
+  __shared__ int redq_s[RL][D];
+  const int k = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int32_t* co = chunk_off + static_cast<size_t>(bh) * (C + 1);
+  if (k >= co[C]) return;
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (co[mid] <= k) lo = mid;
+    else hi = mid - 1;
+  }
+  const int j = lo;
+  const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
+  const int first = (k - co[j]) * kUpdChunk;
+  const int cnt = min(kUpdChunk, off[j + 1] - off[j] - first);
+  const int32_t* ph = perm + static_cast<size_t>(bh) * N + off[j] + first;
+  for (int r = tid; r < kUpdChunk; r += kPartThreads) {
+    const int t = r < cnt ? ph[r] : -1;
+    rows_s[r] = (t >= 0 && t < N) ? t : -1;
+  }
+  __syncthreads();
+  const int g = tid % G, rl = tid / G;
+  const uint4* xh = reinterpret_cast<const uint4*>(x + static_cast<size_t>(bh) * N * D);
+  double sa[8], aa[8];
+  int qa[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    sa[e] = 0.0;
+    aa[e] = 0.0;
+    qa[e] = kNoUlp;
+  }
+  constexpr int BATCH = PER < 8 ? PER : 8;  // rows loaded before any is added
+#pragma unroll
+  for (int i0 = 0; i0 < PER; i0 += BATCH) {
+    uint4 w[BATCH];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int t = rows_s[rl + (i0 + i) * RL];
+      w[i] = t >= 0 ? __ldg(xh + static_cast<size_t>(t) * G + g) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t word = e < 2 ? w[i].x : e < 4 ? w[i].y : e < 6 ? w[i].z : w[i].w;
+        const uint32_t bits = (e & 1) ? (word >> 16) : (word & 0xffffu);
+        const double v = static_cast<double>(__uint_as_float(bits << 16));
+        sa[e] += v;
+        aa[e] += fabs(v);
+        qa[e] = min(qa[e], bf16_ulp_exp(bits));
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red_s[rl][g * 8 + e] = sa[e];
+    reda_s[rl][g * 8 + e] = aa[e];
+    redq_s[rl][g * 8 + e] = qa[e];
+  }
+  __syncthreads();
+  for (int dd = tid; dd < D; dd += kPartThreads) {
+    double s = 0.0, a = 0.0;
+    int q = kNoUlp;
+    for (int l = 0; l < RL; ++l) {
+      s += red_s[l][dd];
+      a += reda_s[l][dd];
+      q = min(q, redq_s[l][dd]);
+    }
+    const size_t o = (static_cast<size_t>(bh) * max_chunks + k) * D + dd;
+    psum[o] = s;
+    pabs[o] = a;
+    pq[o] = q;
+  }
+}
+
+// One CTA (d threads) per (cluster, head): the cluster's chunk sums in order, the exactness
+// check, the fallback, then the centroid as fp32(sum / n), its bf16 halves and its norm.  An
+// empty cluster keeps its centroid.
+template <int D>
+__global__ void __launch_bounds__(D) kmeans_combine_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                           const int32_t* __restrict__ counts,
+                                                           const int32_t* __restrict__ offsets,
+                                                           const int32_t* __restrict__ chunk_off,
+                                                           const int32_t* __restrict__ perm, int max_chunks,
+                                                           const double* __restrict__ psum,
+                                                           const double* __restrict__ pabs,
+                                                           const int32_t* __restrict__ pq, float* __restrict__ cent,
+                                                           float* __restrict__ cnorm, __nv_bfloat16* __restrict__ chi,
+                                                           __nv_bfloat16* __restrict__ clo) {
+  __shared__ float cnew[D];
   const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int n = counts[static_cast<size_t>(bh) * C + j];
-  if (n <= 0) return;  // an empty cluster keeps its centroid
-  const int off = offsets[static_cast<size_t>(bh) * (C + 1) + j];
-  const int32_t* ph = perm + static_cast<size_t>(bh) * N + off;
-  const uint4* xh = reinterpret_cast<const uint4*>(x + static_cast<size_t>(bh) * N * D);
-  uint4 reg[PER_T];
-  auto load = [&](int m0) {
-#pragma unroll
-    for (int q = 0; q < PER_T; ++q) {
-      const int e = tid + q * kUpdThreads, r = e / VPR, v = e - r * VPR;
-      const int m = m0 + r;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (m < n) {
-        const int t = ph[m];
-        if (t >= 0 && t < N) val = xh[static_cast<size_t>(t) * VPR + v];
-      }
-      reg[q] = val;
-    }
-  };
-  auto store = [&](int buf) {
-#pragma unroll
-    for (int q = 0; q < PER_T; ++q) upd_smem[buf * kUpdRows * VPR + tid + q * kUpdThreads] = reg[q];
-  };
-  load(0);
-  store(0);
-  __syncthreads();
-  double s = 0.0;
-  int buf = 0;
-  for (int m0 = 0; m0 < n; m0 += kUpdRows) {
-    const bool more = m0 + kUpdRows < n;
-    if (more) load(m0 + kUpdRows);
-    if (tid < D) {
-      const __nv_bfloat16* rows = reinterpret_cast<const __nv_bfloat16*>(upd_smem + buf * kUpdRows * VPR);
-      const int cnt = min(kUpdRows, n - m0);
-      for (int r = 0; r < cnt; ++r) s = __dadd_rn(s, static_cast<double>(__bfloat162float(rows[r * D + tid])));
-    }
-    if (more) store(buf ^ 1);
-    __syncthreads();
-    buf ^= 1;
+  if (n <= 0) return;
+  const int32_t* co = chunk_off + static_cast<size_t>(bh) * (C + 1);
+  double sum = 0.0, abs_sum = 0.0;
+  int q = kNoUlp;
+  for (int k = co[j]; k < co[j + 1]; ++k) {
+    const size_t o = (static_cast<size_t>(bh) * max_chunks + k) * D + tid;
+    sum = __dadd_rn(sum, psum[o]);
+    abs_sum = __dadd_rn(abs_sum, pabs[o]);
+    q = min(q, pq[o]);
   }
-  float* cnew = reinterpret_cast<float*>(upd_smem);  // the staged rows are no longer read
-  if (tid < D) {
-    const float c = __double2float_rn(__ddiv_rn(s, static_cast<double>(n)));
-    const size_t o = (static_cast<size_t>(bh) * C + j) * D + tid;
-    cent[o] = c;
-    cnew[tid] = c;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(c);
-    chi[o] = hi;
-    clo[o] = __float2bfloat16_rn(__fsub_rn(c, __bfloat162float(hi)));
+  if (!(abs_sum < ldexp(1.0, q + 53))) {  // not provably exact: the ordered sum itself
+    const int32_t* ph = perm + static_cast<size_t>(bh) * N + offsets[static_cast<size_t>(bh) * (C + 1) + j];
+    const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * N * D;
+    sum = 0.0;
+    for (int m = 0; m < n; ++m) {
+      const int t = ph[m];
+      if (t >= 0 && t < N) sum = __dadd_rn(sum, static_cast<double>(__bfloat162float(xh[static_cast<size_t>(t) * D + tid])));
+    }
   }
+  const float c = __double2float_rn(__ddiv_rn(sum, static_cast<double>(n)));
+  const size_t o = (static_cast<size_t>(bh) * C + j) * D + tid;
+  cent[o] = c;
+  cnew[tid] = c;
+  const __nv_bfloat16 h = __float2bfloat16_rn(c);
+  chi[o] = h;
+  clo[o] = __float2bfloat16_rn(__fsub_rn(c, __bfloat162float(h)));
   __syncthreads();
   if (tid == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(cnew, D);
 }
@@ -596,10 +694,46 @@ int rows_grid_x(int N, int vpr, int BH) {
   return static_cast<int>(want < cap ? want : cap);
 }
 
+// k-means scratch, carved from the caller's workspace (256-byte aligned pieces).
+struct KmWork {
+  int32_t* offsets;    // [BH, C + 1] cluster offsets in the cluster-major order
+  int32_t* chunk_off;  // [BH, C + 1] first partial-sum chunk of every cluster
+  float* cnorm;        // [BH, C] squared centroid norms
+  __nv_bfloat16* chi;  // [BH, C, d] bf16 high halves of the centroids
+  __nv_bfloat16* clo;  // [BH, C, d] bf16 low halves
+  double* psum;        // [BH, max_chunks, d] chunk sums
+  double* pabs;        // [BH, max_chunks, d] chunk sums of |v|
+  int32_t* pq;         // [BH, max_chunks, d] chunk ulp exponents
+  int max_chunks;      // ceil(N / kUpdChunk) + C bounds a head's chunk count
+  size_t bytes;
+};
+
+KmWork kmeans_layout(void* ws, int BH, int N, int C, int d) {
+  KmWork w{};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~static_cast<size_t>(255);
+    return p;
+  };
+  const size_t bh = static_cast<size_t>(BH);
+  w.max_chunks = (N + kUpdChunk - 1) / kUpdChunk + C;
+  w.offsets = static_cast<int32_t*>(take(bh * (C + 1) * sizeof(int32_t)));
+  w.chunk_off = static_cast<int32_t*>(take(bh * (C + 1) * sizeof(int32_t)));
+  w.cnorm = static_cast<float*>(take(bh * C * sizeof(float)));
+  w.chi = static_cast<__nv_bfloat16*>(take(bh * C * d * sizeof(__nv_bfloat16)));
+  w.clo = static_cast<__nv_bfloat16*>(take(bh * C * d * sizeof(__nv_bfloat16)));
+  w.psum = static_cast<double*>(take(bh * w.max_chunks * d * sizeof(double)));
+  w.pabs = static_cast<double*>(take(bh * w.max_chunks * d * sizeof(double)));
+  w.pq = static_cast<int32_t*>(take(bh * w.max_chunks * d * sizeof(int32_t)));
+  w.bytes = off;
+  return w;
+}
+
 template <int D>
 cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, float* cent, int32_t* label,
-                     int32_t* counts, int32_t* perm, int32_t* offsets, float* cnorm, __nv_bfloat16* chi,
-                     __nv_bfloat16* clo, int* err, cudaStream_t stream) {
+                     int32_t* counts, int32_t* perm, const KmWork& w, int* err, cudaStream_t stream) {
   using K = KmTcCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
@@ -610,51 +744,35 @@ cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, fl
   }
   CUtensorMap tx, thi, tlo;
   if ((e = encode_rows_map(&tx, x, D, N, BH, kTcRows)) != cudaSuccess) return e;
-  if ((e = encode_rows_map(&thi, chi, D, C, BH, kTcRows)) != cudaSuccess) return e;
-  if ((e = encode_rows_map(&tlo, clo, D, C, BH, kTcRows)) != cudaSuccess) return e;
-  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, cnorm, chi, clo);
-  constexpr size_t usmem = update_smem_bytes<D>();
-  e = cudaFuncSetAttribute(kmeans_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(usmem));
-  if (e != cudaSuccess) return e;
-  const dim3 agrid((N + kTcRows - 1) / kTcRows, BH), ugrid(C, BH);
+  if ((e = encode_rows_map(&thi, w.chi, D, C, BH, kTcRows)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(&tlo, w.clo, D, C, BH, kTcRows)) != cudaSuccess) return e;
+  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, w.cnorm, w.chi, w.clo);
+  const dim3 agrid((N + kTcRows - 1) / kTcRows, BH), pgrid(w.max_chunks, BH), cgrid(C, BH);
   for (int it = 0; it < iters; ++it) {
-    kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, cnorm, label, err);
-    kmeans_sort_kernel<<<BH, kSortWarps * 32, ssmem, stream>>>(label, N, C, counts, offsets, perm, err);
-    kmeans_update_kernel<D><<<ugrid, kUpdThreads, usmem, stream>>>(x, N, C, counts, offsets, perm, cent, cnorm, chi,
-                                                                   clo);
+    kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
+    kmeans_sort_kernel<<<BH, kSortWarps * 32, ssmem, stream>>>(label, N, C, counts, w.offsets, w.chunk_off, perm,
+                                                                err);
+    kmeans_partial_kernel<D><<<pgrid, kPartThreads, 0, stream>>>(x, N, C, w.offsets, w.chunk_off, perm, w.max_chunks,
+                                                                 w.psum, w.pabs, w.pq);
+    kmeans_combine_kernel<D><<<cgrid, D, 0, stream>>>(x, N, C, counts, w.offsets, w.chunk_off, perm, w.max_chunks,
+                                                      w.psum, w.pabs, w.pq, cent, w.cnorm, w.chi, w.clo);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-namespace {
-constexpr size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-}  // namespace
-
-size_t kmeans_workspace_bytes(int BH, int C, int d) {
-  const size_t offs = round256(static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t));
-  const size_t norms = round256(static_cast<size_t>(BH) * C * sizeof(float));
-  const size_t half = round256(static_cast<size_t>(BH) * C * d * sizeof(__nv_bfloat16));
-  return offs + norms + 2 * half;
+size_t kmeans_workspace_bytes(int BH, int N, int C, int d) {
+  KmWork w = kmeans_layout(nullptr, BH, N, C, d);
+  return w.bytes;
 }
 
 cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
                           int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream) {
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  const size_t offs = round256(static_cast<size_t>(BH) * (C + 1) * sizeof(int32_t));
-  const size_t norms = round256(static_cast<size_t>(BH) * C * sizeof(float));
-  const size_t half = round256(static_cast<size_t>(BH) * C * d * sizeof(__nv_bfloat16));
-  int32_t* offsets = reinterpret_cast<int32_t*>(w);
-  float* cnorm = reinterpret_cast<float*>(w + offs);
-  __nv_bfloat16* chi = reinterpret_cast<__nv_bfloat16*>(w + offs + norms);
-  __nv_bfloat16* clo = reinterpret_cast<__nv_bfloat16*>(w + offs + norms + half);
-  if (d == 128)
-    return kmeans_d<128>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, chi, clo, err, stream);
-  if (d == 64)
-    return kmeans_d<64>(xb, BH, N, C, iters, cent, label, counts, perm, offsets, cnorm, chi, clo, err, stream);
+  const KmWork w = kmeans_layout(ws, BH, N, C, d);
+  if (d == 128) return kmeans_d<128>(xb, BH, N, C, iters, cent, label, counts, perm, w, err, stream);
+  if (d == 64) return kmeans_d<64>(xb, BH, N, C, iters, cent, label, counts, perm, w, err, stream);
   return cudaErrorInvalidValue;
 }
 

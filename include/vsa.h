@@ -399,9 +399,10 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
  * rows, 1 <= C <= min(N, 1024) clusters and 1 <= iters <= 1000.
  * ------------------------------------------------------------------------------------- */
 
-/* Scratch bytes of vsa_kmeans: cluster offsets [B*H, C+1] int32, centroid norms [B*H, C] fp32
- * and the centroids' bf16 halves [B*H, C, d] twice, each 256-byte aligned; 0 for an invalid
- * shape or count. */
+/* Scratch bytes of vsa_kmeans, each piece 256-byte aligned: cluster offsets and chunk offsets
+ * [B*H, C+1] int32 each, centroid norms [B*H, C] fp32, the centroids' bf16 halves [B*H, C, d]
+ * twice, and the update's partial sums over chunks of 128 members: [B*H, M, d] fp64 twice and
+ * int32 once, M = ceil(N / 128) + C.  0 for an invalid shape or count. */
 VSA_API size_t vsa_kmeans_workspace_size(const vsa_shape *shape, int n_clusters);
 
 /*
