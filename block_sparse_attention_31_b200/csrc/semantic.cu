@@ -57,7 +57,8 @@ __device__ __forceinline__ bool better(float dist, int j, float bd, int bj) {
 __global__ void __launch_bounds__(128) kmeans_init_kernel(const __nv_bfloat16* __restrict__ x, int N, int d, int C,
                                                           float* __restrict__ cent, float* __restrict__ cnorm,
                                                           __nv_bfloat16* __restrict__ chi,
-                                                          __nv_bfloat16* __restrict__ clo) {
+                                                          __nv_bfloat16* __restrict__ clo,
+                                                          int32_t* __restrict__ bad) {
   __shared__ float row_s[128];
   const int j = blockIdx.x, bh = blockIdx.y;
   const long long r = ((2LL * j + 1) * N) / (2LL * C);
@@ -73,6 +74,7 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(const __nv_bfloat16* _
   }
   __syncthreads();
   if (threadIdx.x == 0) cnorm[static_cast<size_t>(bh) * C + j] = sq_norm(row_s, d);
+  if (threadIdx.x == 0 && j == 0) bad[bh] = 0;  // the sort's label check starts clear
 }
 
 // label[bh, t] on the tensor cores: one CTA of 128 threads per 128 tokens of one head.  For each
@@ -197,49 +199,72 @@ __global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_cons
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
-// Counts, offsets and the stable cluster-major order of one head.  The head's tokens are cut
-// into kSortWarps contiguous segments, one per warp: per-segment histograms, offsets from their
-// column sums, each segment's first slot per cluster from the segments before it, then every
-// warp ranks its own segment in token order (32 tokens per step, ranks among equal labels from
-// __match_any_sync).  Shared memory: (kSortWarps + 1) * C ints.
+// Counts, offsets and the stable cluster-major order (slots sorted by (cluster, token)) of
+// every head, in three launches.  A head's tokens are cut into kSortSegs contiguous segments:
+//   hist     one CTA per (segment, head): the segment's label histogram;
+//   scan     one CTA per head: counts, offsets, chunk offsets (exclusive scans over the
+//            clusters), then every segment's first slot per cluster (segments before it);
+//   scatter  one CTA per (segment, head): the segment is cut again into kSortWarps warp
+//            segments with their own histograms, and every warp ranks its tokens in token
+//            order, 32 per step (ranks among equal labels from __match_any_sync).
+// A label outside [0, C) anywhere in a head sets VSA_DEVERR_KV_RANGE and leaves that head with
+// empty clusters (counts and offsets zero, no slot written).
 constexpr int kSortWarps = 16;
+constexpr int kSortSegs = 8;
 constexpr int kSortPrefetch = 8;  // 32-token steps whose labels are loaded ahead
 constexpr int kUpdChunk = 128;    // member rows per partial-sum CTA of the update
 
-__global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int32_t* __restrict__ label, int N, int C,
-                                                                      int32_t* __restrict__ counts,
-                                                                      int32_t* __restrict__ offsets,
-                                                                      int32_t* __restrict__ chunk_off,
-                                                                      int32_t* __restrict__ perm, int* err) {
-  extern __shared__ int sort_smem[];
-  int* hist = sort_smem;              // [kSortWarps][C]: counts, then first free slot, per segment
-  int* tot = sort_smem + kSortWarps * C;  // [C]
-  __shared__ int bad_s;
-  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__device__ __forceinline__ int seg_begin(int N, int nseg, int s) {
+  return static_cast<int>((static_cast<long long>(N) * s) / nseg);
+}
+
+// seg_hist [BH, kSortSegs, C]; bad [BH] (set to 1 on a label outside [0, C))
+__global__ void __launch_bounds__(256) kmeans_hist_kernel(const int32_t* __restrict__ label, int N, int C,
+                                                          int32_t* __restrict__ seg_hist, int32_t* __restrict__ bad) {
+  extern __shared__ int hist_smem[];
+  const int sg = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  for (int j = tid; j < C; j += blockDim.x) hist_smem[j] = 0;
+  __syncthreads();
   const int32_t* lh = label + static_cast<size_t>(bh) * N;
-  const int seg = (N + kSortWarps - 1) / kSortWarps;
-  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
-  for (int e = tid; e < kSortWarps * C; e += kSortWarps * 32) hist[e] = 0;
-  if (tid == 0) bad_s = 0;
-  __syncthreads();
-  for (int t = s0 + lane; t < s1; t += 32) {
+  const int a = seg_begin(N, kSortSegs, sg), b = seg_begin(N, kSortSegs, sg + 1);
+  bool badl = false;
+  for (int t = a + tid; t < b; t += blockDim.x) {
     const int l = lh[t];
-    if (l >= 0 && l < C) atomicAdd(&hist[warp * C + l], 1);
-    else bad_s = 1;
+    if (l >= 0 && l < C) atomicAdd(&hist_smem[l], 1);
+    else badl = true;
   }
+  if (badl) atomicExch(&bad[bh], 1);
   __syncthreads();
-  if (bad_s) {  // empty clusters: the update and the mask read nothing
+  int32_t* out = seg_hist + (static_cast<size_t>(bh) * kSortSegs + sg) * C;
+  for (int j = tid; j < C; j += blockDim.x) out[j] = hist_smem[j];
+}
+
+// Turns seg_hist into every segment's first slot per cluster, in place.
+__global__ void __launch_bounds__(256) kmeans_scan_kernel(int C, int32_t* __restrict__ seg_hist,
+                                                          int32_t* __restrict__ bad,
+                                                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ chunk_off, int* err) {
+  extern __shared__ int tot[];  // [C]
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int32_t* hh = seg_hist + static_cast<size_t>(bh) * kSortSegs * C;
+  const bool is_bad = bad[bh] != 0;
+  __syncthreads();
+  if (tid == 0) bad[bh] = 0;  // clear for the next round (the scatter tests offsets[C] instead)
+  if (is_bad) {  // empty clusters: the update and the mask read nothing
     if (tid == 0) atomicOr(err, kDevErrKvRange);
-    for (int j = tid; j < C; j += kSortWarps * 32) {
+    for (int j = tid; j < C; j += blockDim.x) {
       counts[static_cast<size_t>(bh) * C + j] = 0;
       offsets[static_cast<size_t>(bh) * (C + 1) + j] = 0;
     }
-    for (int j = tid; j <= C; j += kSortWarps * 32) chunk_off[static_cast<size_t>(bh) * (C + 1) + j] = 0;
+    for (int j = tid; j <= C; j += blockDim.x) {
+      chunk_off[static_cast<size_t>(bh) * (C + 1) + j] = 0;
+      if (j == C) offsets[static_cast<size_t>(bh) * (C + 1) + C] = 0;
+    }
     return;
   }
-  for (int j = tid; j < C; j += kSortWarps * 32) {
+  for (int j = tid; j < C; j += blockDim.x) {
     int sum = 0;
-    for (int w = 0; w < kSortWarps; ++w) sum += hist[w * C + j];
+    for (int sg = 0; sg < kSortSegs; ++sg) sum += hh[sg * C + j];
     tot[j] = sum;
     counts[static_cast<size_t>(bh) * C + j] = sum;
   }
@@ -276,8 +301,35 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int3
     }
   }
   __syncthreads();
-  for (int j = tid; j < C; j += kSortWarps * 32) {
+  for (int j = tid; j < C; j += blockDim.x) {
     int run = tot[j];
+    for (int sg = 0; sg < kSortSegs; ++sg) {
+      const int c = hh[sg * C + j];
+      hh[sg * C + j] = run;
+      run += c;
+    }
+  }
+}
+
+// Shared memory: kSortWarps * C ints.  A head whose labels were bad has offsets[C] = 0 != N.
+__global__ void __launch_bounds__(kSortWarps * 32) kmeans_scatter_kernel(const int32_t* __restrict__ label, int N,
+                                                                         int C, const int32_t* __restrict__ seg_start,
+                                                                         const int32_t* __restrict__ offsets,
+                                                                         int32_t* __restrict__ perm) {
+  extern __shared__ int sort_smem[];
+  int* hist = sort_smem;  // [kSortWarps][C]: counts, then first free slot, per warp segment
+  const int sg = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (offsets[static_cast<size_t>(bh) * (C + 1) + C] != N) return;
+  const int32_t* lh = label + static_cast<size_t>(bh) * N;
+  const int a = seg_begin(N, kSortSegs, sg), b = seg_begin(N, kSortSegs, sg + 1);
+  const int s0 = a + seg_begin(b - a, kSortWarps, warp), s1 = a + seg_begin(b - a, kSortWarps, warp + 1);
+  for (int e = tid; e < kSortWarps * C; e += kSortWarps * 32) hist[e] = 0;
+  __syncthreads();
+  for (int t = s0 + lane; t < s1; t += 32) atomicAdd(&hist[warp * C + lh[t]], 1);  // labels checked by hist
+  __syncthreads();
+  const int32_t* base = seg_start + (static_cast<size_t>(bh) * kSortSegs + sg) * C;
+  for (int j = tid; j < C; j += kSortWarps * 32) {
+    int run = base[j];
     for (int w = 0; w < kSortWarps; ++w) {
       const int c = hist[w * C + j];
       hist[w * C + j] = run;
@@ -288,16 +340,16 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_sort_kernel(const int3
   const unsigned lt = (1u << lane) - 1u;
   int* cur = hist + warp * C;
   int32_t* ph = perm + static_cast<size_t>(bh) * N;
-  for (int base = s0; base < s1; base += 32 * kSortPrefetch) {
+  for (int base_t = s0; base_t < s1; base_t += 32 * kSortPrefetch) {
     int lab[kSortPrefetch];
 #pragma unroll
     for (int u = 0; u < kSortPrefetch; ++u) {
-      const int t = base + u * 32 + lane;
+      const int t = base_t + u * 32 + lane;
       lab[u] = t < s1 ? lh[t] : -1;
     }
 #pragma unroll
     for (int u = 0; u < kSortPrefetch; ++u) {
-      const int t = base + u * 32 + lane;
+      const int t = base_t + u * 32 + lane;
       const int l = lab[u];
       const unsigned peers = __match_any_sync(0xffffffffu, l);
       const int rank = __popc(peers & lt);
@@ -704,6 +756,8 @@ struct KmWork {
   double* psum;        // [BH, max_chunks, d] chunk sums
   double* pabs;        // [BH, max_chunks, d] chunk sums of |v|
   int32_t* pq;         // [BH, max_chunks, d] chunk ulp exponents
+  int32_t* seg_hist;   // [BH, kSortSegs, C] segment histograms, then segment first slots
+  int32_t* bad;        // [BH] a label outside [0, C) was seen
   int max_chunks;      // ceil(N / kUpdChunk) + C bounds a head's chunk count
   size_t bytes;
 };
@@ -727,6 +781,8 @@ KmWork kmeans_layout(void* ws, int BH, int N, int C, int d) {
   w.psum = static_cast<double*>(take(bh * w.max_chunks * d * sizeof(double)));
   w.pabs = static_cast<double*>(take(bh * w.max_chunks * d * sizeof(double)));
   w.pq = static_cast<int32_t*>(take(bh * w.max_chunks * d * sizeof(int32_t)));
+  w.seg_hist = static_cast<int32_t*>(take(bh * kSortSegs * C * sizeof(int32_t)));
+  w.bad = static_cast<int32_t*>(take(bh * sizeof(int32_t)));
   w.bytes = off;
   return w;
 }
@@ -737,21 +793,25 @@ cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, fl
   using K = KmTcCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
-  const size_t ssmem = sizeof(int) * (kSortWarps + 1) * static_cast<size_t>(C);
+  const size_t ssmem = sizeof(int) * kSortWarps * static_cast<size_t>(C);
   if (ssmem > 48 * 1024) {
-    e = cudaFuncSetAttribute(kmeans_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem));
+    e = cudaFuncSetAttribute(kmeans_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(ssmem));
     if (e != cudaSuccess) return e;
   }
   CUtensorMap tx, thi, tlo;
   if ((e = encode_rows_map(&tx, x, D, N, BH, kTcRows)) != cudaSuccess) return e;
   if ((e = encode_rows_map(&thi, w.chi, D, C, BH, kTcRows)) != cudaSuccess) return e;
   if ((e = encode_rows_map(&tlo, w.clo, D, C, BH, kTcRows)) != cudaSuccess) return e;
-  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, w.cnorm, w.chi, w.clo);
+  kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, w.cnorm, w.chi, w.clo, w.bad);
   const dim3 agrid((N + kTcRows - 1) / kTcRows, BH), pgrid(w.max_chunks, BH), cgrid(C, BH);
   for (int it = 0; it < iters; ++it) {
     kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
-    kmeans_sort_kernel<<<BH, kSortWarps * 32, ssmem, stream>>>(label, N, C, counts, w.offsets, w.chunk_off, perm,
-                                                                err);
+    const dim3 sgrid(kSortSegs, BH);
+    kmeans_hist_kernel<<<sgrid, 256, sizeof(int) * C, stream>>>(label, N, C, w.seg_hist, w.bad);
+    kmeans_scan_kernel<<<BH, 256, sizeof(int) * C, stream>>>(C, w.seg_hist, w.bad, counts, w.offsets, w.chunk_off,
+                                                             err);
+    kmeans_scatter_kernel<<<sgrid, kSortWarps * 32, ssmem, stream>>>(label, N, C, w.seg_hist, w.offsets, perm);
     kmeans_partial_kernel<D><<<pgrid, kPartThreads, 0, stream>>>(x, N, C, w.offsets, w.chunk_off, perm, w.max_chunks,
                                                                  w.psum, w.pabs, w.pq);
     kmeans_combine_kernel<D><<<cgrid, D, 0, stream>>>(x, N, C, counts, w.offsets, w.chunk_off, perm, w.max_chunks,
