@@ -22,6 +22,7 @@
 // assignment's fp32 distances can differ from exact ones by a bounded amount: where two
 // centroids are that close to a tie, either label is a correct nearest-centroid choice.
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -44,10 +45,6 @@ __device__ __forceinline__ float sq_norm(const float* c, int D) {
   return acc;
 }
 
-// (dist, j) is a better assignment than (bd, bj): smaller distance, ties to the smaller index.
-__device__ __forceinline__ bool better(float dist, int j, float bd, int bj) {
-  return bj < 0 || dist < bd || (dist == bd && j < bj);
-}
 
 // ---------------------------------------------------------------------------------------
 // k-means
@@ -127,8 +124,8 @@ __global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = tmem_s;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  float best_d = 0.f;
-  int best_j = -1;
+  float best_d = INFINITY;
+  int best_j = 0;
   bool ok = true;
   const int ntiles = (C + kTcRows - 1) / kTcRows;
   for (int ct = 0; ct < ntiles && ok; ++ct) {
@@ -177,15 +174,13 @@ __global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_cons
       float sv[32];
       tmem_ld32(t_lane + q * 32, sv);
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
+      for (int x = 0; x < 32; ++x) {  // ascending index, strict <: ties keep the smaller index
         const int jl = q * 32 + x;
-        if (jl < nc) {
-          const float dist = __fmaf_rn(-2.f, sv[x], cn[jl]);  // |c|^2 - 2 s, rounded once
-          if (better(dist, c0 + jl, best_d, best_j)) {
-            best_d = dist;
-            best_j = c0 + jl;
-          }
-        }
+        float dist = __fmaf_rn(-2.f, sv[x], cn[jl]);  // |c|^2 - 2 s, rounded once
+        dist = jl < nc ? dist : INFINITY;
+        const bool lt = dist < best_d;
+        best_d = lt ? dist : best_d;
+        best_j = lt ? c0 + jl : best_j;
       }
     }
     tc_fence_before();
@@ -197,6 +192,175 @@ __global__ void __launch_bounds__(128) kmeans_assign_tc_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// The same assignment with the centroids resident, for C <= 128 * NCT (NCT <= 2): CTAs are
+// persistent per head (grid (ctas_per_head, BH)) and walk the head's token tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...  The centroid halves are loaded once; token tiles
+// stream through two shared-memory stages and S through two TMEM buffers, so the load of the
+// next tile and its MMAs overlap this tile's argmin.  Roles: warp 8 lane 0 loads (TMA),
+// warp 9 lane 0 issues the MMAs; warps 0-3 and 4-7 (one token row per thread) read S buffer 0
+// and 1 respectively (even and odd tiles) and write the labels.
+constexpr int kPcThreads = 320;
+
+template <int D, int NCT>
+struct KmPcCfg {
+  static constexpr int X_BYTES = kTcRows * D * 2;      // one token tile
+  static constexpr int CT_BYTES = kTcRows * D * 2;     // one 128-centroid tile of one half
+  static constexpr int OFF_C = 0;                      // [NCT][hi, lo]
+  static constexpr int OFF_X = NCT * 2 * CT_BYTES;     // [2 stages]
+  static constexpr int OFF_BAR = OFF_X + 2 * X_BYTES;  // 9 barriers
+  static constexpr int OFF_CN = OFF_BAR + 128;         // [NCT * 128] centroid norms
+  static constexpr int SMEM = OFF_CN + NCT * kTcRows * 4 + 1024;
+  static constexpr int SCOLS = NCT * kTcRows;          // TMEM columns of one S buffer
+  static constexpr int TMEM_COLS = 2 * SCOLS;          // 256 or 512
+  static constexpr uint32_t IDESC = idesc_bf16_f32(kTcRows, kTcRows, false, false);
+};
+
+enum { KB_C = 0, KB_XF = 1, KB_XE = 3, KB_SF = 5, KB_SE = 7 };
+
+template <int D, int NCT>
+__global__ void __launch_bounds__(kPcThreads, 1)
+    kmeans_assign_pc_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap thi,
+                            const __grid_constant__ CUtensorMap tlo, int N, int C, const float* __restrict__ cnorm,
+                            int32_t* __restrict__ label, int* err) {
+  using K = KmPcCfg<D, NCT>;
+  extern __shared__ uint8_t pc_raw[];
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  const int bh = blockIdx.y;
+  const int ntiles = (N + kTcRows - 1) / kTcRows;
+  const int mine = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;  // tiles of this CTA
+  if (mine == 0) return;
+  const uint32_t raw = smem_u32(pc_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  float* cn = reinterpret_cast<float*>(pc_raw + (sb - raw) + K::OFF_CN);
+  auto bar = [&](int i) -> uint32_t { return sb + K::OFF_BAR + 8u * i; };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &abort_s;
+  if (tid == 0) {
+    mbar_init(bar(KB_C), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(KB_XF + s), 1);
+      mbar_init(bar(KB_XE + s), 1);
+      mbar_init(bar(KB_SF + s), 1);
+      mbar_init(bar(KB_SE + s), 128);
+    }
+    mbar_init_fence();
+    abort_s = 0;
+  }
+  for (int c = tid; c < NCT * kTcRows; c += kPcThreads) cn[c] = c < C ? cnorm[static_cast<size_t>(bh) * C + c] : 0.f;
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&tmem_s), K::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+
+  if (warp == 8) {  // ---- loads ----
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(KB_C), NCT * 2 * K::CT_BYTES);
+#pragma unroll
+      for (int ct = 0; ct < NCT; ++ct)
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t dst = sb + K::OFF_C + (2 * ct) * K::CT_BYTES + c * kTcRows * 128;
+          tma_load_3d(dst, &thi, bar(KB_C), c * 64, ct * kTcRows, bh);
+          tma_load_3d(dst + K::CT_BYTES, &tlo, bar(KB_C), c * 64, ct * kTcRows, bh);
+        }
+      int issued = 0;
+      for (int li = 0; li < mine; ++li) {
+        const int s = li & 1;
+        if (li >= 2 && !mbar_wait(bar(KB_XE + s), ((li - 2) >> 1) & 1, abort_flag, err)) break;
+        const int t0 = (blockIdx.x + li * gridDim.x) * kTcRows;
+        mbar_arrive_expect_tx(bar(KB_XF + s), K::X_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sb + K::OFF_X + s * K::X_BYTES + c * kTcRows * 128, &tx, bar(KB_XF + s), c * 64, t0, bh);
+        issued = li + 1;
+      }
+      // every issued copy lands before the CTA exits (a copy older than the last two was
+      // consumed by an MMA, whose completion freed its stage for a later copy)
+      mbar_wait_drain(bar(KB_C), 0, err);
+      for (int li = (issued > 2 ? issued - 2 : 0); li < issued; ++li)
+        mbar_wait_drain(bar(KB_XF + (li & 1)), (li >> 1) & 1, err);
+    }
+    __syncwarp();
+  } else if (warp == 9) {  // ---- MMAs ----
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(KB_C), 0, abort_flag, err);
+      int issued = 0;
+      for (int li = 0; ok && li < mine; ++li) {
+        const int s = li & 1;
+        if (!mbar_wait(bar(KB_XF + s), (li >> 1) & 1, abort_flag, err)) break;
+        if (li >= 2 && !mbar_wait(bar(KB_SE + s), ((li - 2) >> 1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint64_t dx = sdesc_sw128(sb + K::OFF_X + s * K::X_BYTES, 16, 1024);
+#pragma unroll
+        for (int ct = 0; ct < NCT; ++ct) {
+          const uint64_t dh = sdesc_sw128(sb + K::OFF_C + (2 * ct) * K::CT_BYTES, 16, 1024);
+          const uint64_t dl = sdesc_sw128(sb + K::OFF_C + (2 * ct + 1) * K::CT_BYTES, 16, 1024);
+          const uint32_t d_s = tmem + s * K::SCOLS + ct * kTcRows;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (kTcRows * 128) + (kk & 3) * 32) / 16);
+            tc_mma_ss(d_s, dx + off, dh + off, K::IDESC, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (kTcRows * 128) + (kk & 3) * 32) / 16);
+            tc_mma_ss(d_s, dx + off, dl + off, K::IDESC, 1u);
+          }
+        }
+        tc_commit(bar(KB_XE + s));
+        tc_commit(bar(KB_SF + s));
+        issued = li + 1;
+      }
+      // every issued MMA completes before TMEM is released: the last commits cover them
+      if (issued > 0) mbar_wait_drain(bar(KB_SF + ((issued - 1) & 1)), ((issued - 1) >> 1) & 1, err);
+    }
+    __syncwarp();
+  } else {  // ---- argmin: warpgroup g = warp / 4 takes the tiles li = g, g + 2, ...; row = lane quarter ----
+    const int g = warp >> 2, row = (warp & 3) * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + g * K::SCOLS;
+    for (int li = g; li < mine; li += 2) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(KB_SF + g), (li >> 1) & 1, abort_flag, err))) break;
+      tc_fence_after();
+      // ascending centroid index with a strict < keeps the smaller index on ties
+      float best_d = INFINITY;
+      int best_j = 0;
+#pragma unroll
+      for (int ct = 0; ct < NCT; ++ct) {
+        const int c0 = ct * kTcRows;
+        const int nc = min(kTcRows, C - c0);
+#pragma unroll 1
+        for (int q = 0; q < kTcRows / 32; ++q) {
+          if (q * 32 >= nc) break;
+          float sv[32];
+          tmem_ld32(t_lane + c0 + q * 32, sv);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int jl = q * 32 + x;
+            float dist = __fmaf_rn(-2.f, sv[x], cn[c0 + jl]);  // |c|^2 - 2 s, rounded once
+            dist = jl < nc ? dist : INFINITY;
+            const bool lt = dist < best_d;
+            best_d = lt ? dist : best_d;
+            best_j = lt ? c0 + jl : best_j;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(KB_SE + g));  // S buffer g may be overwritten
+      const int t = (blockIdx.x + li * gridDim.x) * kTcRows + row;
+      if (t < N) label[static_cast<size_t>(bh) * N + t] = best_j;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, K::TMEM_COLS);
 }
 
 // Counts, offsets and the stable cluster-major order (slots sorted by (cluster, token)) of
@@ -805,8 +969,32 @@ cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, fl
   if ((e = encode_rows_map(&tlo, w.clo, D, C, BH, kTcRows)) != cudaSuccess) return e;
   kmeans_init_kernel<<<dim3(C, BH), 128, 0, stream>>>(x, N, D, C, cent, w.cnorm, w.chi, w.clo, w.bad);
   const dim3 agrid((N + kTcRows - 1) / kTcRows, BH), pgrid(w.max_chunks, BH), cgrid(C, BH);
+  // resident centroids (C <= 256): persistent CTAs, one per SM, spread evenly over the heads;
+  // the shared-memory request keeps one CTA per SM so that TMEM never oversubscribes
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int ntiles = (N + kTcRows - 1) / kTcRows;
+  const dim3 pcgrid(std::min(ntiles, std::max(1, sms / BH)), BH);
+  const int pc1 = std::max(KmPcCfg<D, 1>::SMEM, 120 * 1024), pc2 = std::max(KmPcCfg<D, 2>::SMEM, 120 * 1024);
+  if (C <= kTcRows) {
+    if ((e = cudaFuncSetAttribute(kmeans_assign_pc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, pc1)) !=
+        cudaSuccess)
+      return e;
+  } else if (C <= 2 * kTcRows) {
+    if ((e = cudaFuncSetAttribute(kmeans_assign_pc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, pc2)) !=
+        cudaSuccess)
+      return e;
+  }
   for (int it = 0; it < iters; ++it) {
-    kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
+    if (C <= kTcRows)
+      kmeans_assign_pc_kernel<D, 1><<<pcgrid, kPcThreads, pc1, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
+    else if (C <= 2 * kTcRows)
+      kmeans_assign_pc_kernel<D, 2><<<pcgrid, kPcThreads, pc2, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
+    else
+      kmeans_assign_tc_kernel<D><<<agrid, 128, K::SMEM, stream>>>(tx, thi, tlo, N, C, w.cnorm, label, err);
     const dim3 sgrid(kSortSegs, BH);
     kmeans_hist_kernel<<<sgrid, 256, sizeof(int) * C, stream>>>(label, N, C, w.seg_hist, w.bad);
     kmeans_scan_kernel<<<BH, 256, sizeof(int) * C, stream>>>(C, w.seg_hist, w.bad, counts, w.offsets, w.chunk_off,

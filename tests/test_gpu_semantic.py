@@ -76,10 +76,12 @@ def _check_kmeans_rounds(x_head, runs, h, C, what):
 
 
 @pytest.mark.parametrize("F,Hl,Wl,d,C,iters", [(5, 7, 13, 64, 16, 3), (5, 7, 13, 128, 200, 2),
-                                               (3, 10, 20, 128, 1, 1), (4, 8, 16, 64, 512, 2)])
+                                               (3, 10, 20, 128, 1, 1), (4, 8, 16, 64, 512, 2),
+                                               (4, 8, 16, 64, 250, 2), (5, 7, 13, 128, 300, 1)])
 def test_kmeans_matches_oracle(F, Hl, Wl, d, C, iters):
     """Every round's labels (valid nearest centroids), centroids, counts and order (ragged N,
-    one and several centroid tiles, a single cluster)."""
+    a single cluster; one or two resident centroid tiles (C <= 256) and streamed tiles above
+    that, for d = 64 and 128)."""
     wl = _wl(F, Hl, Wl, d)
     q, k, _ = synthetic.make_qkv(wl)
     shape = _lib.make_shape(1, wl.H, F, Hl, Wl, d, 128)
