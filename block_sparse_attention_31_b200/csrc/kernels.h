@@ -32,7 +32,7 @@ constexpr int kMaxClusters = 1024;
 // (slot -> token, cluster-major).  ws (kmeans_workspace_bytes): the cluster offsets and
 // partial-sum chunk offsets [BH, C + 1], the centroids' squared norms [BH, C], their bf16
 // halves [BH, C, d] twice, the update's chunk sums [BH, ceil(N / 128) + C, d], and the
-// sort's segment histograms [BH, 8, C] with one flag per head.
+// sort's segment histograms [BH, 8, C] with one flag per head, and the chunks' clusters.
 size_t kmeans_workspace_bytes(int BH, int N, int C, int d);
 cudaError_t launch_kmeans(const void* x, int BH, int N, int d, int C, int iters, float* cent, int32_t* label,
                           int32_t* counts, int32_t* perm, void* ws, int* err, cudaStream_t stream);

@@ -407,7 +407,8 @@ __global__ void __launch_bounds__(256) kmeans_hist_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(256) kmeans_scan_kernel(int C, int32_t* __restrict__ seg_hist,
                                                           int32_t* __restrict__ bad,
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ chunk_off, int* err) {
+                                                          int32_t* __restrict__ chunk_off,
+                                                          int32_t* __restrict__ chunk_cl, int max_chunks, int* err) {
   extern __shared__ int tot[];  // [C]
   const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int32_t* hh = seg_hist + static_cast<size_t>(bh) * kSortSegs * C;
@@ -472,6 +473,9 @@ __global__ void __launch_bounds__(256) kmeans_scan_kernel(int C, int32_t* __rest
       hh[sg * C + j] = run;
       run += c;
     }
+    // the cluster of every partial-sum chunk (the chunks of j follow its chunk offset)
+    const int32_t* co = chunk_off + static_cast<size_t>(bh) * (C + 1);
+    for (int k = co[j]; k < co[j + 1]; ++k) chunk_cl[static_cast<size_t>(bh) * max_chunks + k] = j;
   }
 }
 
@@ -542,15 +546,8 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_scatter_kernel(const i
 // point exactly when it does in exact arithmetic, so the check itself is exact.
 constexpr int kNoUlp = 1000;  // q of a dimension with no nonzero member
 
-// ulp exponent of a nonzero bf16 value from its bits (kNoUlp for +-0)
-__device__ __forceinline__ int bf16_ulp_exp(uint32_t bits) {
-  const int be = static_cast<int>((bits >> 7) & 0xffu);
-  if ((bits & 0x7fffu) == 0u) return kNoUlp;
-  return be == 0 ? -133 : be - 134;
-}
-
-// One CTA of kPartThreads per chunk k of a head's chunk list (the chunk's cluster is the last j
-// with chunk_off[j] <= k; empty clusters own no chunk).  The chunk's member indices go to
+// One CTA of kPartThreads per chunk k of a head's chunk list (chunk_cl[k]: the chunk's cluster,
+// written by the scan).  The chunk's member indices go to
 // shared memory first; thread (row lane rl, dimension group g) then loads 16-byte pieces (8
 // dimensions) of rows rl, rl + RL, ... all independently, and the row lanes' partial sums
 // are added through shared memory (any order: see above).
@@ -560,6 +557,7 @@ template <int D>
 __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv_bfloat16* __restrict__ x, int N,
                                                                       int C, const int32_t* __restrict__ offsets,
                                                                       const int32_t* __restrict__ chunk_off,
+                                                                      const int32_t* __restrict__ chunk_cl,
                                                                       const int32_t* __restrict__ perm, int max_chunks,
                                                                       double* __restrict__ psum,
                                                                       double* __restrict__ pabs,
@@ -574,13 +572,7 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
   const int k = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int32_t* co = chunk_off + static_cast<size_t>(bh) * (C + 1);
   if (k >= co[C]) return;
-  int lo = 0, hi = C - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (co[mid] <= k) lo = mid;
-    else hi = mid - 1;
-  }
-  const int j = lo;
+  const int j = chunk_cl[static_cast<size_t>(bh) * max_chunks + k];
   const int32_t* off = offsets + static_cast<size_t>(bh) * (C + 1);
   const int first = (k - co[j]) * kUpdChunk;
   const int cnt = min(kUpdChunk, off[j + 1] - off[j] - first);
@@ -592,13 +584,17 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
   __syncthreads();
   const int g = tid % G, rl = tid / G;
   const uint4* xh = reinterpret_cast<const uint4*>(x + static_cast<size_t>(bh) * N * D);
-  double sa[8], aa[8];
-  int qa[8];
+  // Per dimension: the fp32 sum and |v| sum of this thread's PER rows, and the smallest nonzero
+  // magnitude (15-bit bf16 pattern, packed in 16-bit halves, zeros counted as 0xffff).  The
+  // fp32 sums are exact while the |v| sum stays below 2^(q + 24) (the argument above with a
+  // 24-bit significand); a thread whose sums may not be exact adds its rows again in fp64.
+  uint64_t s2[4], a2[4];
+  uint32_t mm[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    sa[e] = 0.0;
-    aa[e] = 0.0;
-    qa[e] = kNoUlp;
+  for (int p = 0; p < 4; ++p) {
+    s2[p] = 0ull;
+    a2[p] = 0ull;
+    mm[p] = 0xffffffffu;
   }
   constexpr int BATCH = PER < 8 ? PER : 8;  // rows loaded before any is added
 #pragma unroll
@@ -611,14 +607,52 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
     }
 #pragma unroll
     for (int i = 0; i < BATCH; ++i) {
+      const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {  // dimensions 2p (low half) and 2p + 1 (high half)
+        const uint32_t lo = ww[p] << 16, hi = ww[p] & 0xffff0000u;
+        s2[p] = f2_add(s2[p], f2_make(__uint_as_float(lo), __uint_as_float(hi)));
+        a2[p] = f2_add(a2[p], f2_make(__uint_as_float(lo & 0x7fffffffu), __uint_as_float(hi & 0x7fffffffu)));
+        const uint32_t mag = ww[p] & 0x7fff7fffu;
+        mm[p] = __vminu2(mm[p], mag | __vcmpeq2(mag, 0u));
+      }
+    }
+  }
+  double sa[8], aa[8];
+  int qa[8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    float f0, f1, g0, g1;
+    f2_split(s2[p], f0, f1);
+    f2_split(a2[p], g0, g1);
+    const uint32_t m0 = mm[p] & 0xffffu, m1 = mm[p] >> 16;
+    // ulp exponent of the smallest nonzero magnitude: max(exponent field, 1) - 134
+    qa[2 * p] = m0 == 0xffffu ? kNoUlp : max(static_cast<int>(m0 >> 7), 1) - 134;
+    qa[2 * p + 1] = m1 == 0xffffu ? kNoUlp : max(static_cast<int>(m1 >> 7), 1) - 134;
+    sa[2 * p] = f0;
+    sa[2 * p + 1] = f1;
+    aa[2 * p] = g0;
+    aa[2 * p + 1] = g1;
+  }
+  bool exact = true;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) exact = exact && (aa[e] < ldexp(1.0, min(qa[e], 200) + 24));
+  if (!exact) {  // rare: the same rows again in fp64
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sa[e] = 0.0;
+      aa[e] = 0.0;
+    }
+    for (int i = 0; i < PER; ++i) {
+      const int t = rows_s[rl + i * RL];
+      const uint4 v4 = t >= 0 ? __ldg(xh + static_cast<size_t>(t) * G + g) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t ww[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const uint32_t word = e < 2 ? w[i].x : e < 4 ? w[i].y : e < 6 ? w[i].z : w[i].w;
-        const uint32_t bits = (e & 1) ? (word >> 16) : (word & 0xffffu);
-        const double v = static_cast<double>(__uint_as_float(bits << 16));
+        const uint32_t bits = (e & 1) ? (ww[e >> 1] & 0xffff0000u) : (ww[e >> 1] << 16);
+        const double v = static_cast<double>(__uint_as_float(bits));
         sa[e] += v;
         aa[e] += fabs(v);
-        qa[e] = min(qa[e], bf16_ulp_exp(bits));
       }
     }
   }
@@ -921,6 +955,7 @@ struct KmWork {
   double* pabs;        // [BH, max_chunks, d] chunk sums of |v|
   int32_t* pq;         // [BH, max_chunks, d] chunk ulp exponents
   int32_t* seg_hist;   // [BH, kSortSegs, C] segment histograms, then segment first slots
+  int32_t* chunk_cl;   // [BH, max_chunks] cluster of every partial-sum chunk
   int32_t* bad;        // [BH] a label outside [0, C) was seen
   int max_chunks;      // ceil(N / kUpdChunk) + C bounds a head's chunk count
   size_t bytes;
@@ -947,6 +982,7 @@ KmWork kmeans_layout(void* ws, int BH, int N, int C, int d) {
   w.pq = static_cast<int32_t*>(take(bh * w.max_chunks * d * sizeof(int32_t)));
   w.seg_hist = static_cast<int32_t*>(take(bh * kSortSegs * C * sizeof(int32_t)));
   w.bad = static_cast<int32_t*>(take(bh * sizeof(int32_t)));
+  w.chunk_cl = static_cast<int32_t*>(take(bh * w.max_chunks * sizeof(int32_t)));
   w.bytes = off;
   return w;
 }
@@ -998,10 +1034,10 @@ cudaError_t kmeans_d(const __nv_bfloat16* x, int BH, int N, int C, int iters, fl
     const dim3 sgrid(kSortSegs, BH);
     kmeans_hist_kernel<<<sgrid, 256, sizeof(int) * C, stream>>>(label, N, C, w.seg_hist, w.bad);
     kmeans_scan_kernel<<<BH, 256, sizeof(int) * C, stream>>>(C, w.seg_hist, w.bad, counts, w.offsets, w.chunk_off,
-                                                             err);
+                                                             w.chunk_cl, w.max_chunks, err);
     kmeans_scatter_kernel<<<sgrid, kSortWarps * 32, ssmem, stream>>>(label, N, C, w.seg_hist, w.offsets, perm);
-    kmeans_partial_kernel<D><<<pgrid, kPartThreads, 0, stream>>>(x, N, C, w.offsets, w.chunk_off, perm, w.max_chunks,
-                                                                 w.psum, w.pabs, w.pq);
+    kmeans_partial_kernel<D><<<pgrid, kPartThreads, 0, stream>>>(x, N, C, w.offsets, w.chunk_off, w.chunk_cl, perm,
+                                                                 w.max_chunks, w.psum, w.pabs, w.pq);
     kmeans_combine_kernel<D><<<cgrid, D, 0, stream>>>(x, N, C, counts, w.offsets, w.chunk_off, perm, w.max_chunks,
                                                       w.psum, w.pabs, w.pq, cent, w.cnorm, w.chi, w.clo);
   }

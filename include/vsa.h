@@ -402,8 +402,9 @@ VSA_API vsa_status vsa_attention_workspace_layout(const vsa_shape *shape, const 
 /* Scratch bytes of vsa_kmeans, each piece 256-byte aligned: cluster offsets and chunk offsets
  * [B*H, C+1] int32 each, centroid norms [B*H, C] fp32, the centroids' bf16 halves [B*H, C, d]
  * twice, the update's partial sums over chunks of 128 members ([B*H, M, d] fp64 twice and
- * int32 once, M = ceil(N / 128) + C), the sort's segment histograms [B*H, 8, C] int32 and one
- * int32 flag per head.  0 for an invalid shape or count. */
+ * int32 once, M = ceil(N / 128) + C), the sort's segment histograms [B*H, 8, C] int32, one
+ * int32 flag per head and the chunks' clusters [B*H, M] int32.  0 for an invalid shape or
+ * count. */
 VSA_API size_t vsa_kmeans_workspace_size(const vsa_shape *shape, int n_clusters);
 
 /*

@@ -170,12 +170,13 @@ def test_semantic_entry_points_validate_before_launch():
     cube = _lib.make_shape(1, 2, 8, 8, 8, 64, 128, (4, 4, 8))
     # offsets and chunk offsets B*H*(C+1) int32, norms B*H*C fp32, two bf16 halves B*H*C*d,
     # the update's chunk sums B*H*M*d (fp64 twice, int32 once), M = ceil(N/128) + C, the sort's
-    # segment histograms B*H*8*C int32 and one flag per head; each piece 256-aligned
+    # segment histograms B*H*8*C int32, one flag per head and the chunk -> cluster map B*H*M
+    # int32; each piece 256-aligned
     m16, m64 = 2 + 16, 2 + 64
     assert _lib.vsa_kmeans_workspace_size(shape, 16) == (2 * 256 + 256 + 2 * 4096 + 2 * (2 * m16 * 64 * 8)
-                                                        + 2 * m16 * 64 * 4 + 1024 + 256)
+                                                        + 2 * m16 * 64 * 4 + 1024 + 256 + 256)
     assert _lib.vsa_kmeans_workspace_size(shape, 64) == (2 * 768 + 512 + 2 * 16384 + 2 * (2 * m64 * 64 * 8)
-                                                        + 2 * m64 * 64 * 4 + 4096 + 256)
+                                                        + 2 * m64 * 64 * 4 + 4096 + 256 + 768)
     assert _lib.vsa_kmeans_workspace_size(shape, 0) == 0
     assert _lib.vsa_kmeans_workspace_size(shape, 257) == 0   # more clusters than rows
     assert _lib.vsa_kmeans_workspace_size(cube, 16) == 0
