@@ -92,6 +92,24 @@ def test_kmeans_matches_oracle(F, Hl, Wl, d, C, iters):
             _check_kmeans_rounds(x[0, h], runs, h, C, f"{name} head {h}")
 
 
+def test_kmeans_update_wide_range_exact():
+    """Member values of one dimension spanning more than 53 binades (2^-60 next to values of
+    order 1): the update's parallel sums are not provably exact there, so both of its fallbacks
+    run (a thread's fp32 sums redone in fp64, and the cluster's ordered token-order sum); the
+    centroids must still equal the oracle's token-order fp64 update bit for bit."""
+    F, Hl, Wl, d, C = 4, 8, 16, 64, 8
+    N = F * Hl * Wl
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    x[0, 0, ::3, 5] = 2.0 ** -60
+    x[0, 0, 1::7, 9] = -3 * 2.0 ** -60
+    assert float(x[0, 0, 0, 5]) == 2.0 ** -60       # exact in bf16
+    shape = _lib.make_shape(1, 1, F, Hl, Wl, d, 128)
+    xd = x.cuda()
+    runs = [_kmeans_gpu(xd, shape, C, T) for T in range(1, 3)]
+    _check_kmeans_rounds(x[0, 0], runs, 0, C, "wide-range head")
+
+
 def test_kmeans_wan_heads_match_oracle():
     """The Wan grid at the benchmark's cluster counts and rounds: one spatial- and one
     temporal-structured head, every round."""
