@@ -547,14 +547,15 @@ __global__ void __launch_bounds__(kSortWarps * 32) kmeans_scatter_kernel(const i
 constexpr int kNoUlp = 1000;  // q of a dimension with no nonzero member
 
 // One CTA of kPartThreads per chunk k of a head's chunk list (chunk_cl[k]: the chunk's cluster,
-// written by the scan).  The chunk's member indices go to
-// shared memory first; thread (row lane rl, dimension group g) then loads 16-byte pieces (8
-// dimensions) of rows rl, rl + RL, ... all independently, and the row lanes' partial sums
-// are added through shared memory (any order: see above).
+// written by the scan).  Thread (row lane rl, dimension group g) loads 16-byte pieces (8
+// dimensions) of rows rl, rl + RL, ... all at once (the member index of a row is one load the
+// G threads of a row share), so a CTA waits for one round of memory latency; the row lanes'
+// partial sums are then added with shuffles inside each warp and through shared memory across
+// the warps (any order: see above).
 constexpr int kPartThreads = 128;
 
 template <int D>
-__global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv_bfloat16* __restrict__ x, int N,
+__global__ void __launch_bounds__(kPartThreads, 4) kmeans_partial_kernel(const __nv_bfloat16* __restrict__ x, int N,
                                                                       int C, const int32_t* __restrict__ offsets,
                                                                       const int32_t* __restrict__ chunk_off,
                                                                       const int32_t* __restrict__ chunk_cl,
@@ -565,11 +566,12 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
   constexpr int G = D / 8;               // dimension groups of 8
   constexpr int RL = kPartThreads / G;   // row lanes
   constexpr int PER = kUpdChunk / RL;    // rows per thread
-  __shared__ int rows_s[kUpdChunk];
-  __shared__ double red_s[RL][D];
-  __shared__ double reda_s[RL][D];
-  __shared__ int redq_s[RL][D];
-  const int k = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  constexpr int NW = kPartThreads / 32;  // warps
+  static_assert(G <= 32 && 32 % G == 0, "a warp holds whole rows");
+  __shared__ double red_s[NW][D];
+  __shared__ double reda_s[NW][D];
+  __shared__ int redq_s[NW][D];
+  const int k = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t* co = chunk_off + static_cast<size_t>(bh) * (C + 1);
   if (k >= co[C]) return;
   const int j = chunk_cl[static_cast<size_t>(bh) * max_chunks + k];
@@ -577,13 +579,19 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
   const int first = (k - co[j]) * kUpdChunk;
   const int cnt = min(kUpdChunk, off[j + 1] - off[j] - first);
   const int32_t* ph = perm + static_cast<size_t>(bh) * N + off[j] + first;
-  for (int r = tid; r < kUpdChunk; r += kPartThreads) {
-    const int t = r < cnt ? ph[r] : -1;
-    rows_s[r] = (t >= 0 && t < N) ? t : -1;
-  }
-  __syncthreads();
   const int g = tid % G, rl = tid / G;
   const uint4* xh = reinterpret_cast<const uint4*>(x + static_cast<size_t>(bh) * N * D);
+  int rows[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int r = rl + i * RL;
+    const int t = r < cnt ? __ldg(ph + r) : -1;
+    rows[i] = (t >= 0 && t < N) ? t : -1;
+  }
+  uint4 w[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i)
+    w[i] = rows[i] >= 0 ? __ldg(xh + static_cast<size_t>(rows[i]) * G + g) : make_uint4(0u, 0u, 0u, 0u);
   // Per dimension: the fp32 sum and |v| sum of this thread's PER rows, and the smallest nonzero
   // magnitude (15-bit bf16 pattern, packed in 16-bit halves, zeros counted as 0xffff).  The
   // fp32 sums are exact while the |v| sum stays below 2^(q + 24) (the argument above with a
@@ -596,26 +604,16 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
     a2[p] = 0ull;
     mm[p] = 0xffffffffu;
   }
-  constexpr int BATCH = PER < 8 ? PER : 8;  // rows loaded before any is added
 #pragma unroll
-  for (int i0 = 0; i0 < PER; i0 += BATCH) {
-    uint4 w[BATCH];
+  for (int i = 0; i < PER; ++i) {
+    const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
-    for (int i = 0; i < BATCH; ++i) {
-      const int t = rows_s[rl + (i0 + i) * RL];
-      w[i] = t >= 0 ? __ldg(xh + static_cast<size_t>(t) * G + g) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < BATCH; ++i) {
-      const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {  // dimensions 2p (low half) and 2p + 1 (high half)
-        const uint32_t lo = ww[p] << 16, hi = ww[p] & 0xffff0000u;
-        s2[p] = f2_add(s2[p], f2_make(__uint_as_float(lo), __uint_as_float(hi)));
-        a2[p] = f2_add(a2[p], f2_make(__uint_as_float(lo & 0x7fffffffu), __uint_as_float(hi & 0x7fffffffu)));
-        const uint32_t mag = ww[p] & 0x7fff7fffu;
-        mm[p] = __vminu2(mm[p], mag | __vcmpeq2(mag, 0u));
-      }
+    for (int p = 0; p < 4; ++p) {  // dimensions 2p (low half) and 2p + 1 (high half)
+      const uint32_t lo = ww[p] << 16, hi = ww[p] & 0xffff0000u;
+      s2[p] = f2_add(s2[p], f2_make(__uint_as_float(lo), __uint_as_float(hi)));
+      a2[p] = f2_add(a2[p], f2_make(__uint_as_float(lo & 0x7fffffffu), __uint_as_float(hi & 0x7fffffffu)));
+      const uint32_t mag = ww[p] & 0x7fff7fffu;
+      mm[p] = __vminu2(mm[p], mag | __vcmpeq2(mag, 0u));
     }
   }
   double sa[8], aa[8];
@@ -643,9 +641,11 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
       sa[e] = 0.0;
       aa[e] = 0.0;
     }
+#pragma unroll 1
     for (int i = 0; i < PER; ++i) {
-      const int t = rows_s[rl + i * RL];
-      const uint4 v4 = t >= 0 ? __ldg(xh + static_cast<size_t>(t) * G + g) : make_uint4(0u, 0u, 0u, 0u);
+      const int r = rl + i * RL;
+      const int t = r < cnt ? __ldg(ph + r) : -1;
+      const uint4 v4 = (t >= 0 && t < N) ? __ldg(xh + static_cast<size_t>(t) * G + g) : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t ww[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -656,24 +656,37 @@ __global__ void __launch_bounds__(kPartThreads) kmeans_partial_kernel(const __nv
       }
     }
   }
+  // row lanes of one warp (lanes g, g + G, ...), then the warps
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    red_s[rl][g * 8 + e] = sa[e];
-    reda_s[rl][g * 8 + e] = aa[e];
-    redq_s[rl][g * 8 + e] = qa[e];
+  for (int o = G; o < 32; o <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sa[e] += __shfl_xor_sync(0xffffffffu, sa[e], o);
+      aa[e] += __shfl_xor_sync(0xffffffffu, aa[e], o);
+      qa[e] = min(qa[e], __shfl_xor_sync(0xffffffffu, qa[e], o));
+    }
+  }
+  if (lane < G) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red_s[warp][g * 8 + e] = sa[e];
+      reda_s[warp][g * 8 + e] = aa[e];
+      redq_s[warp][g * 8 + e] = qa[e];
+    }
   }
   __syncthreads();
   for (int dd = tid; dd < D; dd += kPartThreads) {
-    double s = 0.0, a = 0.0;
+    double sm = 0.0, am = 0.0;
     int q = kNoUlp;
-    for (int l = 0; l < RL; ++l) {
-      s += red_s[l][dd];
-      a += reda_s[l][dd];
+#pragma unroll
+    for (int l = 0; l < NW; ++l) {
+      sm += red_s[l][dd];
+      am += reda_s[l][dd];
       q = min(q, redq_s[l][dd]);
     }
     const size_t o = (static_cast<size_t>(bh) * max_chunks + k) * D + dd;
-    psum[o] = s;
-    pabs[o] = a;
+    psum[o] = sm;
+    pabs[o] = am;
     pq[o] = q;
   }
 }
