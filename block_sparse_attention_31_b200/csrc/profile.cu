@@ -36,9 +36,9 @@ constexpr int kProfThreads = 320;  // producer, MMA issuer, two softmax warpgrou
 constexpr int kPM = 128;  // rows per tile
 constexpr int kNumSMs = 148;
 constexpr int kMaxSplits = 16;  // key-range splits per row tile, at most
-// A masked variant whose largest allowed logit lies more than this many base-2 units under
-// the dense running maximum is recomputed exactly: with a margin of 80, every probability the
-// 2^-126 flush can remove is below 2^-46 of the variant's own largest one.
+// The margin the recompute rule below guarantees: a masked variant that is not recomputed has
+// its largest allowed logit within this many base-2 units of every split's dense maximum, so
+// every probability the 2^-126 flush can remove is below 2^-46 of the variant's own largest one.
 constexpr float kProfFlushMargin = 80.0f;
 // Merged masked-variant sums below this (2^-60 of the dense maximum) trigger the recompute:
 // 60 + 18 (at most 2^18 keys) stays inside kProfFlushMargin.
