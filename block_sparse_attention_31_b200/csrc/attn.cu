@@ -184,6 +184,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   bool stop = false;
   if (tid == 0) stop = (*reinterpret_cast<volatile int*>(a.err) & kDevErrTimeout) != 0;
   if (__syncthreads_or(stop)) return;
+  // Q tiles by TMA before anything else, so that their load overlaps the list validation and
+  // the union (TMA layout only; a tile whose list then turns out invalid drains its copy).
+  const bool q_early0 = !gather && !bad0 && cnt0 > 0, q_early1 = !gather && !bad1 && cnt1 > 0;
+  if (tid == 0 && !gather) {
+    mbar_init(bar(B_Q + 0), 1);
+    mbar_init(bar(B_Q + 1), 1);
+    mbar_init_fence();
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (!(t ? q_early1 : q_early0)) continue;
+      mbar_arrive_expect_tx(bar(B_Q + t), C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::QK_PANELS; ++c)
+        tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * C::QK_PANEL,
+                    (t ? qb1 : qb0) * BN, bh);
+    }
+  }
   // Lists must be strictly ascending block indices in [0, nb_head).
   if (!bad0)
     for (int j = tid; j < cnt0; j += nthr) {
@@ -200,7 +217,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   bad0 = __syncthreads_or(bad0);
   bad1 = __syncthreads_or(bad1);
   if (bad0 || bad1) {
-    if (tid == 0) atomicOr(a.err, kDevErrKvRange);
+    if (tid == 0) {
+      atomicOr(a.err, kDevErrKvRange);
+      if (bad0 && q_early0) mbar_wait_drain(bar(B_Q + 0), 0, a.err);  // the copy lands before the tile is dropped
+      if (bad1 && q_early1) mbar_wait_drain(bar(B_Q + 1), 0, a.err);
+    }
     if (bad0) {
       cnt0 = 0;
       for (int x = tid; x < nwords; x += nthr) bits0[x] = 0u;
@@ -280,7 +301,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (tid == 0) {
     const uint32_t nload = gather ? 32u : 1u;  // gather: one cp.async arrival per producer lane
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(B_Q + t), nload);
+      if (gather) mbar_init(bar(B_Q + t), nload);  // TMA layout: initialised above, copy in flight
       mbar_init(bar(B_S_FULL + t), 1);
       mbar_init(bar(B_P_FULL + t), 128);
       mbar_init(bar(B_O_FINAL + t), 1);
@@ -376,16 +397,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == kWarpLoad) {
     // ================= TMA producer =================
     if (lane == 0 && U > 0) {
-      int nk = 0, nv = 0;  // copies issued
+      int nk = 0, nv = 0;  // copies issued (the Q tiles were issued in the prologue)
       const int cnts[2] = {cnt0, cnt1};
-      for (int t = 0; t < 2; ++t) {
-        if (cnts[t] == 0) continue;
-        mbar_arrive_expect_tx(bar(B_Q + t), C::Q_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::QK_PANELS; ++c)
-          tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * kBM * 128, tq, bar(B_Q + t), c * C::QK_PANEL,
-                      (t ? qb1 : qb0) * BN, bh);
-      }
       for (int n = 0; n < U; ++n) {
         const int st = n % C::NS;
         const uint32_t u = n / C::NS;
