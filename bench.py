@@ -37,7 +37,7 @@ import synthetic  # noqa: E402
 METRIC = "ms/attention call and effective TFLOP/s (sparse & dense-equiv) vs bf16 peak"
 # DRAM bytes (read + write) per launch of the attention kernel from one ncu capture of the current
 # kernel on that workload (profiles/ has the command and the figures); absent -> null.
-TRAFFIC = {"hunyuanvideo-720p: B1 H24 33x45x80 d128 block128 bf16": 2216507392 + 711775232}
+TRAFFIC = {"hunyuanvideo-720p: B1 H24 33x45x80 d128 block128 bf16": 2217364736 + 712276736}
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
